@@ -1,0 +1,193 @@
+"""Pins for the oracle's decode attention, precision tail and GQA.
+
+Forum thread on KV compression, attention paragraph: dot the query with every
+prior key, softmax, weighted average of the values.  BeeLlama v0.4.0 news,
+section KV cache 精度尾部: the newest N tokens stay in F16, the rest quantized.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q4_1, Q2_1, RANK
+from oracle import ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION
+from quantized_kv_cache_15_b200 import workloads as W
+
+SCALE = float(np.float32(1.0 / np.sqrt(128.0)))
+
+
+def test_four_token_brute_force_golden():
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "attention_4token.json")))
+    n = g["n"]
+    q = np.zeros(128); q[0] = 1.0
+    K = np.zeros((n, 128))
+    K[:, 0] = np.sqrt(128.0) * np.log(np.array(g["score_ln_args"], dtype=np.float64))
+    V = np.zeros((n, 128))
+    for i, vals in g["values_nonzero"].items():
+        V[int(i), g["value_channels"]] = vals
+    out = oracle.attention(q, K, V, 1.0 / np.sqrt(128.0))
+    for ci, (num, den) in g["expected_output_fraction"].items():
+        assert abs(out[g["value_channels"][int(ci)]] - num / den) < 1e-12
+    mask = np.ones(128, bool); mask[g["value_channels"]] = False
+    assert np.abs(out[mask]).max() == 0.0
+
+
+def test_equal_keys_give_mean_of_values():
+    rng = np.random.default_rng(1)
+    k = rng.standard_normal(128)
+    K = np.tile(k, (37, 1))
+    V = rng.standard_normal((37, 128))
+    out = oracle.attention(rng.standard_normal(128), K, V, SCALE)
+    assert np.allclose(out, V.mean(axis=0), rtol=0, atol=1e-13)
+
+
+def test_dominant_key_selects_its_value():
+    rng = np.random.default_rng(2)
+    q = np.zeros(128); q[3] = 1.0
+    K = rng.standard_normal((50, 128)) * 0.1
+    K[17, 3] = 60.0 / SCALE                                  # score gap > 50
+    V = rng.standard_normal((50, 128))
+    out = oracle.attention(q, K, V, SCALE)
+    assert np.allclose(out, V[17], rtol=0, atol=1e-18)
+
+
+def test_score_shift_invariance_and_permutation():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal(128)
+    K = rng.standard_normal((64, 128))
+    V = rng.standard_normal((64, 128))
+    base = oracle.attention(q, K, V, SCALE)
+    shift = 7.5 * q / (q @ q) / SCALE                       # adds 7.5 to every score
+    assert np.allclose(oracle.attention(q, K + shift, V, SCALE), base, atol=1e-12)
+    p = rng.permutation(64)
+    assert np.allclose(oracle.attention(q, K[p], V[p], SCALE), base, atol=1e-13)
+
+
+def _hist(seed, n, G=4):
+    rng = np.random.default_rng(seed)
+    K = (rng.standard_normal((n, 128)) * 2).astype(np.float16).view(np.uint16)
+    V = rng.standard_normal((n, 128)).astype(np.float16).view(np.uint16)
+    q = rng.standard_normal((G, 128)).astype(np.float16).view(np.uint16)
+    return K, V, q
+
+
+def test_tail_covering_context_is_bitwise_plain_f16():
+    """A precision tail that covers the whole context reproduces F16 attention
+    bit for bit (same code path)."""
+    K, V, q = _hist(4, 300)
+    plain = oracle.decode_head(K, V, q, F16, F16, ROT_NONE, tail=0)
+    for tail in (300, 512, 1024):
+        t = oracle.decode_head(K, V, q, Q2_0, Q2_0, ROT_HADAMARD, tail=tail)
+        assert np.array_equal(t.view(np.uint32), plain.view(np.uint32))
+    # and plain F16 attention equals the dense formula on the raw fp16 values
+    Kd = oracle.f16_to_f32(K).astype(np.float64)
+    Vd = oracle.f16_to_f32(V).astype(np.float64)
+    for g in range(q.shape[0]):
+        ref = oracle.attention(oracle.f16_to_f32(q[g]).astype(np.float64), Kd, Vd, SCALE)
+        assert np.array_equal(plain[g], ref.astype(np.float32))
+
+
+def test_partial_tail_splits_history():
+    """With a tail of T rows, exactly the newest T rows stay raw: the result equals
+    attention over (dequantized old rows + raw newest rows)."""
+    K, V, q = _hist(5, 400)
+    T = 128
+    out = oracle.decode_head(K, V, q, Q4_0, Q4_1, ROT_HADAMARD, tail=T)
+    ck, sk = oracle.encode_rows(Q4_0, ROT_HADAMARD, K[:-T])
+    cv, sv = oracle.encode_rows(Q4_1, ROT_HADAMARD, V[:-T])
+    Kd = np.concatenate([oracle.decode_rows_original(Q4_0, ROT_HADAMARD, ck, sk),
+                         oracle.f16_to_f32(K[-T:]).astype(np.float64)])
+    Vd = np.concatenate([oracle.decode_rows_original(Q4_1, ROT_HADAMARD, cv, sv),
+                         oracle.f16_to_f32(V[-T:]).astype(np.float64)])
+    for g in range(q.shape[0]):
+        ref = oracle.attention(oracle.f16_to_f32(q[g]).astype(np.float64), Kd, Vd, SCALE)
+        assert np.array_equal(out[g], ref.astype(np.float32))
+
+
+def test_gqa_heads_are_independent_single_head_attention():
+    K, V, q = _hist(6, 200, G=6)
+    out = oracle.decode_head(K, V, q, Q8_0, Q6_0, ROT_HADAMARD)
+    for g in range(6):
+        one = oracle.decode_head(K, V, q[g:g + 1], Q8_0, Q6_0, ROT_HADAMARD)
+        assert np.array_equal(out[g], one[0])
+
+
+@pytest.mark.parametrize("codec", [Q8_0, Q4_0, Q2_0, Q4_1, Q2_1])
+def test_hadamard_dequant_in_original_basis_matches_inverse_transform(codec):
+    """Dequantizing a rotated row and rotating back recovers the row within the
+    quantizer bound: the rotation is orthogonal, so the original-basis error norm
+    is at most sqrt(32 * sum_b (d_b / 2)^2) (plus fp32 rounding of the rotation)."""
+    K, _, _ = _hist(7, 64)
+    ck, sk = oracle.encode_rows(codec, ROT_HADAMARD, K)
+    back = oracle.decode_rows_original(codec, ROT_HADAMARD, ck, sk)
+    x = oracle.f16_to_f32(K).astype(np.float64)
+    d = oracle.f16_to_f32(sk).astype(np.float64)
+    if codec in (Q4_1, Q2_1):
+        d = d[:, 0::2]
+    bound = np.sqrt(32.0 * np.square(d / 2.0).sum(axis=1)) + 1e-5 * np.linalg.norm(x, axis=1)
+    assert (np.linalg.norm(back - x, axis=1) <= bound).all()
+
+
+def test_varnorm_roundtrip_divides_by_inv_rms():
+    w = W.make_workload(5, "small")
+    calib = w.calib_rows("K", 0, 512)[:, 0, :].numpy().view(np.uint16)
+    inv = oracle.varnorm_inv_rms(calib)
+    K = w.rows("K", 0, 0, 0, 64)[:, 0, :].numpy().view(np.uint16)
+    ck, sk = oracle.encode_rows(Q8_0, ROT_VARNORM_HADAMARD, K, inv_s=inv)
+    back = oracle.decode_rows_original(Q8_0, ROT_VARNORM_HADAMARD, ck, sk, inv_s=inv)
+    x = oracle.f16_to_f32(K).astype(np.float64)
+    # error norm in the normalised basis is bounded by the quantizer; dividing by
+    # inv_s stretches it by at most max(1/inv_s)
+    d = oracle.f16_to_f32(sk).astype(np.float64)
+    bound = np.sqrt(32.0 * np.square(d / 2.0).sum(axis=1)) * (1.0 / inv.astype(np.float64)).max()
+    assert (np.linalg.norm(back - x, axis=1) <= bound * (1 + 1e-5)).all()
+
+
+def test_projection_full_rank_identity_basis_matches_hadamard_path():
+    """P = I with r = 128: the projected path stores the Hadamard-rotated row; its
+    attention output matches the Hadamard path within rounding of the rotation."""
+    K, V, q = _hist(8, 256)
+    M = oracle.fuse_projection(np.eye(128))
+    zk = oracle.to_stored_basis(RANK, ROT_PROJECTION, K, M=M, r=128)
+    yk = oracle.to_stored_basis(Q4_0, ROT_HADAMARD, K)
+    assert np.abs(zk - yk).max() <= 1e-6 * np.abs(yk).max()
+    # decoding projected codes (M^T zhat) equals rotating the same dequantized
+    # values back with the dense Hadamard rotation
+    codes, scales = oracle.quantize_rows(RANK, zk, r=128, b=4)
+    back_proj = oracle.decode_rows_original(RANK, ROT_PROJECTION, codes, scales, M=M, r=128, b=4)
+    zhat = oracle.dequantize_rows(RANK, codes, scales, r=128, b=4).astype(np.float64)
+    back_h = oracle.rotate_dense(zhat)
+    assert np.abs(back_proj - back_h).max() <= 1e-6 * np.abs(back_h).max()
+
+
+@pytest.mark.slow
+def test_quality_orderings_synthetic_analogue():
+    """Synthetic analogues of the KLD table's orderings (BeeLlama v0.4.0 news,
+    KLD 基准 table): error falls as bits rise; a 1024-token F16 tail beats no tail
+    at low bits; variance-normalised + rotated 4-bit beats plain (unrotated) q4_0
+    on keys with outlier channels.  Metric: relative L2 error of the attention
+    output against exact F16 attention, over config-1-shaped data.  Not parity."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "kld_table.json")))["rows"]
+    assert g["q2_0"][1] < g["q2_0"][0] and g["kvarn4"][0] < g["q4_0"][0]
+    assert g["q8_0"][0] < g["q6_0"][0] < g["q4_0"][0] < g["q3_0"][0] < g["q2_0"][0]
+    w = W.make_workload(1, "full")
+    T = 4096
+    K = w.rows("K", 0, 0, 0, T)[:, 0, :].numpy().view(np.uint16)
+    V = w.rows("V", 0, 0, 0, T)[:, 0, :].numpy().view(np.uint16)
+    qs = np.stack([w.queries(0, 0, s)[:4].numpy().view(np.uint16) for s in range(4)]).reshape(-1, 128)
+    exact = oracle.decode_head(K, V, qs, F16, F16, ROT_NONE)
+
+    def err(kc, vc, rot, tail=0, inv=None):
+        o = oracle.decode_head(K, V, qs, kc, vc, rot, tail=tail, inv_s_k=inv, inv_s_v=inv)
+        return np.linalg.norm(o - exact) / np.linalg.norm(exact)
+
+    e = {c: err(c, c, ROT_HADAMARD) for c in (Q8_0, Q6_0, Q4_0, Q3_0, Q2_0)}
+    assert e[Q8_0] < e[Q6_0] < e[Q4_0] < e[Q3_0] < e[Q2_0]
+    assert err(Q2_0, Q2_0, ROT_HADAMARD, tail=1024) < e[Q2_0]
+    invk = oracle.varnorm_inv_rms(w.rows("K", 0, 7, 0, 512)[:, 0, :].numpy().view(np.uint16))
+    o_kvarn = oracle.decode_head(K, V, qs, Q4_0, Q4_0, ROT_VARNORM_HADAMARD, inv_s_k=invk,
+                                 inv_s_v=np.ones(128, np.float32))
+    e_kvarn = np.linalg.norm(o_kvarn - exact) / np.linalg.norm(exact)
+    assert e_kvarn < err(Q4_0, Q4_0, ROT_NONE)
