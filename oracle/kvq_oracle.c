@@ -231,9 +231,23 @@ static void quant_block_sym(const float* x, int n, int bits, uint8_t* u, uint16_
 
 /* R5: asymmetric block quantizer ("_1"): m = fp16 round-down of the block
  * minimum, d = (max - m)/(2^b - 1) stored fp16 RNE, u = clamp(RNE((x-m)/d)). */
+/* Block minimum / maximum with IEEE-754 minimum / maximum semantics for signed
+ * zeros (-0 < +0), so the result does not depend on the order of the values. */
+static float block_minimum(const float* x, int n) {
+    float mn = x[0];
+    for (int j = 1; j < n; ++j)
+        if (x[j] < mn || (x[j] == 0.0f && mn == 0.0f && signbit(x[j]))) mn = x[j];
+    return mn;
+}
+static float block_maximum(const float* x, int n) {
+    float mx = x[0];
+    for (int j = 1; j < n; ++j)
+        if (x[j] > mx || (x[j] == 0.0f && mx == 0.0f && !signbit(x[j]))) mx = x[j];
+    return mx;
+}
+
 static void quant_block_asym(const float* x, int n, int bits, uint8_t* u, uint16_t* dh_out, uint16_t* mh_out) {
-    float mn = x[0], mx = x[0];
-    for (int j = 1; j < n; ++j) { if (x[j] < mn) mn = x[j]; if (x[j] > mx) mx = x[j]; }
+    float mn = block_minimum(x, n), mx = block_maximum(x, n);
     if (mn < -65504.0f) mn = -65504.0f;
     if (mn > 65504.0f) mn = 65504.0f;
     uint16_t mh = orc_f16_rd(mn);

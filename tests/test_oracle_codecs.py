@@ -218,3 +218,24 @@ def test_f16_codec_is_identity_on_fp16_values():
     codes, scales = oracle.quantize_rows(F16, x)
     assert np.array_equal(codes.view(np.uint16), x.astype(np.float16).view(np.uint16))
     assert np.array_equal(oracle.dequantize_rows(F16, codes, scales), x)
+
+
+@pytest.mark.parametrize("codec", ASYM)
+def test_asymmetric_scale_is_order_independent_with_signed_zeros(codec):
+    """R5: the block minimum and maximum follow IEEE-754 minimum/maximum (-0 < +0),
+    so permuting a block never changes the stored scale or minimum bits: a block
+    whose smallest value is zero stores m = -0 (0x8000) exactly when it holds a -0."""
+    rng = np.random.default_rng(300 + codec)
+    for trial in range(60):
+        x = np.zeros(32, np.float32)
+        x[rng.integers(0, 32, 5)] = rng.uniform(0.5, 3, 5).astype(np.float32)
+        has_neg_zero = trial % 2 == 0
+        if has_neg_zero:
+            x[rng.integers(0, 32, 3)] = np.float32(-0.0)
+        row = np.tile(x, 4)
+        ref = oracle.quantize_rows(codec, row)[1]
+        expect_m = 0x8000 if (np.signbit(x) & (x == 0)).any() else 0x0000
+        assert ref[0, 1] == expect_m
+        for _ in range(4):
+            perm = np.concatenate([rng.permutation(32) + 32 * b for b in range(4)])
+            assert np.array_equal(oracle.quantize_rows(codec, row[perm])[1], ref)
