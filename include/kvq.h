@@ -1,0 +1,229 @@
+/*
+ * kvq.h -- C ABI of the B200 quantized KV cache: append-quantize and decode
+ * attention over packed q8/q6/q4/q3/q2 (_0 and _1), F16 and per-head rank/bit
+ * codecs, with a Hadamard rotation (optionally variance-normalised, or fused
+ * into a per-head projection), an F16 precision tail for the newest tokens, a
+ * per-layer / per-head codec map and grouped-query decode attention.
+ *
+ * Sources (web pages, cited by title and section):
+ *  - "BeeLlama.cpp v0.4.0 发布：聚焦 KV cache 量化，新增 KVarN 与精度尾部机制":
+ *    §核心新特性：KVarN (variance-normalised quantization), §KV cache 精度尾部
+ *    (newest tokens kept in F16), §新增标准 KV cache 类型 (q6_0/q6_1,
+ *    q3_0/q3_1, q2_0/q2_1 next to q8_0 and q5/q4).
+ *  - "KV-COBRA splits the KV-cache budget per head -- Rank vs bit-width
+ *    allocation": §Jargon (Hadamard rotation, scalar quantization to 2^b
+ *    levels, rank / low-rank projection), §The news (per-head rank and bits,
+ *    rotation fused into the projection matrix, frozen per-head settings at
+ *    inference).
+ *  - "Introducing a new KV format: VBR (Variable Bit Rate)": per-layer codec
+ *    mixes and asymmetric K/V codecs.
+ *  - Forum thread on KV compression (swe-vps, maurelius2): decode attention is
+ *    a dot product of the query with every prior key, a softmax and a weighted
+ *    average of the values; decode is bound by memory bandwidth.
+ *
+ * Conventions (every entry point):
+ *  - Pointers marked "device" are CUDA device pointers on the plan's device;
+ *    pointers marked "host" are ordinary host memory read before the call
+ *    returns.  The caller owns every buffer it passes (cache, inputs, outputs,
+ *    workspace).  A plan owns only its own copies of the host tables it was
+ *    given (small device allocations) and host bookkeeping.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously on it; argument errors are reported synchronously,
+ *    before anything is enqueued, and leave the plan unchanged.
+ *  - Errors never throw across the ABI.  Every call returns a kvq_status;
+ *    kvq_last_error() gives a thread-local message for the last failure.
+ *    Conditions that only a kernel can see (a missing page, an exhausted wait)
+ *    are latched in the plan's device error word and reported by
+ *    kvq_check_device_error().
+ *  - head_dim is 128.  Positions, lengths and capacities count tokens.
+ *  - A plan is not thread-safe; calls on one plan must be serialised.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_HEAD_DIM 128
+#define KVQ_PAGE_TOKENS 64      /* tokens per cache page */
+#define KVQ_MAX_KV_HEADS 32
+#define KVQ_MAX_GQA 8           /* query heads per kv head */
+#define KVQ_MAX_BATCH 256       /* sequences per decode / append call */
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size, layer or sequence out of range */
+  KVQ_ERR_UNSUPPORTED = 2,   /* codec, rank/bits, head_dim or GQA ratio this build does not handle */
+  KVQ_ERR_CAPACITY = 3,      /* sequence longer than max_tokens_per_seq, or the page pool is exhausted */
+  KVQ_ERR_OOM = 4,           /* a plan-owned device allocation failed */
+  KVQ_ERR_CUDA = 5,          /* a CUDA runtime call or a launch failed */
+  KVQ_ERR_DEVICE = 6,        /* a kernel latched an error (see kvq_check_device_error) */
+  KVQ_ERR_TIMEOUT = 7,       /* a bounded wait inside a kernel ran out */
+  KVQ_ERR_STATE = 8          /* call out of order (e.g. no cache bound) */
+} kvq_status;
+
+/* Codecs.  Block = 32 consecutive values of a row in the stored basis.
+ *  _0 (symmetric): d = max|x| / (2^(b-1) - 1) stored fp16 (round to nearest
+ *     even); codes round-half-even(x / d) clamped to [-2^(b-1), 2^(b-1) - 1]
+ *     (the tiny workload's q4_0: d = max|x|/7, codes in [-8, 7]).
+ *  _1 (scale + minimum): m = fp16 round-down of the block minimum,
+ *     d = (max - m) / (2^b - 1) fp16; codes round-half-even((x - m)/d) in
+ *     [0, 2^b - 1].
+ *  KVQ_RANK: the KV-COBRA per-head path: the row is projected to r
+ *     coordinates (rotation fused into the projection) and each block of
+ *     min(32, r) coordinates is quantized mid-rise with all 2^b levels
+ *     (levels (k + 1/2) d, d = max|z| / (2^(b-1) - 1/2)); r and b per head.
+ *  KVQ_F16: raw fp16 rows (unrotated).
+ * Codes are stored offset-binary (u = code + 2^(b-1) for _0).  Byte layouts
+ * are given in the repository's design document. */
+typedef enum {
+  KVQ_F16 = 0, KVQ_Q8_0 = 1, KVQ_Q6_0 = 2, KVQ_Q4_0 = 3, KVQ_Q3_0 = 4, KVQ_Q2_0 = 5,
+  KVQ_Q8_1 = 6, KVQ_Q6_1 = 7, KVQ_Q4_1 = 8, KVQ_Q3_1 = 9, KVQ_Q2_1 = 10, KVQ_RANK = 11
+} kvq_codec;
+
+/* Transform applied to rows before quantization (F16 rows are never
+ * transformed).  HADAMARD: y = H x / sqrt(128) (Sylvester H, computed as the
+ * staged fast transform in fp32).  VARNORM_HADAMARD: y = H (x * inv_rms) /
+ * sqrt(128) with a per-(layer, kv-head, K|V, channel) inverse RMS from a
+ * calibration prefix (KVarN).  PROJECTION: z = M_h x with M_h = R_r P_h^T,
+ * P_h the head's 128 x r orthonormal basis and R_r the order-r rotation
+ * (codec must be KVQ_RANK or KVQ_F16). */
+typedef enum {
+  KVQ_ROT_NONE = 0, KVQ_ROT_HADAMARD = 1, KVQ_ROT_VARNORM_HADAMARD = 2, KVQ_ROT_PROJECTION = 3
+} kvq_rot;
+
+typedef struct kvq_plan kvq_plan;
+
+typedef struct {
+  int n_layers;                 /* >= 1 */
+  int n_q_heads;                /* query heads per layer */
+  int n_kv_heads;               /* kv heads per layer (<= KVQ_MAX_KV_HEADS); n_q_heads / n_kv_heads <= KVQ_MAX_GQA */
+  int head_dim;                 /* must be 128 */
+  int max_seqs;                 /* sequence ids are 0 .. max_seqs-1 */
+  int64_t max_tokens_per_seq;   /* capacity of one sequence (every layer) */
+  int64_t max_pages;            /* pages in the pool (each page: 64 tokens x all kv heads of a layer, in
+                                   every layer); 0 = max_seqs * ceil(max_tokens_per_seq / 64) */
+  int tail_tokens;              /* F16 precision tail length per (seq, layer, kv-head); 0 or a multiple of 64 */
+  const int* k_codec;           /* host [n_layers][n_kv_heads] kvq_codec of K */
+  const int* v_codec;           /* host [n_layers][n_kv_heads] kvq_codec of V */
+  int rot;                      /* kvq_rot */
+  const float* inv_rms;         /* host [n_layers][n_kv_heads][2 (K,V)][128], VARNORM_HADAMARD only, else NULL */
+  const int* rank;              /* host [n_layers][n_kv_heads] r in {16,32,64,96,128}, PROJECTION only */
+  const int* k_bits;            /* host [n_layers][n_kv_heads] b in {1,2,3,4} for K, PROJECTION only */
+  const int* v_bits;            /* host [n_layers][n_kv_heads] b in {1,2,3,4} for V, PROJECTION only */
+  const double* proj_basis;     /* host, PROJECTION only: for each (layer, head) in order, P_h as a
+                                   row-major [128][r] matrix with orthonormal columns; concatenated */
+  float softmax_scale;          /* 0 => 1/sqrt(128) */
+} kvq_plan_desc;
+
+/* Create a plan on the current CUDA device: validates the descriptor, lays out
+ * the paged cache, copies the host tables (and fuses the rotation into the
+ * projections: M_h = R_r P_h^T) into plan-owned device memory.
+ * [KV-COBRA explainer, §The news: frozen per-head settings, rotation fused]. */
+kvq_status kvq_plan_create(const kvq_plan_desc* desc, kvq_plan** out);
+void kvq_plan_destroy(kvq_plan* plan);
+
+/* Bytes of device memory the caller must allocate for the cache. */
+kvq_status kvq_plan_cache_bytes(const kvq_plan* plan, size_t* bytes);
+
+/* Bytes of device workspace kvq_decode_attention needs for n_seqs sequences.
+ * The workspace must be zero-filled once before its first use; every call
+ * leaves its counters back at zero. */
+kvq_status kvq_plan_workspace_bytes(const kvq_plan* plan, int n_seqs, size_t* bytes);
+
+/* Attach caller-owned device memory of at least kvq_plan_cache_bytes(), 256-byte
+ * aligned.  Its contents need not be initialised.  Resets every sequence. */
+kvq_status kvq_cache_bind(kvq_plan* plan, void* dev_cache, size_t bytes);
+
+/* Append n_new[i] new tokens to sequence seq_ids[i] in one layer
+ * [BeeLlama v0.4.0 news §KV cache 精度尾部 and §KVarN; KV-COBRA §The news].
+ *  k_new, v_new: device fp16 [sum(n_new)][n_kv_heads][128], the sequences'
+ *  rows concatenated in call order.
+ * New rows enter the layer's F16 tail; rows pushed out of the tail (or every
+ * row, when tail_tokens = 0) are transformed and quantized into the paged
+ * cache.  seq_ids must be distinct.  Lengths advance at enqueue time (per
+ * sequence and layer).  KVQ_ERR_CAPACITY if a sequence would exceed
+ * max_tokens_per_seq or the page pool runs out (nothing is enqueued then). */
+kvq_status kvq_append_quantize(kvq_plan* plan, int layer, int n_seqs, const int* seq_ids /*host*/,
+                               const int* n_new /*host*/, const void* k_new, const void* v_new, void* stream);
+
+/* Decode attention for one new query token per sequence
+ * [forum thread on KV compression: dot, softmax, weighted average of values].
+ *  q:   device fp16 [n_seqs][n_q_heads][128]
+ *  out: device fp32 [n_seqs][n_q_heads][128]
+ *  workspace: device, kvq_plan_workspace_bytes(plan, n_seqs), zeroed before first use.
+ * Query head h attends with kv head h / (n_q_heads / n_kv_heads) over every
+ * cached token of the sequence in this layer (quantized rows dequantized in
+ * registers, tail rows in F16).  Split-K over pages; partial softmax states
+ * are merged in a fixed order (deterministic). */
+kvq_status kvq_decode_attention(kvq_plan* plan, int layer, int n_seqs, const int* seq_ids /*host*/,
+                                const void* q, float* out, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Reconstruct cached rows t0 .. t1-1 of one sequence and layer in the ORIGINAL
+ * basis (inverse rotation / projection applied; tail rows copied).
+ *  k_out, v_out: device fp32 [t1-t0][n_kv_heads][128] (either may be NULL). */
+kvq_status kvq_dequantize(const kvq_plan* plan, int layer, int seq_id, int64_t t0, int64_t t1,
+                          float* k_out, float* v_out, void* stream);
+
+/* Packed row sizes of one (layer, kv head, K=0|V=1): code bytes and scale bytes
+ * of one canonical row (F16: 256 and 0). */
+kvq_status kvq_row_bytes(const kvq_plan* plan, int layer, int head, int kv, int* code_bytes,
+                         int* scale_bytes);
+
+/* Copy quantized rows t0 .. t1-1 (all below the tail) of one sequence, layer and
+ * K|V out of the paged cache into canonical packed rows, head after head:
+ * head h's rows start at sum_{h'<h} (t1-t0) * code_bytes(h') in codes_out and
+ * likewise in scales_out.  Device buffers. */
+kvq_status kvq_read_rows(const kvq_plan* plan, int layer, int seq_id, int64_t t0, int64_t t1, int kv,
+                         void* codes_out, void* scales_out, void* stream);
+
+/* Host mirror of a sequence's length in one layer. */
+kvq_status kvq_seq_length(const kvq_plan* plan, int seq_id, int layer, int64_t* len);
+
+/* Forget a sequence (all layers) and return its pages to the pool. */
+kvq_status kvq_seq_reset(kvq_plan* plan, int seq_id);
+
+/* Per-channel inverse RMS of a calibration prefix [BeeLlama v0.4.0 news
+ * §KVarN: variance normalisation]: inv_rms[c] = fp32(1 / sqrt(mean_t x[t][c]^2))
+ * with the sum taken in double in token order (1 where the RMS is < 1e-6).
+ *  x: device fp16 [n_tokens][row_stride] (channels 0 .. n_channels-1 used)
+ *  inv_rms: device fp32 [n_channels] */
+kvq_status kvq_calibrate_varnorm(int64_t n_tokens, int n_channels, int64_t row_stride, const void* x,
+                                 float* inv_rms, void* stream);
+
+/* Synchronise `stream`, read and clear the plan's device error word. */
+kvq_status kvq_check_device_error(kvq_plan* plan, void* stream);
+
+/* Thread-local description of the last failure ("" if none). */
+const char* kvq_last_error(void);
+
+/* Total number of CUDA kernels this library has launched in the process
+ * (every entry point that enqueues work adds its launches). */
+kvq_status kvq_launch_count(uint64_t* count);
+
+/* --- inspection entry points (used by the parity tests) ------------------ */
+
+/* Rows in the stored basis, fp32, exactly as the append path computes them
+ * before quantization: the staged Hadamard transform (after variance
+ * normalisation) for rotated codecs, z = M_h x on the tensor cores for the
+ * projection path, the raw values for F16.
+ *  x: device fp16 [n][128];  y: device fp32 [n][128] (or [n][r]). */
+kvq_status kvq_debug_rotate(const kvq_plan* plan, int layer, int head, int kv, int n, const void* x,
+                            float* y, void* stream);
+
+/* The block quantizer alone: fp32 rows in the stored basis -> canonical packed
+ * rows.  codec: kvq_codec; r, b: rank and bits (KVQ_RANK only, else ignored).
+ *  y: device fp32 [n_rows][128 or r]; codes: device [n_rows][code_bytes];
+ *  scales: device [n_rows][scale_bytes]. */
+kvq_status kvq_debug_quantize_f32(int codec, int r, int b, int n_rows, const float* y, void* codes,
+                                  void* scales, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H_ */

@@ -1,0 +1,594 @@
+// Host side of the kvq C ABI: plan creation and validation, the paged cache
+// layout, page allocation, split-K sizing and the launches.  Everything that
+// touches data runs in the CUDA kernels of this directory; this file only moves
+// host bookkeeping and enqueues work on the caller's stream.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "kvq_internal.h"
+
+using namespace kvq;
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<unsigned long long> g_launches{0};
+
+kvq_status fail(kvq_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+kvq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool valid_codec(int c) { return c >= KVQ_F16 && c <= KVQ_RANK; }
+bool valid_rank(int r) { return r == 16 || r == 32 || r == 64 || r == 96 || r == 128; }
+
+// In-place Sylvester Walsh-Hadamard transform of length n (power of two), double.
+void wht_inplace(double* v, int n) {
+  for (int h = 1; h < n; h <<= 1)
+    for (int i = 0; i < n; ++i)
+      if ((i & h) == 0) {
+        double a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+}
+
+}  // namespace
+
+void kvq::note_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+struct kvq_plan {
+  int device = 0;
+  int num_sms = 148;
+  int L = 0, Hq = 0, Hkv = 0, G = 0, T = 0, max_seqs = 0;
+  int64_t max_tokens = 0;
+  int mpps = 0;            // max pages per sequence
+  int64_t n_pages = 0;
+  int rot = 0;
+  float scale = 0.f;
+  std::vector<HeadInfo> heads;        // [L][Hkv]
+  std::vector<uint64_t> layer_off;    // [L]
+  std::vector<uint32_t> page_bytes;   // [L]
+  std::vector<int> stage_bytes;       // [L] max region (and tail page) bytes
+  uint64_t tail_off = 0, cache_bytes = 0;
+  uint8_t* cache = nullptr;
+  float* d_inv = nullptr;   // [L][Hkv][2][128] inverse RMS (append)
+  float* d_sk = nullptr;    // [L][Hkv][128] 1/inv_rms of K (decode, dequantize)
+  float* d_sv = nullptr;    // [L][Hkv][128] 1/inv_rms of V
+  float* d_M = nullptr;     // fused projections
+  int* d_bt = nullptr;      // block table [max_seqs][mpps]
+  int* d_err = nullptr;
+  std::vector<int64_t> len;           // [max_seqs][L]
+  std::vector<int> bt;                // host mirror of the block table
+  std::vector<int> npages;            // pages held per sequence
+  std::vector<int> free_pages;        // stack of free page ids
+
+  ~kvq_plan() {
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(device);
+    cudaFree(d_inv); cudaFree(d_sk); cudaFree(d_sv); cudaFree(d_M); cudaFree(d_bt); cudaFree(d_err);
+    cudaSetDevice(prev);
+  }
+
+  const HeadInfo& head(int l, int h) const { return heads[(size_t)l * Hkv + h]; }
+
+  void reset_all() {
+    std::fill(len.begin(), len.end(), 0);
+    std::fill(bt.begin(), bt.end(), -1);
+    std::fill(npages.begin(), npages.end(), 0);
+    free_pages.clear();
+    for (int64_t i = n_pages - 1; i >= 0; --i) free_pages.push_back((int)i);
+  }
+
+  DecodeParams base_params(int layer) const {
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.pool = cache + layer_off[layer];
+    p.page_bytes = page_bytes[layer];
+    p.block_table = d_bt;
+    p.max_pages_per_seq = mpps;
+    p.tail = cache + tail_off;
+    p.T = T; p.L = L; p.layer = layer; p.Hkv = Hkv; p.Hq = Hq; p.G = G;
+    p.rot = rot;
+    p.s_k = (rot == KVQ_ROT_VARNORM_HADAMARD) ? d_sk + (size_t)layer * Hkv * D : nullptr;
+    p.s_v = (rot == KVQ_ROT_VARNORM_HADAMARD) ? d_sv + (size_t)layer * Hkv * D : nullptr;
+    p.M = d_M;
+    p.qscale = scale * 1.4426950408889634f;
+    p.err = d_err;
+    for (int h = 0; h < Hkv; ++h) p.heads[h] = head(layer, h);
+    return p;
+  }
+};
+
+extern "C" {
+
+const char* kvq_last_error(void) { return g_err.c_str(); }
+
+kvq_status kvq_launch_count(uint64_t* count) {
+  if (!count) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  *count = (uint64_t)g_launches.load(std::memory_order_relaxed);
+  return KVQ_OK;
+}
+
+kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
+  if (!d || !out) return fail(KVQ_ERR_INVALID_ARG, "null descriptor or output pointer");
+  *out = nullptr;
+  if (d->head_dim != D) return fail(KVQ_ERR_UNSUPPORTED, "head_dim must be 128 (got %d)", d->head_dim);
+  if (d->n_layers < 1 || d->n_kv_heads < 1 || d->n_q_heads < 1)
+    return fail(KVQ_ERR_INVALID_ARG, "n_layers, n_q_heads and n_kv_heads must be >= 1");
+  if (d->n_kv_heads > MAX_HKV) return fail(KVQ_ERR_UNSUPPORTED, "n_kv_heads > %d", MAX_HKV);
+  if (d->n_q_heads % d->n_kv_heads) return fail(KVQ_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  if (d->n_q_heads / d->n_kv_heads > MAX_G) return fail(KVQ_ERR_UNSUPPORTED, "GQA ratio above %d", MAX_G);
+  if (d->max_seqs < 1 || d->max_tokens_per_seq < 1) return fail(KVQ_ERR_INVALID_ARG, "max_seqs and max_tokens_per_seq must be >= 1");
+  if (d->max_tokens_per_seq > (int64_t)1 << 30) return fail(KVQ_ERR_UNSUPPORTED, "max_tokens_per_seq above 2^30");
+  if (d->tail_tokens < 0 || d->tail_tokens % PAGE) return fail(KVQ_ERR_INVALID_ARG, "tail_tokens must be 0 or a multiple of 64");
+  if (d->rot < KVQ_ROT_NONE || d->rot > KVQ_ROT_PROJECTION) return fail(KVQ_ERR_INVALID_ARG, "bad rot %d", d->rot);
+  if (!d->k_codec || !d->v_codec) return fail(KVQ_ERR_INVALID_ARG, "k_codec and v_codec tables are required");
+  if (d->rot == KVQ_ROT_VARNORM_HADAMARD && !d->inv_rms) return fail(KVQ_ERR_INVALID_ARG, "VARNORM_HADAMARD needs inv_rms");
+  if (d->rot == KVQ_ROT_PROJECTION && (!d->rank || !d->k_bits || !d->v_bits || !d->proj_basis))
+    return fail(KVQ_ERR_INVALID_ARG, "PROJECTION needs rank, k_bits, v_bits and proj_basis");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  kvq_plan* p = new kvq_plan();
+  p->device = dev;
+  cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  p->L = d->n_layers; p->Hq = d->n_q_heads; p->Hkv = d->n_kv_heads; p->G = p->Hq / p->Hkv;
+  p->T = d->tail_tokens; p->max_seqs = d->max_seqs; p->max_tokens = d->max_tokens_per_seq;
+  p->mpps = (int)((p->max_tokens + PAGE - 1) / PAGE);
+  p->n_pages = d->max_pages > 0 ? d->max_pages : (int64_t)p->max_seqs * p->mpps;
+  p->rot = d->rot;
+  p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / std::sqrt((double)D));
+
+  // per-head codec info and page layout
+  std::vector<float> Mhost;
+  const double* pb = d->proj_basis;
+  p->heads.resize((size_t)p->L * p->Hkv);
+  p->layer_off.resize(p->L);
+  p->page_bytes.resize(p->L);
+  p->stage_bytes.resize(p->L);
+  uint64_t off = 0;
+  for (int l = 0; l < p->L; ++l) {
+    uint32_t poff = 0;
+    int stage = 0;
+    for (int h = 0; h < p->Hkv; ++h) {
+      const size_t i = (size_t)l * p->Hkv + h;
+      HeadInfo hi;
+      std::memset(&hi, 0, sizeof(hi));
+      const int kc = d->k_codec[i], vc = d->v_codec[i];
+      if (!valid_codec(kc) || !valid_codec(vc)) { delete p; return fail(KVQ_ERR_UNSUPPORTED, "bad codec at layer %d head %d", l, h); }
+      const bool rank = (kc == KVQ_RANK || vc == KVQ_RANK);
+      if (rank != (d->rot == KVQ_ROT_PROJECTION) && !(d->rot == KVQ_ROT_PROJECTION && kc == KVQ_F16 && vc == KVQ_F16)) {
+        delete p;
+        return fail(KVQ_ERR_UNSUPPORTED, "KVQ_RANK codecs need rot = PROJECTION and vice versa (layer %d head %d)", l, h);
+      }
+      int r = D, kb = 0, vb = 0;
+      if (d->rot == KVQ_ROT_PROJECTION) {
+        r = d->rank[i]; kb = d->k_bits[i]; vb = d->v_bits[i];
+        if (!valid_rank(r) || kb < 1 || kb > 4 || vb < 1 || vb > 4) {
+          delete p;
+          return fail(KVQ_ERR_UNSUPPORTED, "rank must be 16/32/64/96/128 and bits 1..4 (layer %d head %d)", l, h);
+        }
+      }
+      hi.kcodec = (uint8_t)kc; hi.vcodec = (uint8_t)vc; hi.r = (uint8_t)r;
+      hi.kbits = (uint8_t)(kc == KVQ_RANK ? kb : codec_bits(kc));
+      hi.vbits = (uint8_t)(vc == KVQ_RANK ? vb : codec_bits(vc));
+      int cbK, sbK, cbV, sbV;
+      row_bytes(kc, r, kb, &cbK, &sbK);
+      row_bytes(vc, r, vb, &cbV, &sbV);
+      hi.cbK = (uint16_t)cbK; hi.sbK = (uint16_t)sbK; hi.cbV = (uint16_t)cbV; hi.sbV = (uint16_t)sbV;
+      hi.off = poff;
+      hi.bytes = (uint32_t)(PAGE * (cbK + sbK + cbV + sbV));
+      poff += hi.bytes;
+      stage = std::max(stage, (int)hi.bytes);
+      if (d->rot == KVQ_ROT_PROJECTION) {
+        // M_h = R_r P_h^T (R_r: Sylvester Hadamard / sqrt(r), block-diagonal H_32 for r = 96)
+        hi.m_off = (uint32_t)Mhost.size();
+        const int blk = (r == 96) ? 32 : r;
+        std::vector<double> col(r);
+        std::vector<float> M((size_t)r * D);
+        for (int c = 0; c < D; ++c) {
+          for (int k = 0; k < r; ++k) col[k] = pb[(size_t)c * r + k];
+          for (int b0 = 0; b0 < r; b0 += blk) wht_inplace(col.data() + b0, blk);
+          const double s = 1.0 / std::sqrt((double)blk);
+          for (int k = 0; k < r; ++k) M[(size_t)k * D + c] = (float)(col[k] * s);
+        }
+        Mhost.insert(Mhost.end(), M.begin(), M.end());
+        while (Mhost.size() % 4) Mhost.push_back(0.f);
+        pb += (size_t)D * r;
+      }
+      p->heads[i] = hi;
+    }
+    if (p->T > 0) stage = std::max(stage, TAIL_PAGE_BYTES);
+    p->stage_bytes[l] = (stage + 127) & ~127;
+    p->page_bytes[l] = poff;
+    p->layer_off[l] = off;
+    off += (uint64_t)poff * (uint64_t)p->n_pages;
+    off = (off + 255) & ~(uint64_t)255;
+  }
+  p->tail_off = off;
+  off += (uint64_t)p->max_seqs * p->L * p->Hkv * (uint64_t)p->T * (D * 2 * 2);
+  p->cache_bytes = off;
+
+  // device tables
+  auto dmalloc = [&](void** ptr, size_t bytes) -> bool {
+    if (std::getenv("KVQ_TEST_FAIL_ALLOC")) return false;
+    return cudaMalloc(ptr, bytes) == cudaSuccess;
+  };
+  if (!dmalloc((void**)&p->d_err, sizeof(int)) ||
+      !dmalloc((void**)&p->d_bt, sizeof(int) * (size_t)p->max_seqs * p->mpps)) {
+    delete p;
+    return fail(KVQ_ERR_OOM, "device allocation for the plan tables failed");
+  }
+  cudaMemset(p->d_err, 0, sizeof(int));
+  if (d->rot == KVQ_ROT_VARNORM_HADAMARD) {
+    const size_t n = (size_t)p->L * p->Hkv * 2 * D;
+    std::vector<float> sk((size_t)p->L * p->Hkv * D), sv((size_t)p->L * p->Hkv * D);
+    for (int l = 0; l < p->L; ++l)
+      for (int h = 0; h < p->Hkv; ++h)
+        for (int c = 0; c < D; ++c) {
+          const float ik = d->inv_rms[(((size_t)l * p->Hkv + h) * 2 + 0) * D + c];
+          const float iv = d->inv_rms[(((size_t)l * p->Hkv + h) * 2 + 1) * D + c];
+          if (!(ik > 0.f) || !(iv > 0.f) || !std::isfinite(ik) || !std::isfinite(iv)) {
+            delete p;
+            return fail(KVQ_ERR_INVALID_ARG, "inv_rms must be finite and positive");
+          }
+          sk[((size_t)l * p->Hkv + h) * D + c] = (float)(1.0 / (double)ik);
+          sv[((size_t)l * p->Hkv + h) * D + c] = (float)(1.0 / (double)iv);
+        }
+    if (!dmalloc((void**)&p->d_inv, n * 4) || !dmalloc((void**)&p->d_sk, sk.size() * 4) ||
+        !dmalloc((void**)&p->d_sv, sv.size() * 4)) {
+      delete p;
+      return fail(KVQ_ERR_OOM, "device allocation for the variance tables failed");
+    }
+    cudaMemcpy(p->d_inv, d->inv_rms, n * 4, cudaMemcpyHostToDevice);
+    cudaMemcpy(p->d_sk, sk.data(), sk.size() * 4, cudaMemcpyHostToDevice);
+    cudaMemcpy(p->d_sv, sv.data(), sv.size() * 4, cudaMemcpyHostToDevice);
+  }
+  if (!Mhost.empty()) {
+    if (!dmalloc((void**)&p->d_M, Mhost.size() * 4)) {
+      delete p;
+      return fail(KVQ_ERR_OOM, "device allocation for the projections failed");
+    }
+    cudaMemcpy(p->d_M, Mhost.data(), Mhost.size() * 4, cudaMemcpyHostToDevice);
+  }
+  p->len.assign((size_t)p->max_seqs * p->L, 0);
+  p->bt.assign((size_t)p->max_seqs * p->mpps, -1);
+  p->npages.assign(p->max_seqs, 0);
+  std::vector<int> neg(p->bt.size(), -1);
+  e = cudaMemcpy(p->d_bt, neg.data(), neg.size() * sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) { delete p; return cuda_fail(e, "block table init"); }
+  p->reset_all();
+  *out = p;
+  return KVQ_OK;
+}
+
+void kvq_plan_destroy(kvq_plan* plan) { delete plan; }
+
+kvq_status kvq_plan_cache_bytes(const kvq_plan* p, size_t* bytes) {
+  if (!p || !bytes) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  *bytes = (size_t)p->cache_bytes;
+  return KVQ_OK;
+}
+
+static size_t workspace_bytes(const kvq_plan* p, int n_seqs) {
+  return (size_t)n_seqs * p->Hkv * MAX_SPLITS * p->G * PARTIAL_FLOATS * sizeof(float) +
+         (size_t)n_seqs * p->Hkv * sizeof(int);
+}
+
+kvq_status kvq_plan_workspace_bytes(const kvq_plan* p, int n_seqs, size_t* bytes) {
+  if (!p || !bytes) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
+  *bytes = workspace_bytes(p, n_seqs);
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_bind(kvq_plan* p, void* dev, size_t bytes) {
+  if (!p || !dev) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if ((uintptr_t)dev % 256) return fail(KVQ_ERR_INVALID_ARG, "cache must be 256-byte aligned");
+  if (bytes < p->cache_bytes) return fail(KVQ_ERR_INVALID_ARG, "cache has %zu bytes, plan needs %llu", bytes,
+                                         (unsigned long long)p->cache_bytes);
+  p->cache = (uint8_t*)dev;
+  p->reset_all();
+  std::vector<int> neg(p->bt.size(), -1);
+  cudaError_t e = cudaMemcpy(p->d_bt, neg.data(), neg.size() * sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "block table reset");
+  return KVQ_OK;
+}
+
+kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* n_new,
+                               const void* k_new, const void* v_new, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
+  if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
+  if (n_seqs == 0) return KVQ_OK;
+  if (!seq_ids || !n_new) return fail(KVQ_ERR_INVALID_ARG, "null seq_ids or n_new");
+  int64_t total = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int s = seq_ids[i];
+    if (s < 0 || s >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d out of range", s);
+    for (int j = 0; j < i; ++j)
+      if (seq_ids[j] == s) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d repeated", s);
+    if (n_new[i] < 0) return fail(KVQ_ERR_INVALID_ARG, "negative n_new");
+    if (p->len[(size_t)s * p->L + layer] + n_new[i] > p->max_tokens)
+      return fail(KVQ_ERR_CAPACITY, "sequence %d would exceed max_tokens_per_seq", s);
+    total += n_new[i];
+  }
+  if (total == 0) return KVQ_OK;
+  if (!k_new || !v_new) return fail(KVQ_ERR_INVALID_ARG, "null k_new or v_new");
+  if (((uintptr_t)k_new | (uintptr_t)v_new) % 16) return fail(KVQ_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+  // pages: check capacity first, then allocate
+  int64_t need = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int s = seq_ids[i];
+    const int64_t nl = p->len[(size_t)s * p->L + layer] + n_new[i];
+    const int64_t nq = nl > p->T ? nl - p->T : 0;
+    const int pages = (int)((nq + PAGE - 1) / PAGE);
+    need += std::max(0, pages - p->npages[s]);
+  }
+  if (need > (int64_t)p->free_pages.size()) return fail(KVQ_ERR_CAPACITY, "page pool exhausted (%lld pages needed, %zu free)",
+                                                        (long long)need, p->free_pages.size());
+  cudaStream_t st = (cudaStream_t)stream;
+  std::vector<int> idx, val;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int s = seq_ids[i];
+    const int64_t nl = p->len[(size_t)s * p->L + layer] + n_new[i];
+    const int64_t nq = nl > p->T ? nl - p->T : 0;
+    const int pages = (int)((nq + PAGE - 1) / PAGE);
+    while (p->npages[s] < pages) {
+      const int pid = p->free_pages.back();
+      p->free_pages.pop_back();
+      const int j = p->npages[s]++;
+      p->bt[(size_t)s * p->mpps + j] = pid;
+      idx.push_back(s * p->mpps + j);
+      val.push_back(pid);
+    }
+  }
+  if (!idx.empty()) {
+    cudaError_t e = launch_block_table_update(p->d_bt, (int)idx.size(), idx.data(), val.data(), st);
+    if (e != cudaSuccess) return cuda_fail(e, "block table update");
+  }
+  // work items, in chunks of MAX_APPEND_SEQS sequences
+  const int T = p->T;
+  int row0 = 0;
+  for (int c0 = 0; c0 < n_seqs; c0 += MAX_APPEND_SEQS) {
+    const int cn = std::min(MAX_APPEND_SEQS, n_seqs - c0);
+    AppendParams ap;
+    std::memset(&ap, 0, sizeof(ap));
+    ap.pool = p->cache + p->layer_off[layer];
+    ap.page_bytes = p->page_bytes[layer];
+    ap.block_table = p->d_bt;
+    ap.max_pages_per_seq = p->mpps;
+    ap.tail = p->cache + p->tail_off;
+    ap.T = T; ap.L = p->L; ap.layer = layer; ap.Hkv = p->Hkv; ap.rot = p->rot;
+    ap.k_in = (const __half*)k_new;
+    ap.v_in = (const __half*)v_new;
+    ap.inv_s = p->d_inv ? p->d_inv + (size_t)layer * p->Hkv * 2 * D : nullptr;
+    ap.M = p->d_M;
+    ap.err = p->d_err;
+    for (int h = 0; h < p->Hkv; ++h) ap.heads[h] = p->head(layer, h);
+    int items = 0;
+    for (int k = 0; k < cn; ++k) {
+      const int i = c0 + k;
+      const int s = seq_ids[i];
+      const int64_t lo = p->len[(size_t)s * p->L + layer];
+      const int64_t ln = lo + n_new[i];
+      AppendSeq& q = ap.seqs[k];
+      q.seq = s; q.len_old = (int)lo; q.in_row0 = row0; q.item0 = items;
+      if (T == 0) {
+        q.nE = 0; q.nP = n_new[i]; q.nF = 0; q.e0 = 0; q.f0 = (int)ln;
+      } else {
+        const int64_t e0 = std::max<int64_t>(0, lo - T);
+        const int64_t e1 = std::min<int64_t>(lo, ln - T);
+        q.e0 = (int)e0;
+        q.nE = (int)std::max<int64_t>(0, e1 - e0);
+        q.nP = (int)std::max<int64_t>(0, ln - T - lo);
+        const int64_t f0 = std::max<int64_t>(lo, ln - T);
+        q.f0 = (int)f0;
+        q.nF = (int)(ln - f0);
+      }
+      items += q.nE + q.nP + q.nF;
+      row0 += n_new[i];
+    }
+    ap.n_seqs = cn;
+    ap.total_items = items;
+    cudaError_t e = launch_append(ap, st);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  }
+  for (int i = 0; i < n_seqs; ++i) p->len[(size_t)seq_ids[i] * p->L + layer] += n_new[i];
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const void* q, float* out,
+                                void* workspace, size_t workspace_bytes_given, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
+  if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
+  if (n_seqs == 0) return KVQ_OK;
+  if (!seq_ids || !q || !out) return fail(KVQ_ERR_INVALID_ARG, "null seq_ids, q or out");
+  if (((uintptr_t)q % 16) || ((uintptr_t)out % 16)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  DecodeParams dp = p->base_params(layer);
+  dp.q = (const __half*)q;
+  dp.out = out;
+  dp.n_seqs = n_seqs;
+  int64_t work = 0;
+  int maxpages = 1;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int s = seq_ids[i];
+    if (s < 0 || s >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d out of range", s);
+    const int64_t len = p->len[(size_t)s * p->L + layer];
+    dp.seq[i] = s;
+    dp.len[i] = (int)len;
+    const int64_t nq = len > p->T ? len - p->T : 0, nt = std::min<int64_t>(len, p->T);
+    const int pages = (int)((nq + PAGE - 1) / PAGE + (nt + PAGE - 1) / PAGE);
+    work += (int64_t)pages * p->Hkv;
+    maxpages = std::max(maxpages, pages);
+  }
+  dp.stage_bytes = p->stage_bytes[layer];
+  dp.n_stages = (8 * dp.stage_bytes <= 112 * 1024) ? 8 : 4;
+  const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G);
+  const int per_sm = std::max(1, (int)((228 * 1024) / (smem + 1024)));
+  const int64_t target = (int64_t)p->num_sms * std::min(per_sm, 4);
+  int pps = (int)std::max<int64_t>(1, (work + target - 1) / target);
+  if (pps > 2) pps = (pps + 3) & ~3;
+  const int min_pps = (maxpages + MAX_SPLITS - 3) / (MAX_SPLITS - 2);
+  pps = std::max(pps, min_pps);
+  if (const char* env = std::getenv("KVQ_DECODE_PAGES_PER_SPLIT")) {   // fixed split size (tests, tuning)
+    const int v = std::atoi(env);
+    if (v > 0) pps = std::max(v, min_pps);
+  }
+  dp.pps = pps;
+  int grid_x = 1;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int64_t len = dp.len[i];
+    const int64_t nq = len > p->T ? len - p->T : 0, nt = std::min<int64_t>(len, p->T);
+    const int qs = (int)(((nq + PAGE - 1) / PAGE + pps - 1) / pps);
+    const int ts = (int)(((nt + PAGE - 1) / PAGE + pps - 1) / pps);
+    grid_x = std::max(grid_x, qs + ts);
+  }
+  if (grid_x > 1) {
+    const size_t need = workspace_bytes(p, n_seqs);
+    if (!workspace || workspace_bytes_given < need)
+      return fail(KVQ_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes_given);
+    if ((uintptr_t)workspace % 16) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    dp.ws = (float*)workspace;
+    dp.tickets = (int*)((char*)workspace + (size_t)n_seqs * p->Hkv * MAX_SPLITS * p->G * PARTIAL_FLOATS * sizeof(float));
+  }
+  cudaError_t e = launch_decode(dp, grid_x, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_dequantize(const kvq_plan* p, int layer, int seq_id, int64_t t0, int64_t t1, float* k_out,
+                          float* v_out, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
+  if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id out of range");
+  const int64_t len = p->len[(size_t)seq_id * p->L + layer];
+  if (t0 < 0 || t1 < t0 || t1 > len) return fail(KVQ_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, %lld)",
+                                                 (long long)t0, (long long)t1, (long long)len);
+  if (((uintptr_t)k_out | (uintptr_t)v_out) % 16) return fail(KVQ_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  DecodeParams dp = p->base_params(layer);
+  dp.len[0] = (int)len;
+  cudaError_t e = launch_dequantize(dp, seq_id, t0, t1, k_out, v_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "dequantize launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_row_bytes(const kvq_plan* p, int layer, int head, int kv, int* cb, int* sb) {
+  if (!p || !cb || !sb) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (layer < 0 || layer >= p->L || head < 0 || head >= p->Hkv || (kv != 0 && kv != 1))
+    return fail(KVQ_ERR_INVALID_ARG, "layer, head or kv out of range");
+  const HeadInfo& h = p->head(layer, head);
+  *cb = kv ? h.cbV : h.cbK;
+  *sb = kv ? h.sbV : h.sbK;
+  return KVQ_OK;
+}
+
+kvq_status kvq_read_rows(const kvq_plan* p, int layer, int seq_id, int64_t t0, int64_t t1, int kv, void* codes,
+                         void* scales, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
+  if (layer < 0 || layer >= p->L || (kv != 0 && kv != 1)) return fail(KVQ_ERR_INVALID_ARG, "layer or kv out of range");
+  if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id out of range");
+  const int64_t len = p->len[(size_t)seq_id * p->L + layer];
+  const int64_t nq = len > p->T ? len - p->T : 0;
+  if (t0 < 0 || t1 < t0 || t1 > nq) return fail(KVQ_ERR_INVALID_ARG, "rows must lie in the quantized range [0, %lld)", (long long)nq);
+  if (!codes || !scales) return fail(KVQ_ERR_INVALID_ARG, "null output");
+  DecodeParams dp = p->base_params(layer);
+  cudaError_t e = launch_read_rows(dp, seq_id, t0, t1, kv, (uint8_t*)codes, (uint8_t*)scales, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "read_rows launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_length(const kvq_plan* p, int seq_id, int layer, int64_t* len) {
+  if (!p || !len) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (seq_id < 0 || seq_id >= p->max_seqs || layer < 0 || layer >= p->L)
+    return fail(KVQ_ERR_INVALID_ARG, "sequence or layer out of range");
+  *len = p->len[(size_t)seq_id * p->L + layer];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_reset(kvq_plan* p, int seq_id) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id out of range");
+  for (int l = 0; l < p->L; ++l) p->len[(size_t)seq_id * p->L + l] = 0;
+  for (int j = 0; j < p->npages[seq_id]; ++j) {
+    int& slot = p->bt[(size_t)seq_id * p->mpps + j];
+    p->free_pages.push_back(slot);
+    slot = -1;
+  }
+  p->npages[seq_id] = 0;
+  // the device table keeps stale ids for this sequence; they are overwritten
+  // before any read because reads are bounded by the (now zero) lengths.
+  return KVQ_OK;
+}
+
+kvq_status kvq_calibrate_varnorm(int64_t n_tokens, int n_channels, int64_t row_stride, const void* x, float* inv_rms,
+                                 void* stream) {
+  if (n_tokens < 1 || n_channels < 1 || row_stride < n_channels) return fail(KVQ_ERR_INVALID_ARG, "bad sizes");
+  if (!x || !inv_rms) return fail(KVQ_ERR_INVALID_ARG, "null pointer");
+  cudaError_t e = launch_calibrate(n_tokens, n_channels, row_stride, (const __half*)x, inv_rms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "calibrate launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_check_device_error(kvq_plan* p, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, p->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "error word read");
+  if (v == 0) return KVQ_OK;
+  cudaMemset(p->d_err, 0, sizeof(int));
+  if (v & ERR_TIMEOUT) return fail(KVQ_ERR_TIMEOUT, "a bounded wait inside a kernel ran out (error word 0x%x)", v);
+  return fail(KVQ_ERR_DEVICE, "a kernel latched device error word 0x%x (1 = missing page)", v);
+}
+
+kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int n, const void* x, float* y,
+                            void* stream) {
+  if (!p || !x || !y) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (layer < 0 || layer >= p->L || head < 0 || head >= p->Hkv || (kv != 0 && kv != 1) || n < 0)
+    return fail(KVQ_ERR_INVALID_ARG, "argument out of range");
+  const HeadInfo& h = p->head(layer, head);
+  const float* inv = p->d_inv ? p->d_inv + (((size_t)layer * p->Hkv + head) * 2 + kv) * D : nullptr;
+  const float* M = p->d_M ? p->d_M + h.m_off : nullptr;
+  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, M, n, (const __half*)x, y, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "debug_rotate launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_debug_quantize_f32(int codec, int r, int b, int n_rows, const float* y, void* codes, void* scales,
+                                  void* stream) {
+  if (!valid_codec(codec)) return fail(KVQ_ERR_UNSUPPORTED, "bad codec");
+  if (codec == KVQ_RANK && (!valid_rank(r) || b < 1 || b > 4)) return fail(KVQ_ERR_UNSUPPORTED, "bad rank or bits");
+  if (n_rows < 0 || !y || !codes || (!scales && codec != KVQ_F16)) return fail(KVQ_ERR_INVALID_ARG, "bad argument");
+  if (codec != KVQ_RANK) r = D;
+  cudaError_t e = launch_debug_quantize(codec, r, b, n_rows, y, (uint8_t*)codes, (uint8_t*)scales, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "debug_quantize launch");
+  return KVQ_OK;
+}
+
+}  // extern "C"

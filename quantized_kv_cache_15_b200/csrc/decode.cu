@@ -1,0 +1,564 @@
+// Decode attention over the paged, quantized cache: one new query token per
+// sequence attends over every cached token of its kv head (grouped-query
+// attention: G query heads share a kv head).
+//
+// Forum thread on KV compression (attention paragraph): dot the query with every
+// prior key, softmax, weighted average of the values -- and (bandwidth
+// paragraph) decode is bound by the bytes it must read, which is why the cache
+// is read once, in its packed form, and dequantized in registers.
+// BeeLlama v0.4.0 news, §KV cache 精度尾部: the tail segment is F16.
+//
+// Work split (split-K): grid (split, kv head, sequence).  A sequence's pages are
+// cut into splits of `pps` pages: first the quantized pages, then the tail
+// pages (never mixed in one split).  Each CTA:
+//   * warp 4 (producer) streams one page-head region per tile into a ring of
+//     shared-memory stages with cp.async.bulk (completion on mbarriers);
+//   * warps 0-3 (consumers) take tiles round-robin, each keeping its own online
+//     softmax state (max m, sum l, accumulator) for the G heads;
+//   * the four states are merged, then either finalised (single split) or
+//     written as a partial; the last CTA of the (sequence, kv head) -- found with
+//     an atomic ticket, no waiting -- merges all partials in split order and
+//     applies the inverse transform of the value basis.
+// Scores are kept in log2 units: q' carries softmax_scale * log2(e).
+//
+// The key score uses the stored basis: q . khat = (R (s_k * q)) . yhat for the
+// rotated paths (R symmetric orthogonal), (M_h q) . zhat for the projection, and
+// the raw q for F16 rows.  Per block, yhat = d*u + off, so
+//   q'.yhat_block = d * sum_j q'_j u_j + off * sum_j q'_j
+// with sum_j q'_j precomputed per block (qsum).
+#include <cfloat>
+
+#include "kvq_internal.h"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace kvq {
+
+enum { BASIS_RAW = 0, BASIS_ROT = 1, BASIS_PROJ = 2 };
+
+__host__ __device__ inline int basis_of(int codec, int rot) {
+  if (codec == KVQ_F16 || rot == KVQ_ROT_NONE) return BASIS_RAW;
+  if (codec == KVQ_RANK) return BASIS_PROJ;
+  return BASIS_ROT;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  return v;
+}
+
+// Offset term of a block: yhat = d*u + off.
+__device__ __forceinline__ float block_off(int codec, int bits, float d, float m) {
+  if (codec == KVQ_RANK) return -0.5f * (float)((1 << bits) - 1) * d;
+  if (codec_is_asym(codec)) return m;
+  return -(float)(1 << (bits - 1)) * d;
+}
+
+// Code j (0..n-1) of token t from an interleaved K plane (generic path).
+__device__ __forceinline__ uint32_t kcode_generic(const uint8_t* kp, int cb, int t, int bits, int n, int j) {
+  switch (bits) {
+    case 8: return kp[kplane_off(cb, t, j)];
+    case 4: return (kp[kplane_off(cb, t, j >> 1)] >> (4 * (j & 1))) & 15u;
+    case 2: return (kp[kplane_off(cb, t, j >> 2)] >> (2 * (j & 3))) & 3u;
+    case 1: return (kp[kplane_off(cb, t, j >> 3)] >> (j & 7)) & 1u;
+    case 6: {
+      uint32_t lo = (kp[kplane_off(cb, t, j >> 1)] >> (4 * (j & 1))) & 15u;
+      uint32_t hi = (kp[kplane_off(cb, t, n / 2 + (j >> 2))] >> (2 * (j & 3))) & 3u;
+      return lo | (hi << 4);
+    }
+    case 3: {
+      uint32_t lo = (kp[kplane_off(cb, t, j >> 2)] >> (2 * (j & 3))) & 3u;
+      uint32_t hi = (kp[kplane_off(cb, t, n / 4 + (j >> 3))] >> (j & 7)) & 1u;
+      return lo | (hi << 2);
+    }
+    default: return 0;
+  }
+}
+
+// Scores of token t for the G heads (log2 units).
+template <int G>
+__device__ __forceinline__ void score_token(int kc, int kbits, int n, int cb, int sb, const uint8_t* kp,
+                                            const uint8_t* ks, int t, const float* __restrict__ qv,
+                                            const float* __restrict__ qsum, float s[G]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g) s[g] = 0.f;
+  if (kc == KVQ_F16) {
+#pragma unroll 2
+    for (int c = 0; c < 16; ++c) {
+      uint4 v = *reinterpret_cast<const uint4*>(kp + (c * PAGE + t) * 16);
+      const __half2* hv = reinterpret_cast<const __half2*>(&v);
+      float x[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float2 f = __half22float2(hv[k]);
+        x[2 * k] = f.x; x[2 * k + 1] = f.y;
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[g] = fmaf(qv[g * D + 8 * c + j], x[j], s[g]);
+    }
+    return;
+  }
+  const int blk = n < 32 ? n : 32;
+  const int nb = n / blk;
+  const bool asym = codec_is_asym(kc);
+  for (int b = 0; b < nb; ++b) {
+    float a[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) a[g] = 0.f;
+    if (kc != KVQ_RANK && kbits == 8) {
+      uint4 v0 = *reinterpret_cast<const uint4*>(kp + ((2 * b) * PAGE + t) * 16);
+      uint4 v1 = *reinterpret_cast<const uint4*>(kp + ((2 * b + 1) * PAGE + t) * 16);
+      uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float u = (float)((w[k] >> (8 * i)) & 0xffu);
+#pragma unroll
+          for (int g = 0; g < G; ++g) a[g] = fmaf(qv[g * D + 32 * b + 4 * k + i], u, a[g]);
+        }
+    } else if (kc != KVQ_RANK && kbits == 4) {
+      uint4 v = *reinterpret_cast<const uint4*>(kp + (b * PAGE + t) * 16);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float u = (float)((w[k] >> (4 * i)) & 15u);
+#pragma unroll
+          for (int g = 0; g < G; ++g) a[g] = fmaf(qv[g * D + 32 * b + 8 * k + i], u, a[g]);
+        }
+    } else {
+      for (int j = 0; j < blk; ++j) {
+        const float u = (float)kcode_generic(kp, cb, t, kbits, n, b * blk + j);
+#pragma unroll
+        for (int g = 0; g < G; ++g) a[g] = fmaf(qv[g * D + b * blk + j], u, a[g]);
+      }
+    }
+    float d, m = 0.f;
+    if (asym) {
+      __half2 dm = *reinterpret_cast<const __half2*>(ks + t * sb + 4 * b);
+      d = __low2float(dm); m = __high2float(dm);
+    } else {
+      d = __half2float(*reinterpret_cast<const __half*>(ks + t * sb + 2 * b));
+    }
+    const float off = block_off(kc, kbits, d, m);
+#pragma unroll
+    for (int g = 0; g < G; ++g) s[g] = fmaf(d, a[g], fmaf(off, qsum[g * 4 + b], s[g]));
+  }
+}
+
+// Dequantized values of the lane's 4 channels (4l..4l+3) of V row t (row-major plane).
+__device__ __forceinline__ void v_lane(int vc, int vbits, int n, int cb, int sb, const uint8_t* vp, const uint8_t* vs,
+                                       int t, int lane, float v[4]) {
+  if (4 * lane >= n) { v[0] = v[1] = v[2] = v[3] = 0.f; return; }
+  const uint8_t* row = vp + t * cb;
+  if (vc == KVQ_F16) {
+    uint2 w = *reinterpret_cast<const uint2*>(row + 8 * lane);
+    float2 a = __half22float2(*reinterpret_cast<__half2*>(&w.x));
+    float2 b = __half22float2(*reinterpret_cast<__half2*>(&w.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+    return;
+  }
+  uint32_t u[4];
+  switch (vbits) {
+    case 8: { uint32_t w = *reinterpret_cast<const uint32_t*>(row + 4 * lane);
+      for (int i = 0; i < 4; ++i) u[i] = (w >> (8 * i)) & 0xffu; } break;
+    case 4: { uint32_t w = *reinterpret_cast<const uint16_t*>(row + 2 * lane);
+      for (int i = 0; i < 4; ++i) u[i] = (w >> (4 * i)) & 15u; } break;
+    case 2: { uint32_t w = row[lane];
+      for (int i = 0; i < 4; ++i) u[i] = (w >> (2 * i)) & 3u; } break;
+    case 1: { uint32_t w = (row[lane >> 1] >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = (w >> i) & 1u; } break;
+    case 6: { uint32_t lo = *reinterpret_cast<const uint16_t*>(row + 2 * lane); uint32_t hi = row[n / 2 + lane];
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> (2 * i)) & 3u) << 4); } break;
+    case 3: { uint32_t lo = row[lane]; uint32_t hi = (row[n / 4 + (lane >> 1)] >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (2 * i)) & 3u) | (((hi >> i) & 1u) << 2); } break;
+    default: u[0] = u[1] = u[2] = u[3] = 0;
+  }
+  const int blk = n < 32 ? n : 32;
+  const int b = (4 * lane) / blk;
+  float d, m = 0.f;
+  if (codec_is_asym(vc)) {
+    __half2 dm = *reinterpret_cast<const __half2*>(vs + t * sb + 4 * b);
+    d = __low2float(dm); m = __high2float(dm);
+  } else {
+    d = __half2float(*reinterpret_cast<const __half*>(vs + t * sb + 2 * b));
+  }
+  const float off = block_off(vc, vbits, d, m);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = fmaf((float)u[i], d, off);
+}
+
+size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
+  size_t ring = (size_t)stage_bytes * n_stages;
+  size_t merge = (size_t)4 * G * (D + 4) * sizeof(float);
+  size_t a = ring > merge ? ring : merge;
+  a = (a + 127) & ~(size_t)127;
+  a += (size_t)G * D * 4;            // qv
+  a += (size_t)G * 4 * 4;            // qsum
+  a += (size_t)4 * PAGE * G * 4;     // pbuf
+  a += (size_t)2 * G * D * 4;        // final accumulators (quantized basis, tail)
+  a += (size_t)2 * G * 4 + 16;       // final m, l, flag
+  a += (size_t)4 * D * 4;            // per-warp scratch
+  a = (a + 15) & ~(size_t)15;
+  a += (size_t)2 * 8 * 8;            // mbarriers
+  return a;
+}
+
+// Apply the value-basis inverse transform and write out[g][:] =
+// (T_v(aq) + at) / L for the CTA's G heads.  aq/at: smem [G][D].
+template <int G>
+__device__ void finalize(const DecodeParams& p, const HeadInfo& h, int vbasis, int head, float* aq, float* at,
+                         const float* fl, float* out_base) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp >= 4) return;
+  for (int g = warp; g < G; g += 4) {
+    const float L = fl[g];
+    const float invL = 1.0f / L;
+    float x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = aq[g * D + 4 * lane + i];
+    if (vbasis == BASIS_ROT) {
+      fwht_row(x);
+      if (p.s_v) {
+        const float* sv = p.s_v + (size_t)head * D;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] *= sv[4 * lane + i];
+      }
+    } else if (vbasis == BASIS_PROJ) {
+      const float* M = p.M + h.m_off;
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < h.r; ++i) {
+        const float a = aq[g * D + i];
+        float4 mrow = *reinterpret_cast<const float4*>(M + (size_t)i * D + 4 * lane);
+        y[0] = fmaf(mrow.x, a, y[0]); y[1] = fmaf(mrow.y, a, y[1]);
+        y[2] = fmaf(mrow.z, a, y[2]); y[3] = fmaf(mrow.w, a, y[3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) x[i] = y[i];
+    }
+    float4 o;
+    o.x = (x[0] + at[g * D + 4 * lane + 0]) * invL;
+    o.y = (x[1] + at[g * D + 4 * lane + 1]) * invL;
+    o.z = (x[2] + at[g * D + 4 * lane + 2]) * invL;
+    o.w = (x[3] + at[g * D + 4 * lane + 3]) * invL;
+    *reinterpret_cast<float4*>(out_base + (size_t)g * D + 4 * lane) = o;
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
+  const int seq = p.seq[si], len = p.len[si];
+  const int T = p.T;
+  const int nq = len > T ? len - T : 0;
+  const int nt = len < T ? len : T;
+  const int NQP = (nq + PAGE - 1) / PAGE, NTP = (nt + PAGE - 1) / PAGE;
+  const int qsplits = (NQP + p.pps - 1) / p.pps, tsplits = (NTP + p.pps - 1) / p.pps;
+  const int S = qsplits + tsplits;
+  float* out_base = p.out + ((size_t)si * p.Hq + (size_t)head * G) * D;
+  if (S == 0) {
+    if (split == 0)
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x) out_base[i] = 0.f;
+    return;
+  }
+  if (split >= S) return;
+  const bool is_tail = split >= qsplits;
+  const int pg0 = (is_tail ? split - qsplits : split) * p.pps;
+  const int pg1 = min(pg0 + p.pps, is_tail ? NTP : NQP);
+  const int n_tiles = pg1 - pg0;
+  const int seg_tokens = is_tail ? nt : nq;
+  const HeadInfo h = p.heads[head];
+  const int kc = is_tail ? (int)KVQ_F16 : (int)h.kcodec;
+  const int vc = is_tail ? (int)KVQ_F16 : (int)h.vcodec;
+  const int kbits = is_tail ? 16 : h.kbits, vbits = is_tail ? 16 : h.vbits;
+  const int kbasis = basis_of(kc, p.rot), vbasis = basis_of(vc, p.rot);
+  const int nK = kc == KVQ_RANK ? h.r : D, nV = vc == KVQ_RANK ? h.r : D;
+  const int cbK = is_tail ? 2 * D : h.cbK, sbK = is_tail ? 0 : h.sbK;
+  const int cbV = is_tail ? 2 * D : h.cbV, sbV = is_tail ? 0 : h.sbV;
+  const uint32_t tile_bytes = is_tail ? (uint32_t)TAIL_PAGE_BYTES : h.bytes;
+  const int NS = p.n_stages;
+
+  // shared memory carve-up
+  size_t ring = (size_t)p.stage_bytes * NS;
+  size_t merge = (size_t)4 * G * (D + 4) * sizeof(float);
+  size_t off = ((ring > merge ? ring : merge) + 127) & ~(size_t)127;
+  uint8_t* stages = smem;
+  float* mg = reinterpret_cast<float*>(smem);                 // merge area, aliases the ring after the loop
+  float* qv = reinterpret_cast<float*>(smem + off); off += (size_t)G * D * 4;
+  float* qsum = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4 * 4;
+  float* pbuf = reinterpret_cast<float*>(smem + off); off += (size_t)4 * PAGE * G * 4;
+  float* aq = reinterpret_cast<float*>(smem + off); off += (size_t)G * D * 4;
+  float* at = reinterpret_cast<float*>(smem + off); off += (size_t)G * D * 4;
+  float* fm = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4;
+  float* fl = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4;
+  int* flag = reinterpret_cast<int*>(smem + off); off += 16;
+  float* scratch = reinterpret_cast<float*>(smem + off); off += (size_t)4 * D * 4;
+  off = (off + 15) & ~(size_t)15;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
+  uint64_t* empty = full + 8;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    fence_mbar_init();
+  }
+
+  // ---- query preparation (consumer warps): q' in the K basis, scaled to log2 units
+  if (warp < 4) {
+    float* tmp = scratch + warp * D;
+    for (int g = warp; g < G; g += 4) {
+      const __half* qsrc = p.q + ((size_t)si * p.Hq + (size_t)head * G + g) * D;
+      uint2 raw = *reinterpret_cast<const uint2*>(qsrc + 4 * lane);
+      float2 a = __half22float2(*reinterpret_cast<__half2*>(&raw.x));
+      float2 b = __half22float2(*reinterpret_cast<__half2*>(&raw.y));
+      float x[4] = {a.x, a.y, b.x, b.y};
+      if (kbasis == BASIS_ROT) {
+        if (p.s_k) {
+          const float* sk = p.s_k + (size_t)head * D;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) x[i] *= sk[4 * lane + i];
+        }
+        fwht_row(x);
+      } else if (kbasis == BASIS_PROJ) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmp[4 * lane + i] = x[i];
+        __syncwarp();
+        const float* M = p.M + h.m_off;
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < D; ++c) {
+          const float xc = tmp[c];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (4 * lane + i < h.r) z[i] = fmaf(M[(size_t)(4 * lane + i) * D + c], xc, z[i]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = z[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[i] = (4 * lane + i < nK) ? x[i] * p.qscale : 0.f;
+        qv[g * D + 4 * lane + i] = x[i];
+      }
+      // per-block sums of q'
+      const int blk = nK < 32 ? nK : 32;
+      float ssum = (x[0] + x[1]) + (x[2] + x[3]);
+      for (int m = 1; m < blk / 4; m <<= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, m);
+      if (4 * lane < nK && ((4 * lane) % blk) == 0) qsum[g * 4 + (4 * lane) / blk] = ssum;
+    }
+  }
+  __syncthreads();
+
+  float m[G], l[G], acc[G][4];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m[g] = -INFINITY; l[g] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
+  }
+  if (warp == 4) {
+    // ---- producer
+    if (lane == 0) {
+      const uint8_t* tail_base =
+          is_tail ? p.tail + (((size_t)seq * p.L + p.layer) * p.Hkv + head) * (size_t)T * (D * 2 * 2) : nullptr;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int st = i % NS;
+        if (i >= NS && !mbar_wait(&empty[st], ((i / NS) - 1) & 1)) atomicOr(p.err, ERR_TIMEOUT);
+        const uint8_t* src;
+        if (is_tail) {
+          src = tail_base + (size_t)(pg0 + i) * TAIL_PAGE_BYTES;
+        } else {
+          int pid = p.block_table[(size_t)seq * p.max_pages_per_seq + pg0 + i];
+          if (pid < 0) { atomicOr(p.err, ERR_NO_PAGE); pid = 0; }
+          src = p.pool + (size_t)pid * p.page_bytes + h.off;
+        }
+        mbar_arrive_expect_tx(&full[st], tile_bytes);
+        bulk_g2s(stages + (size_t)st * p.stage_bytes, src, tile_bytes, &full[st]);
+      }
+    }
+  } else {
+    // ---- consumers
+    float* pw = pbuf + warp * PAGE * G;
+    for (int i = warp; i < n_tiles; i += 4) {
+      const int st = i % NS;
+      if (!mbar_wait(&full[st], (i / NS) & 1)) atomicOr(p.err, ERR_TIMEOUT);
+      const uint8_t* sp = stages + (size_t)st * p.stage_bytes;
+      const uint8_t* kp = sp;
+      const uint8_t* ks = kp + PAGE * cbK;
+      const uint8_t* vp = ks + PAGE * sbK;
+      const uint8_t* vs = vp + PAGE * cbV;
+      const int tok0 = (pg0 + i) * PAGE;
+      const int nvalid = min(PAGE, seg_tokens - tok0);
+      float s0[G], s1[G];
+      score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0);
+      score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (lane >= nvalid) s0[g] = -INFINITY;
+        if (lane + 32 >= nvalid) s1[g] = -INFINITY;
+        const float tmax = warp_max(fmaxf(s0[g], s1[g]));
+        const float mnew = fmaxf(m[g], tmax);
+        const float alpha = exp2f(m[g] - mnew);
+        const float p0 = exp2f(s0[g] - mnew), p1 = exp2f(s1[g] - mnew);
+        l[g] = l[g] * alpha + (p0 + p1);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[g][c] *= alpha;
+        m[g] = mnew;
+        pw[lane * G + g] = p0;
+        pw[(lane + 32) * G + g] = p1;
+      }
+      __syncwarp();
+      for (int t = 0; t < nvalid; ++t) {
+        float v[4];
+        v_lane(vc, vbits, nV, cbV, sbV, vp, vs, t, lane, v);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float w = pw[t * G + g];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[g][c] = fmaf(w, v[c], acc[g][c]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) l[g] = warp_sum(l[g]);
+  }
+  __syncthreads();   // every stage consumed: the ring is reused as the merge area below
+  if (warp < 4) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float* dst = mg + ((size_t)warp * G + g) * (D + 4);
+      if (lane == 0) { dst[0] = m[g]; dst[1] = l[g]; }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) dst[4 + 4 * lane + c] = acc[g][c];
+    }
+  }
+  __syncthreads();
+
+  // ---- merge the four warps' states
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, mg[((size_t)w * G + g) * (D + 4)]);
+    float L = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float mw = mg[((size_t)w * G + g) * (D + 4)];
+      L += (mw == -INFINITY) ? 0.f : exp2f(mw - M) * mg[((size_t)w * G + g) * (D + 4) + 1];
+    }
+    fm[g] = M; fl[g] = L;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, c = idx % D;
+    const float M = fm[g];
+    float A = 0.f;
+    for (int w = 0; w < 4; ++w) {
+      const float mw = mg[((size_t)w * G + g) * (D + 4)];
+      if (mw != -INFINITY) A += exp2f(mw - M) * mg[((size_t)w * G + g) * (D + 4) + 4 + c];
+    }
+    aq[idx] = is_tail ? 0.f : A;
+    at[idx] = is_tail ? A : 0.f;
+  }
+  __syncthreads();
+
+  if (S == 1) {
+    finalize<G>(p, h, vbasis, head, aq, at, fl, out_base);
+    return;
+  }
+  // ---- publish the partial, take a ticket
+  float* part = p.ws + (((size_t)si * p.Hkv + head) * MAX_SPLITS + split) * G * PARTIAL_FLOATS;
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, c = idx % D;
+    part[(size_t)g * PARTIAL_FLOATS + 4 + c] = is_tail ? at[idx] : aq[idx];
+  }
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    part[(size_t)g * PARTIAL_FLOATS + 0] = fm[g];
+    part[(size_t)g * PARTIAL_FLOATS + 1] = fl[g];
+    part[(size_t)g * PARTIAL_FLOATS + 2] = is_tail ? 1.f : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int old = atomicAdd(&p.tickets[si * p.Hkv + head], 1);
+    flag[0] = (old == S - 1);
+  }
+  __syncthreads();
+  if (!flag[0]) return;
+  __threadfence();
+  // ---- last CTA: merge every split in order
+  const float* base = p.ws + (((size_t)si * p.Hkv + head) * MAX_SPLITS) * G * PARTIAL_FLOATS;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS));
+    float L = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* ps = base + ((size_t)s * G + g) * PARTIAL_FLOATS;
+      const float ms = __ldcg(ps);
+      if (ms != -INFINITY) L += exp2f(ms - M) * __ldcg(ps + 1);
+    }
+    fm[g] = M; fl[g] = L;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, c = idx % D;
+    const float M = fm[g];
+    float Aq = 0.f, At = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* ps = base + ((size_t)s * G + g) * PARTIAL_FLOATS;
+      const float ms = __ldcg(ps);
+      if (ms == -INFINITY) continue;
+      const float f = exp2f(ms - M) * __ldcg(ps + 4 + c);
+      if (__ldcg(ps + 2) != 0.f) At += f; else Aq += f;
+    }
+    aq[idx] = Aq;
+    at[idx] = At;
+  }
+  if (threadIdx.x == 0) p.tickets[si * p.Hkv + head] = 0;
+  __syncthreads();
+  const int vb_final = basis_of(h.vcodec, p.rot);
+  finalize<G>(p, h, vb_final, head, aq, at, fl, out_base);
+}
+
+int decode_max_smem() { return 227 * 1024; }
+
+template <int G>
+static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
+  const size_t smem = decode_smem_bytes(p.stage_bytes, p.n_stages, G);
+  static size_t configured = 0;
+  if (smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  dim3 grid(grid_x, p.Hkv, p.n_seqs);
+  decode_kernel<G><<<grid, 160, smem, s>>>(p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int grid_x, cudaStream_t s) {
+  switch (p.G) {
+    case 1: return launch_g<1>(p, grid_x, s);
+    case 2: return launch_g<2>(p, grid_x, s);
+    case 3: return launch_g<3>(p, grid_x, s);
+    case 4: return launch_g<4>(p, grid_x, s);
+    case 5: return launch_g<5>(p, grid_x, s);
+    case 6: return launch_g<6>(p, grid_x, s);
+    case 7: return launch_g<7>(p, grid_x, s);
+    case 8: return launch_g<8>(p, grid_x, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace kvq

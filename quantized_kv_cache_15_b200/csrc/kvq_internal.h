@@ -1,0 +1,155 @@
+// Internal declarations of the kvq library (not part of the public ABI).
+//
+// Cache layout (all offsets in bytes, every region 128-byte aligned):
+//   [layer 0 pool][layer 1 pool]...[layer L-1 pool][tail rings]
+// A layer pool is n_pages pages; a page holds 64 consecutive token positions of
+// one sequence for every kv head of that layer.  Inside a page, head h owns a
+// contiguous region [K codes][K scales][V codes][V scales]:
+//   K codes : 64 rows of cbK bytes, "interleaved": byte i of token t sits at
+//             ((i / w) * 64 + t) * w + i % w, with w the largest of 16, 8, 4, 2
+//             that divides cbK -- lane t of a warp reads its token's w-byte piece
+//             next to lane t+1's (conflict-free, coalesced).
+//   K scales: 64 rows of sbK bytes, row-major.
+//   V codes : 64 rows of cbV bytes, row-major (lanes split one row's channels).
+//   V scales: 64 rows of sbV bytes, row-major.
+// Canonical packed rows (codes then scales) are defined by the quantizer: see
+// quant.cuh.  The tail ring of (seq, layer, kv head) is T/64 tail pages of
+// 32 KiB: [K fp16, interleaved as above with cb = 256][V fp16 row-major];
+// token position p lives in ring slot p % T.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int D = KVQ_HEAD_DIM;
+constexpr int PAGE = KVQ_PAGE_TOKENS;
+constexpr int MAX_HKV = KVQ_MAX_KV_HEADS;
+constexpr int MAX_G = KVQ_MAX_GQA;
+constexpr int MAX_BATCH = KVQ_MAX_BATCH;
+constexpr int MAX_SPLITS = 64;            // split-K pieces per (sequence, kv head)
+constexpr int TAIL_PAGE_BYTES = PAGE * D * 2 * 2;
+constexpr int PARTIAL_FLOATS = 4 + D;     // m, l, kind, pad, acc[128]
+
+// Device error word bits.
+constexpr int ERR_NO_PAGE = 1;
+constexpr int ERR_TIMEOUT = 2;
+constexpr int ERR_BAD_ARG = 4;
+
+struct HeadInfo {                // one (layer, kv head); 32 bytes
+  uint8_t kcodec, vcodec;        // kvq_codec
+  uint8_t r;                     // rank (KVQ_RANK), else 128
+  uint8_t kbits, vbits;          // code bits of K / V (16 for F16)
+  uint8_t pad[3];
+  uint16_t cbK, sbK, cbV, sbV;   // canonical row bytes (codes, scales)
+  uint32_t off;                  // region offset inside a page
+  uint32_t bytes;                // region bytes = 64 * (cbK + sbK + cbV + sbV)
+  uint32_t m_off;                // float offset of M_h (r x 128) in the projection table
+  uint32_t pad2;
+};
+
+__host__ __device__ inline int codec_bits(int c) {
+  switch (c) {
+    case KVQ_Q8_0: case KVQ_Q8_1: return 8;
+    case KVQ_Q6_0: case KVQ_Q6_1: return 6;
+    case KVQ_Q4_0: case KVQ_Q4_1: return 4;
+    case KVQ_Q3_0: case KVQ_Q3_1: return 3;
+    case KVQ_Q2_0: case KVQ_Q2_1: return 2;
+    default: return 16;
+  }
+}
+__host__ __device__ inline bool codec_is_asym(int c) { return c >= KVQ_Q8_1 && c <= KVQ_Q2_1; }
+__host__ __device__ inline int interleave_w(int cb) {
+  return (cb % 16 == 0) ? 16 : (cb % 8 == 0) ? 8 : (cb % 4 == 0) ? 4 : 2;
+}
+// Canonical row bytes of a codec (n = 128, or r for KVQ_RANK).
+__host__ __device__ inline void row_bytes(int codec, int r, int b, int* cb, int* sb) {
+  int n = codec == KVQ_RANK ? r : D;
+  int bits = codec == KVQ_RANK ? b : codec_bits(codec);
+  int blk = n < 32 ? n : 32;
+  int nb = n / blk;
+  *cb = n * bits / 8;
+  if (codec == KVQ_F16) *sb = 0;
+  else if (codec == KVQ_RANK) *sb = 2 * nb;
+  else *sb = codec_is_asym(codec) ? 4 * nb : 2 * nb;
+}
+
+// ---------------------------------------------------------------- append
+struct AppendSeq {
+  int seq;        // sequence id
+  int len_old;    // tokens in this layer before the call
+  int in_row0;    // first input row of this sequence
+  int item0;      // first work item of this sequence
+  int nE, nP, nF; // evicted-from-tail, pass-through, final-tail-occupant counts
+  int e0, f0;     // first evicted position, first final tail position
+};
+constexpr int MAX_APPEND_SEQS = 64;
+
+struct AppendParams {
+  uint8_t* pool;                 // this layer's page pool
+  uint32_t page_bytes;
+  const int* block_table;        // device [max_seqs][max_pages_per_seq]
+  int max_pages_per_seq;
+  uint8_t* tail;                 // tail region base (all sequences and layers)
+  int T, L, layer, Hkv;
+  int rot;
+  const __half* k_in;
+  const __half* v_in;
+  const float* inv_s;            // [Hkv][2][128] of this layer, or null
+  const float* M;                // projection table (floats), or null
+  int* err;
+  int n_seqs;
+  int total_items;
+  HeadInfo heads[MAX_HKV];
+  AppendSeq seqs[MAX_APPEND_SEQS];
+};
+
+// ---------------------------------------------------------------- decode
+struct DecodeParams {
+  const uint8_t* pool;
+  uint32_t page_bytes;
+  const int* block_table;
+  int max_pages_per_seq;
+  const uint8_t* tail;
+  int T, L, layer, Hkv, Hq, G;
+  int rot;
+  const __half* q;               // [n_seqs][Hq][128]
+  float* out;                    // [n_seqs][Hq][128]
+  const float* s_k;              // [Hkv][128] per-channel K dequant multiplier (varnorm) or null
+  const float* s_v;              // [Hkv][128] per-channel V multiplier or null
+  const float* M;                // projection table (floats), or null
+  float qscale;                  // softmax scale * log2(e)
+  int pps;                       // pages per split
+  int stage_bytes;               // bytes of one pipeline stage
+  int n_stages;                  // 4 or 8
+  float* ws;                     // partials [n_seqs*Hkv][MAX_SPLITS][G][PARTIAL_FLOATS]
+  int* tickets;                  // [n_seqs*Hkv]
+  int* err;
+  int n_seqs;
+  HeadInfo heads[MAX_HKV];
+  int seq[MAX_BATCH];
+  int len[MAX_BATCH];
+};
+
+// ---------------------------------------------------------------- launchers (host)
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t launch_block_table_update(int* table, int n, const int* idx_host, const int* val_host, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams& p, int grid_x, cudaStream_t s);
+cudaError_t launch_dequantize(const DecodeParams& p, int seq, int64_t t0, int64_t t1, float* k_out, float* v_out,
+                              cudaStream_t s);
+cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t t1, int kv, uint8_t* codes,
+                             uint8_t* scales, cudaStream_t s);
+cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __half* x, float* inv, cudaStream_t s);
+cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, const float* M, int n,
+                                const __half* x, float* y, cudaStream_t s);
+cudaError_t launch_debug_quantize(int codec, int r, int b, int n, const float* y, uint8_t* codes, uint8_t* scales,
+                                  cudaStream_t s);
+size_t decode_smem_bytes(int stage_bytes, int n_stages, int G);
+void note_launches(int n);   // counts kernel launches made by the library
+int decode_max_smem();
+
+}  // namespace kvq

@@ -91,9 +91,11 @@ def gauss(key: int, start: int, n: int, device) -> torch.Tensor:
 
 
 def student_t3(key: int, start: int, n: int, device) -> torch.Tensor:
-    z = gauss(key, 4 * start, 4 * n, device).reshape(n, 4)
+    """Z0 / sqrt((Z1^2 + Z2^2 + Z3^2) / 3), evaluated in fp64 (where division and
+    square root are correctly rounded on every device) and rounded once to fp32."""
+    z = gauss(key, 4 * start, 4 * n, device).reshape(n, 4).to(torch.float64)
     chi = (z[:, 1] * z[:, 1] + z[:, 2] * z[:, 2]) + z[:, 3] * z[:, 3]
-    return z[:, 0] / torch.sqrt(chi * (1.0 / 3.0))
+    return (z[:, 0] / torch.sqrt(chi / 3.0)).to(torch.float32)
 
 
 # ----------------------------------------------------------------------------- workloads
