@@ -35,6 +35,8 @@ sys.path.insert(0, ROOT)
 
 from quantized_kv_cache_15_b200 import workloads as W  # noqa: E402
 
+W_NAMES = {0: "f16", 1: "q8_0", 2: "q6_0", 3: "q4_0", 4: "q3_0", 5: "q2_0", 6: "q8_1", 7: "q6_1", 8: "q4_1",
+           9: "q3_1", 10: "q2_1", 11: "rank"}
 METRIC = "decode-attn µs/token & HBM GB/s (% of 8 TB/s); append-quantize tokens/s, 1 B200"
 NOMINAL_HBM_GBS = 8000.0
 
@@ -48,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs only)")
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5],
+                    help="which workload (default 2: the Llama-3.1-8B-shaped 32k decode)")
     return ap.parse_args()
 
 
@@ -63,6 +67,15 @@ def dist_setup(args):
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest value over all ranks (every rank gets it); identity at world size 1."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 def measured_peaks():
@@ -155,35 +168,54 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
-def cpu_oracle_decode_us_per_token(w, seconds, log):
+def cpu_oracle_decode_us_per_token(w, seconds, log, max_pairs=None):
     """Time the CPU oracle on a bounded sample of the same step: decode attention of
-    one (layer, kv head) over the full context from the oracle's own packed rows, for
-    as many kv heads as fit in `seconds`; extrapolated to the step (all layers and kv
-    heads).  Single-threaded C."""
+    one (layer, kv head) of sequence 0 over its full context, from the oracle's own
+    packed rows (plus the raw tail rows), for as many pairs as fit in `seconds`;
+    the mean time per cached token is scaled to the step (every layer, kv head and
+    sequence) and divided by the sequences decoded.  Single-threaded C."""
     import oracle
-    T = w.ctx[0]
-    times = []
+
+    def bits16(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    per_tok = []
     t_start = time.time()
     h = 0
+    n_pairs = w.n_layers * w.n_kv_heads
     while True:
-        layer, head = h // w.n_kv_heads, h % w.n_kv_heads
-        K = w.rows("K", layer, 0, 0, T)[:, head, :].contiguous().view(torch.int16).numpy().view(np.uint16)
-        V = w.rows("V", layer, 0, 0, T)[:, head, :].contiguous().view(torch.int16).numpy().view(np.uint16)
-        q = w.queries(layer, 0, 0)[head * w.G:(head + 1) * w.G].contiguous().view(torch.int16).numpy().view(np.uint16)
+        layer, head = (h * 7) % w.n_layers, h % w.n_kv_heads
+        n = w.ctx[0]
+        nq = max(0, n - w.tail)
+        K = bits16(w.rows("K", layer, 0, 0, n)[:, head, :])
+        V = bits16(w.rows("V", layer, 0, 0, n)[:, head, :])
+        q = bits16(w.queries(layer, 0, 0)[head * w.G:(head + 1) * w.G])
         kc, vc = w.k_codec[layer][head], w.v_codec[layer][head]
-        ck, sk = oracle.encode_rows(kc, w.rot, K)
-        cv, sv = oracle.encode_rows(vc, w.rot, V)
+        kw = {}
+        r, kb, vb = 128, 0, 0
+        if w.rot == W.ROT_PROJECTION:
+            r, kb, vb = w.rank[layer][head], w.k_bits[layer][head], w.v_bits[layer][head]
+            kw["M"] = oracle.fuse_projection(w.proj_basis(layer, head))
+        if w.rot == W.ROT_VARNORM_HADAMARD:
+            kw["inv_s_k"] = oracle.varnorm_inv_rms(bits16(w.calib_rows("K", layer, 512)[:, head, :]))
+            kw["inv_s_v"] = oracle.varnorm_inv_rms(bits16(w.calib_rows("V", layer, 512)[:, head, :]))
+        ck = sk = cv = sv = None
+        if nq:
+            ck, sk = oracle.encode_rows(kc, w.rot, K[:nq], inv_s=kw.get("inv_s_k"), M=kw.get("M"), r=r, b=kb)
+            cv, sv = oracle.encode_rows(vc, w.rot, V[:nq], inv_s=kw.get("inv_s_v"), M=kw.get("M"), r=r, b=vb)
         t0 = time.perf_counter()
-        oracle.decode_packed(ck, sk, cv, sv, None, None, q, kc, vc, w.rot)
-        times.append(time.perf_counter() - t0)
+        oracle.decode_packed(ck, sk, cv, sv, K[nq:], V[nq:], q, kc, vc, w.rot, r=r, kb=kb, vb=vb, **kw)
+        per_tok.append((time.perf_counter() - t0) / n)
         h += 1
-        if (time.time() - t_start > seconds and h >= 2) or h >= w.n_layers * w.n_kv_heads:
+        if (time.time() - t_start > seconds and h >= 2) or h >= n_pairs or (max_pairs and h >= max_pairs):
             break
-    per_head = statistics.mean(times)
-    us_per_token = per_head * w.n_layers * w.n_kv_heads * 1e6
-    sample = (f"oracle decode of {len(times)} (layer, kv head) pairs x {T} tokens x G={w.G}, from the oracle's own "
-              f"packed rows; mean {per_head:.3f} s per pair, scaled by {w.n_layers * w.n_kv_heads} pairs per step")
-    log(f"cpu oracle: {per_head:.3f} s per (layer, head) -> {us_per_token:.3e} us/token")
+    sec_per_token_head = statistics.mean(per_tok)
+    step_s = sec_per_token_head * sum(w.ctx) * w.n_layers * w.n_kv_heads
+    us_per_token = step_s * 1e6 / w.batch
+    sample = (f"oracle decode of {len(per_tok)} (layer, kv head) pairs of sequence 0 ({w.ctx[0]} tokens, G={w.G}) "
+              f"from the oracle's own packed rows; {sec_per_token_head * 1e6:.3f} us per cached (token, kv head), "
+              f"scaled to {sum(w.ctx)} tokens x {w.n_layers * w.n_kv_heads} (layer, kv head) per step / {w.batch} seq")
+    log(f"cpu oracle: {us_per_token:.3e} us/token")
     return {"value": us_per_token, "unit": "us/token", "cores": 1, "kind": "oracle", "sample": sample}
 
 
@@ -191,11 +223,11 @@ def cpu_oracle_decode_us_per_token(w, seconds, log):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    w = W.make_workload(2, "full")
+    w = W.make_workload(args.workload, "full")
     log = lambda m: print(m, file=sys.stderr, flush=True)  # noqa: E731
     vals = []
     for i in range(args.warmup + args.steps):
-        cb = cpu_oracle_decode_us_per_token(w, 0.0, log)     # one bounded sample (2 kv heads) per step
+        cb = cpu_oracle_decode_us_per_token(w, 0.0, log, max_pairs=2)   # one bounded sample per step
         if i >= args.warmup:
             vals.append(cb["value"])
     v = statistics.mean(vals)
@@ -205,58 +237,89 @@ def run_reference(args, world, rank):
             "config": {"workload": w.name, "layers": w.n_layers, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                        "context": w.ctx[0], "batch": 1},
             "cpu_baseline": {"value": v, "unit": "us/token", "cores": 1, "kind": "oracle",
-                             "sample": "each step: oracle decode of 2 (layer, kv head) pairs over the full context, "
-                                       "scaled to all 256 pairs of the step"},
+                             "sample": "each step: oracle decode of 2 (layer, kv head) pairs of sequence 0 over its "
+                                       "full context, scaled to every (layer, kv head, sequence) of the step"},
             "e2e": {"value": v, "unit": "us/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ----------------------------------------------------------------------------- kvq arm
+def make_plan(kvq, w, extra, dev):
+    """Plan for workload w with `extra` tokens of growth per sequence."""
+    kw = {}
+    if w.rot == W.ROT_VARNORM_HADAMARD:
+        inv = np.zeros((w.n_layers, w.n_kv_heads, 2, 128), np.float32)
+        for l in range(w.n_layers):
+            for kv, kind in enumerate("KV"):
+                x = w.calib_rows(kind, l, 512, device=dev).reshape(512, w.n_kv_heads * 128).contiguous()
+                o = torch.empty(w.n_kv_heads * 128, dtype=torch.float32, device=dev)
+                kvq.calibrate_varnorm(x, w.n_kv_heads * 128, w.n_kv_heads * 128, o)
+                inv[l, :, kv, :] = o.cpu().numpy().reshape(w.n_kv_heads, 128)
+        kw["inv_rms"] = inv
+    if w.rot == W.ROT_PROJECTION:
+        kw.update(rank=np.array(w.rank), k_bits=np.array(w.k_bits), v_bits=np.array(w.v_bits),
+                  proj_basis=[w.proj_basis(l, h) for l in range(w.n_layers) for h in range(w.n_kv_heads)])
+    pages = sum((c + extra + 63) // 64 for c in w.ctx) + 2 * w.batch
+    return kvq.Plan(w.n_layers, w.n_q_heads, w.n_kv_heads, max_seqs=w.batch, max_tokens_per_seq=max(w.ctx) + extra,
+                    k_codec=w.k_codec, v_codec=w.v_codec, rot=w.rot, tail_tokens=w.tail, max_pages=pages, **kw)
+
+
 def run_kvq(args, world, rank, local):
     from quantized_kv_cache_15_b200 import kvq
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     log = (lambda m: print(m, file=sys.stderr, flush=True)) if rank == 0 else (lambda m: None)
-    w = W.make_workload(2, "full")
+    w = W.make_workload(args.workload, "full")
     if args.layers:
         w.n_layers = args.layers
-        w.k_codec, w.v_codec = w.k_codec[:args.layers], w.v_codec[:args.layers]
-    L, Hq, Hkv, T = w.n_layers, w.n_q_heads, w.n_kv_heads, w.ctx[0]
+        for f in ("k_codec", "v_codec", "rank", "k_bits", "v_bits"):
+            if getattr(w, f) is not None:
+                setattr(w, f, getattr(w, f)[:args.layers])
+    L, Hq, Hkv, B = w.n_layers, w.n_q_heads, w.n_kv_heads, w.batch
     K, Wm = args.steps, args.warmup
-    extra = 2 * Wm + K + 8 + 2048
-    plan = kvq.Plan(L, Hq, Hkv, max_seqs=1, max_tokens_per_seq=T + extra, k_codec=w.k_codec, v_codec=w.v_codec,
-                    rot=w.rot)
+    # appends per step: one token per layer for every sequence, or (serving workload)
+    # a chunk for `append_seqs` sequences taken in rotation
+    n_app = w.append_tokens if w.append_tokens else 1
+    n_app_seqs = w.append_seqs if w.append_seqs else B
+    n_groups = max(1, B // n_app_seqs)
+    host_steps = Wm + 1 + K                              # warm-up, captured, e2e steps advance host lengths
+    growth = ((host_steps + n_groups - 1) // n_groups) * n_app + 2 * 2048 + 64
+    plan = make_plan(kvq, w, growth, dev)
     plan.allocate_cache(dev)
     t0 = time.time()
-    chunk = 4096
+    chunk = 8192
     for l in range(L):
-        for a in range(0, T, chunk):
-            b = min(T, a + chunk)
-            plan.append(l, [0], [b - a], w.rows("K", l, 0, a, b, dev), w.rows("V", l, 0, a, b, dev))
+        for s in range(B):
+            for a in range(0, w.ctx[s], chunk):
+                b = min(w.ctx[s], a + chunk)
+                plan.append(l, [s], [b - a], w.rows("K", l, s, a, b, dev), w.rows("V", l, s, a, b, dev))
     torch.cuda.synchronize()
     plan.check_device_error()
-    log(f"filled {L} layers x {T} tokens in {time.time() - t0:.1f} s; cache {plan.cache_bytes() / 1e9:.2f} GB")
+    log(f"filled {L} layers x {sum(w.ctx)} tokens in {time.time() - t0:.1f} s; cache {plan.cache_bytes() / 1e9:.2f} GB")
 
     stream = torch.cuda.Stream(dev)
-    ws = plan.new_workspace(1, dev)
-    n_tok_steps = Wm + 1 + K + Wm + 2
-    knew = torch.stack([w.rows("K", l, 0, T, T + n_tok_steps, dev) for l in range(L)])  # [L][n][Hkv][128]
-    vnew = torch.stack([w.rows("V", l, 0, T, T + n_tok_steps, dev) for l in range(L)])
-    qall = torch.stack([torch.stack([w.queries(l, 0, s, dev) for l in range(L)]) for s in range(n_tok_steps)])
-    out = torch.empty((L, 1, Hq, 128), dtype=torch.float32, device=dev)
-    tok = [0]
+    ws = plan.new_workspace(B, dev)
+    seqs = list(range(B))
+    # new rows of one step (same values every step; positions advance) and queries
+    knew = torch.stack([torch.cat([w.rows("K", l, s, w.ctx[s], w.ctx[s] + n_app, dev) for s in range(n_app_seqs)])
+                        for l in range(L)])
+    vnew = torch.stack([torch.cat([w.rows("V", l, s, w.ctx[s], w.ctx[s] + n_app, dev) for s in range(n_app_seqs)])
+                        for l in range(L)])
+    qall = torch.stack([torch.stack([w.queries(l, s, 0, dev) for s in seqs]) for l in range(L)])  # [L][B][Hq][128]
+    out = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+    step_no = [0]
 
-    def step(events=None):
-        i = tok[0]
+    def app_group():
+        g0 = (step_no[0] % n_groups) * n_app_seqs
+        return list(range(g0, g0 + n_app_seqs))
+
+    def step(kd=knew, vd=vnew, qd=qall):
+        grp = app_group()
         for l in range(L):
-            plan.append(l, [0], [1], knew[l, i], vnew[l, i], stream)
-            if events is not None:
-                events[l][0].record(stream)
-            plan.decode(l, [0], qall[i, l].unsqueeze(0), out[l], ws, stream)
-            if events is not None:
-                events[l][1].record(stream)
-        tok[0] += 1
+            plan.append(l, grp, [n_app] * len(grp), kd[l], vd[l], stream)
+            plan.decode(l, seqs, qd[l], out[l], ws, stream)
+        step_no[0] += 1
 
     with torch.cuda.stream(stream):
         for _ in range(Wm):
@@ -265,15 +328,16 @@ def run_kvq(args, world, rank, local):
     plan.check_device_error(stream)
 
     # capture one step (fixed positions; every replay does the full step's work)
-    length_at_capture = plan.seq_length(0, 0) + 1
+    lengths = [[plan.seq_length(s, l) for s in seqs] for l in range(L)]
+    grp = app_group()
+    for l in range(L):
+        for s in grp:
+            lengths[l][s] += n_app
     n0 = kvq.launch_count()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         step()
     launches_per_step = kvq.launch_count() - n0
-    for _ in range(Wm):
-        g.replay()
-    stream.synchronize()
     for _ in range(Wm):
         g.replay()
     stream.synchronize()
@@ -292,73 +356,57 @@ def run_kvq(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
     step_ms = ms / K
     plan.check_device_error(stream)
 
-    # ---- per-launch decode durations: the step's 32 decode launches, each between two
+    # ---- per-launch decode durations: the step's L decode launches, each between two
     # events, enqueued behind a GPU sleep so they run back to back (no host gaps)
     dec = []
     ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-    i_last = tok[0] - 1
     with torch.cuda.stream(stream):
-        for _ in range(K):
-            torch.cuda._sleep(4_000_000)
+        for _ in range(max(3, K // 4)):
+            torch.cuda._sleep(20_000_000 if B > 1 else 4_000_000)
             for l in range(L):
                 ev_pairs[l][0].record(stream)
-                plan.decode(l, [0], qall[i_last, l].unsqueeze(0), out[l], ws, stream)
+                plan.decode(l, seqs, qall[l], out[l], ws, stream)
                 ev_pairs[l][1].record(stream)
             stream.synchronize()
             dec.extend(a.elapsed_time(b) for a, b in ev_pairs)
     dec_ms = statistics.mean(dec)
 
     # ---- e2e through the public API: host buffers in, host buffers out
-    kh = knew.cpu().pin_memory()
-    vh = vnew.cpu().pin_memory()
-    qh = qall.cpu().pin_memory()
-    oh = torch.empty((L, 1, Hq, 128), dtype=torch.float32).pin_memory()
-    kd = torch.empty_like(knew[:, 0]); vd = torch.empty_like(vnew[:, 0]); qd = torch.empty_like(qall[0])
-    h2d = kd.numel() * 2 + vd.numel() * 2 + qd.numel() * 2
+    kh, vh, qh = knew.cpu().pin_memory(), vnew.cpu().pin_memory(), qall.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    kd, vd, qd = torch.empty_like(knew), torch.empty_like(vnew), torch.empty_like(qall)
+    h2d = (kd.numel() + vd.numel() + qd.numel()) * 2
     d2h = oh.numel() * 4
-    tok[0] = 0
     e2e_ms = []
-    base = plan.seq_length(0, 0)
     for s in range(K):
-        i = s % n_tok_steps
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         a.record(stream)
         with torch.cuda.stream(stream):
-            kd.copy_(kh[:, i], non_blocking=True)
-            vd.copy_(vh[:, i], non_blocking=True)
-            qd.copy_(qh[i], non_blocking=True)
-            for l in range(L):
-                plan.append(l, [0], [1], kd[l], vd[l], stream)
-                plan.decode(l, [0], qd[l].unsqueeze(0), out[l], ws, stream)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            qd.copy_(qh, non_blocking=True)
+            step(kd, vd, qd)
             oh.copy_(out, non_blocking=True)
         b.record(stream)
         stream.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    e2e_step = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_step], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_step = float(t.item())
+    e2e_step = max_over_ranks(statistics.mean(e2e_ms), world, dev)
     plan.check_device_error(stream)
 
-    # ---- append-quantize throughput: a 2048-token chunk into every layer (graph replay)
+    # ---- append-quantize throughput: a 2048-token chunk into every layer of sequence 0
     ck = torch.stack([w.rows("K", l, 0, 0, 2048, dev) for l in range(L)])
     cv = torch.stack([w.rows("V", l, 0, 0, 2048, dev) for l in range(L)])
-    ga = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         for l in range(L):
             plan.append(l, [0], [2048], ck[l], cv[l], stream)   # warm: allocates the chunk's pages
     stream.synchronize()
+    ga = torch.cuda.CUDAGraph()
     with torch.cuda.graph(ga, stream=stream):
         for l in range(L):
             plan.append(l, [0], [2048], ck[l], cv[l], stream)
@@ -374,36 +422,54 @@ def run_kvq(args, world, rank, local):
     stream.synchronize()
     app_ms = a.elapsed_time(b) / reps
     append_tps = 2048 / (app_ms / 1e3)
-    app_bytes = L * 2048 * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, 0, Hkv))
+    app_bytes = sum(2048 * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, l, Hkv)) for l in range(L))
     plan.check_device_error(stream)
 
-    # ---- accounting
-    dec_bytes = decode_algorithmic_bytes(plan, w, 0, length_at_capture)
-    step_bytes = L * dec_bytes + L * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, 0, Hkv))
+    # ---- accounting (algorithmic bytes of the captured step's decode launches)
+    def layer_decode_bytes(l):
+        tot = 0
+        bpt = bytes_per_token_head(plan, l, Hkv)
+        for s in seqs:
+            n = lengths[l][s]
+            nq = max(0, n - w.tail)
+            nt = n - nq
+            tot += nq * bpt + nt * Hkv * 2 * 128 * 2
+        return tot + B * Hq * 128 * (2 + 4)
+
+    dec_bytes_all = [layer_decode_bytes(l) for l in range(L)]
+    dec_bytes = statistics.mean(dec_bytes_all)
+    app_step_bytes = sum(n_app * n_app_seqs * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, l, Hkv)) for l in range(L))
+    step_bytes = sum(dec_bytes_all) + app_step_bytes
     peaks = measured_peaks()
     peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     traffic = traffic_from_profile(os.path.join(ROOT, "quantized_kv_cache_15_b200", "csrc", "decode.cu"))
     hbm_gbs = step_bytes / (step_ms / 1e3) / 1e9
-    us_per_token = step_ms * 1e3 / world
+    us_per_token = step_ms * 1e3 / (B * world)
+    codecs = sorted({W_NAMES[c] for row in w.k_codec for c in row}) + sorted({W_NAMES[c] for row in w.v_codec for c in row})
     line = {
         "metric": METRIC, "value": us_per_token, "unit": "us/token", "n_gpus": world, "steps": K, "warmup": Wm,
         "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": Hkv, "head_dim": 128,
-                   "context": T, "batch": 1, "k_codec": "q8_0", "v_codec": "q4_0", "rotation": "hadamard-128",
-                   "step": "per layer: append 1 token + decode attention", "parallelism": f"replicas x{world}",
-                   "l2": "no flush: packed cache read per step (%.2f GB) >> L2 (126 MB)" % (L * dec_bytes / 1e9)},
+                   "batch": B, "context": w.ctx[0] if B == 1 else f"{min(w.ctx)}..{max(w.ctx)} (mean {sum(w.ctx) / B:.0f})",
+                   "tail": w.tail, "codecs_k_v": codecs, "rotation": ["none", "hadamard-128", "varnorm+hadamard-128",
+                                                                       "per-head projection"][w.rot],
+                   "step": f"per layer: append {n_app} token(s) x {n_app_seqs} seq(s) + decode attention for {B} seq(s)",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "no flush: packed cache read per step (%.2f GB) >> L2 (126 MB)" % (sum(dec_bytes_all) / 1e9)},
+        "us_per_step": step_ms * 1e3,
         "hbm_gbs": hbm_gbs, "hbm_frac_of_8tbs": hbm_gbs / NOMINAL_HBM_GBS,
         "hbm_frac_of_measured": hbm_gbs / peak,
         "append_tokens_per_s": append_tps,
         "append_note": f"2048-token chunk appended to all {L} layers (K and V quantized): {app_ms:.3f} ms, "
                        f"{app_bytes / (app_ms / 1e3) / 1e9:.0f} GB/s algorithmic",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "decode_kernel<4>",
+                     "traffic": traffic, "kernel": f"decode_kernel<{w.G}>",
                      "bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
-                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, burst)" if peaks else "fallback 6650 GB/s"},
-        "e2e": {"value": e2e_step * 1e3 / world, "unit": "us/token", "h2d_bytes_per_step": h2d,
+                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, burst), of measured" if peaks
+                     else "fallback 6650 GB/s"},
+        "e2e": {"value": e2e_step * 1e3 / (B * world), "unit": "us/token", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * K,
         "clocks": clk,
