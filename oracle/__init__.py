@@ -24,12 +24,12 @@ _lock = threading.Lock()
 _lib = None
 
 # Codec and rotation ids (same numbering as the public C header, by value).
-F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK = range(12)
+F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK, Q5_0, Q5_1 = range(14)
 ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION = range(4)
-CODEC_BITS = {F16: 16, Q8_0: 8, Q6_0: 6, Q4_0: 4, Q3_0: 3, Q2_0: 2,
-              Q8_1: 8, Q6_1: 6, Q4_1: 4, Q3_1: 3, Q2_1: 2}
-CODEC_NAMES = {F16: "f16", Q8_0: "q8_0", Q6_0: "q6_0", Q4_0: "q4_0", Q3_0: "q3_0", Q2_0: "q2_0",
-               Q8_1: "q8_1", Q6_1: "q6_1", Q4_1: "q4_1", Q3_1: "q3_1", Q2_1: "q2_1", RANK: "rank"}
+CODEC_BITS = {F16: 16, Q8_0: 8, Q6_0: 6, Q5_0: 5, Q4_0: 4, Q3_0: 3, Q2_0: 2,
+              Q8_1: 8, Q6_1: 6, Q5_1: 5, Q4_1: 4, Q3_1: 3, Q2_1: 2}
+CODEC_NAMES = {F16: "f16", Q8_0: "q8_0", Q6_0: "q6_0", Q5_0: "q5_0", Q4_0: "q4_0", Q3_0: "q3_0", Q2_0: "q2_0",
+               Q8_1: "q8_1", Q6_1: "q6_1", Q5_1: "q5_1", Q4_1: "q4_1", Q3_1: "q3_1", Q2_1: "q2_1", RANK: "rank"}
 D = 128
 
 

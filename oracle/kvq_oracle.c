@@ -176,19 +176,20 @@ void orc_fwht_spec(int64_t n_rows, float* x) {
 
 /* Codec ids (shared numbering with the public header by value only). */
 enum { C_F16 = 0, C_Q8_0, C_Q6_0, C_Q4_0, C_Q3_0, C_Q2_0,
-       C_Q8_1, C_Q6_1, C_Q4_1, C_Q3_1, C_Q2_1, C_RANK = 11 };
+       C_Q8_1, C_Q6_1, C_Q4_1, C_Q3_1, C_Q2_1, C_RANK = 11, C_Q5_0 = 12, C_Q5_1 = 13 };
 
 static int codec_bits(int codec) {
     switch (codec) {
         case C_Q8_0: case C_Q8_1: return 8;
         case C_Q6_0: case C_Q6_1: return 6;
+        case C_Q5_0: case C_Q5_1: return 5;
         case C_Q4_0: case C_Q4_1: return 4;
         case C_Q3_0: case C_Q3_1: return 3;
         case C_Q2_0: case C_Q2_1: return 2;
         default: return 16;
     }
 }
-static int codec_is_1(int codec) { return codec >= C_Q8_1 && codec <= C_Q2_1; }
+static int codec_is_1(int codec) { return (codec >= C_Q8_1 && codec <= C_Q2_1) || codec == C_Q5_1; }
 
 /* Bytes of one packed row (R7): codes for n values at b bits, plus fp16
  * scales.  For the rank variant n = r and the block is min(32, r). */
@@ -296,6 +297,7 @@ static void quant_block_midrise(const float* x, int n, int bits, uint8_t* u, uin
 /* R7 packing.  u[0..n) with b bits each into a canonical row:
  *  b=8: byte j = u_j;  b=4: nibble j (LSB first);  b=2: 2-bit field j;
  *  b=1: bit j;  b=6: 4-bit plane of (u & 15) followed by 2-bit plane of u>>4;
+ *  b=5: 4-bit plane of (u & 15) followed by 1-bit plane of u>>4;
  *  b=3: 2-bit plane of (u & 3) followed by 1-bit plane of u>>2;
  *  b=16 (F16): little-endian binary16 values. */
 static void pack_field(const uint8_t* v, int n, int w, uint8_t* out) {
@@ -318,6 +320,9 @@ void orc_pack_codes(const uint8_t* u, int n, int bits, uint8_t* out) {
         case 6:
             for (int j = 0; j < n; ++j) { lo[j] = u[j] & 15; hi[j] = u[j] >> 4; }
             pack_field(lo, n, 4, out); pack_field(hi, n, 2, out + n / 2); break;
+        case 5:
+            for (int j = 0; j < n; ++j) { lo[j] = u[j] & 15; hi[j] = u[j] >> 4; }
+            pack_field(lo, n, 4, out); pack_field(hi, n, 1, out + n / 2); break;
         case 3:
             for (int j = 0; j < n; ++j) { lo[j] = u[j] & 3; hi[j] = u[j] >> 2; }
             pack_field(lo, n, 2, out); pack_field(hi, n, 1, out + n / 4); break;
@@ -333,6 +338,9 @@ void orc_unpack_codes(const uint8_t* in, int n, int bits, uint8_t* u) {
         case 1: unpack_field(in, n, 1, u); break;
         case 6:
             unpack_field(in, n, 4, lo); unpack_field(in + n / 2, n, 2, hi);
+            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 4)); break;
+        case 5:
+            unpack_field(in, n, 4, lo); unpack_field(in + n / 2, n, 1, hi);
             for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 4)); break;
         case 3:
             unpack_field(in, n, 2, lo); unpack_field(in + n / 4, n, 1, hi);

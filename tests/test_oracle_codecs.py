@@ -12,11 +12,11 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle import F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK
+from oracle import F16, Q8_0, Q6_0, Q5_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q5_1, Q4_1, Q3_1, Q2_1, RANK
 
 GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "codec_examples.json")))
-SYM = [Q8_0, Q6_0, Q4_0, Q3_0, Q2_0]
-ASYM = [Q8_1, Q6_1, Q4_1, Q3_1, Q2_1]
+SYM = [Q8_0, Q6_0, Q5_0, Q4_0, Q3_0, Q2_0]
+ASYM = [Q8_1, Q6_1, Q5_1, Q4_1, Q3_1, Q2_1]
 BITS = oracle.CODEC_BITS
 
 
@@ -28,8 +28,9 @@ def _scales_f32(codec, scales):
 
 
 def test_row_bytes():
-    expect = {F16: (256, 0), Q8_0: (128, 8), Q6_0: (96, 8), Q4_0: (64, 8), Q3_0: (48, 8), Q2_0: (32, 8),
-              Q8_1: (128, 16), Q6_1: (96, 16), Q4_1: (64, 16), Q3_1: (48, 16), Q2_1: (32, 16)}
+    expect = {F16: (256, 0), Q8_0: (128, 8), Q6_0: (96, 8), Q5_0: (80, 8), Q4_0: (64, 8), Q3_0: (48, 8),
+              Q2_0: (32, 8), Q8_1: (128, 16), Q6_1: (96, 16), Q5_1: (80, 16), Q4_1: (64, 16), Q3_1: (48, 16),
+              Q2_1: (32, 16)}
     for c, v in expect.items():
         assert oracle.row_bytes(c) == v
 
@@ -71,7 +72,7 @@ def test_packing_golden(name, bits):
 
 
 def test_packing_golden_planes():
-    for name, bits, key in (("pack_q6", 6, "u_first4"), ("pack_q3", 3, "u_first8")):
+    for name, bits, key in (("pack_q6", 6, "u_first4"), ("pack_q3", 3, "u_first8"), ("pack_q5", 5, "u_first8")):
         ex = GOLD[name]
         u = np.zeros(ex["n"], np.uint8)
         u[: len(ex[key])] = ex[key]
@@ -79,7 +80,7 @@ def test_packing_golden_planes():
         assert np.array_equal(oracle.unpack_codes(np.array(ex["bytes"], np.uint8), ex["n"], bits), u)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3, 4, 6, 8])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 8])
 def test_pack_roundtrip(bits):
     rng = np.random.default_rng(bits)
     for n in (16, 32, 96, 128):
@@ -174,7 +175,8 @@ def test_mse_falls_about_4x_per_bit_symmetric():
         mse[BITS[c]] = np.mean((oracle.dequantize_rows(c, codes, scales) - y) ** 2)
     assert 3.0 < (mse[4] / mse[6]) ** 0.5 < 6.5          # per-bit factor over a 2-bit step
     assert 3.0 < (mse[6] / mse[8]) ** 0.5 < 6.5
-    assert mse[2] > mse[3] > mse[4] > mse[6] > mse[8]
+    assert 3.0 < mse[4] / mse[5] < 6.5 and 3.0 < mse[5] / mse[6] < 6.5
+    assert mse[2] > mse[3] > mse[4] > mse[5] > mse[6] > mse[8]
 
 
 @pytest.mark.parametrize("r", [16, 32, 64, 96, 128])
