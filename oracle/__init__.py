@@ -88,6 +88,10 @@ def _declare(L):
     L.orc_decode_head.argtypes = [_I64, _I, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, ctypes.c_float, _P]
     L.orc_decode_packed.argtypes = [_I64, _P, _P, _P, _P, _I64, _P, _P, _I, _P,
                                     _I, _I, _I, _I, _I, _I, _P, _P, _P, ctypes.c_float, _P]
+    L.orc_cobra_error.restype = ctypes.c_double
+    L.orc_cobra_error.argtypes = [_P, _I, _I, _P]
+    L.orc_cobra_best.argtypes = [_P, _I, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
+    L.orc_cobra_allocate.argtypes = [_I, _P, ctypes.c_double, _P, _P, _P]
 
 
 def _ptr(a):
@@ -291,3 +295,30 @@ def decode_packed(ck, sk, cv, sv, Kt, Vt, q_f16, k_codec, v_codec, rot, r=D, kb=
     lib().orc_decode_packed(nq, *[_ptr(a) for a in args], Kt.shape[0], _ptr(Kt), _ptr(Vt), G, _ptr(q),
                             k_codec, v_codec, rot, r, kb, vb, _ptr(inv_s_k), _ptr(inv_s_v), _ptr(M), float(scale), _ptr(out))
     return out
+
+
+# ----------------------------------------------------------------------------- KV-COBRA allocation
+def cobra_error(lam, r, b, eps):
+    lam = _c(lam, np.float64)
+    eps = _c(eps, np.float64)
+    return lib().orc_cobra_error(_ptr(lam), r, b, _ptr(eps))
+
+
+def cobra_best(lam, budget, eps):
+    lam = _c(lam, np.float64)
+    eps = _c(eps, np.float64)
+    r, b = _I(0), _I(0)
+    ok = lib().orc_cobra_best(_ptr(lam), budget, _ptr(eps), ctypes.byref(r), ctypes.byref(b))
+    return (r.value, b.value) if ok else None
+
+
+def cobra_allocate(lambdas, bpd, eps):
+    """lambdas: [n_heads][128] direction variances, each sorted decreasing.
+    Returns (ranks int32 [n], bits int32 [n], bits used)."""
+    lam = _c(lambdas, np.float64)
+    eps = _c(eps, np.float64)
+    n = lam.shape[0]
+    r = np.zeros(n, np.int32)
+    b = np.zeros(n, np.int32)
+    used = lib().orc_cobra_allocate(n, _ptr(lam), float(bpd), _ptr(eps), _ptr(r), _ptr(b))
+    return r, b, used

@@ -626,3 +626,75 @@ void orc_decode_packed(int64_t nq, const uint8_t* ck, const uint16_t* sk, const 
     }
     free(Kd); free(Vd);
 }
+
+/* ------------------------------------------------------------------------- */
+/* KV-COBRA allocation of rank and bits per head [COBRA §The news (steps C1   */
+/* and C2) and §Where the bits actually go]                                   */
+/* ------------------------------------------------------------------------- */
+
+static const int COBRA_R[5] = {16, 32, 64, 96, 128};
+
+/* Error of keeping the top r directions of a head at b bits: the variance of
+ * the dropped directions (lost outright) plus the rounding noise of the kept
+ * ones, eps[b-1] times their variance.  lambda: the head's 128 direction
+ * variances, sorted in decreasing order. */
+double orc_cobra_error(const double* lambda, int r, int b, const double* eps) {
+    double kept = 0.0, lost = 0.0;
+    for (int i = 0; i < D; ++i) {
+        if (i < r) kept += lambda[i];
+        else lost += lambda[i];
+    }
+    return lost + eps[b - 1] * kept;
+}
+
+/* C1: the (r, b) with r*b <= budget of least error (ties: fewer bits, then
+ * smaller r).  Returns 0 and leaves r, b untouched if nothing fits. */
+int orc_cobra_best(const double* lambda, int budget, const double* eps, int* r_out, int* b_out) {
+    double best = INFINITY;
+    int found = 0, best_bits = 0;
+    for (int ri = 0; ri < 5; ++ri)
+        for (int b = 1; b <= 4; ++b) {
+            int bits = COBRA_R[ri] * b;
+            if (bits > budget) continue;
+            double e = orc_cobra_error(lambda, COBRA_R[ri], b, eps);
+            if (!found || e < best || (e == best && bits < best_bits) ||
+                (e == best && bits == best_bits && COBRA_R[ri] < *r_out)) {
+                best = e; best_bits = bits; *r_out = COBRA_R[ri]; *b_out = b; found = 1;
+            }
+        }
+    return found;
+}
+
+/* C2: water-filling over heads.  Every head starts at the cheapest setting
+ * (r = 16, b = 1); the remaining bits of the budget (bpd * 128 per head) go,
+ * one upgrade at a time, to the head whose best affordable upgrade removes the
+ * most error per extra bit (ties: lower head index, then fewer bits), until no
+ * upgrade fits or none lowers the error.  lambdas: [n_heads][128], each sorted
+ * in decreasing order.  Returns the bits used. */
+int orc_cobra_allocate(int n_heads, const double* lambdas, double bpd, const double* eps, int* r, int* b) {
+    const int budget = (int)(bpd * D * n_heads + 0.5);
+    int used = 0;
+    for (int h = 0; h < n_heads; ++h) { r[h] = 16; b[h] = 1; used += 16; }
+    for (;;) {
+        int bh = -1, br = 0, bb = 0, bbits = 0;
+        double bgain = 0.0;
+        for (int h = 0; h < n_heads; ++h) {
+            const double* lam = lambdas + (size_t)h * D;
+            const double e0 = orc_cobra_error(lam, r[h], b[h], eps);
+            const int cur = r[h] * b[h];
+            for (int ri = 0; ri < 5; ++ri)
+                for (int bi = 1; bi <= 4; ++bi) {
+                    int bits = COBRA_R[ri] * bi;
+                    if (bits <= cur || used - cur + bits > budget) continue;
+                    double gain = (e0 - orc_cobra_error(lam, COBRA_R[ri], bi, eps)) / (double)(bits - cur);
+                    if (gain > bgain || (gain == bgain && gain > 0.0 && bh == h && bits < bbits)) {
+                        bgain = gain; bh = h; br = COBRA_R[ri]; bb = bi; bbits = bits;
+                    }
+                }
+        }
+        if (bh < 0) break;
+        used += bbits - r[bh] * b[bh];
+        r[bh] = br; b[bh] = bb;
+    }
+    return used;
+}
