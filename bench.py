@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 from quantized_kv_cache_15_b200 import workloads as W  # noqa: E402
 
 W_NAMES = {0: "f16", 1: "q8_0", 2: "q6_0", 3: "q4_0", 4: "q3_0", 5: "q2_0", 6: "q8_1", 7: "q6_1", 8: "q4_1",
-           9: "q3_1", 10: "q2_1", 11: "rank"}
+           9: "q3_1", 10: "q2_1", 11: "rank", 12: "q5_0", 13: "q5_1"}
 METRIC = "decode-attn µs/token & HBM GB/s (% of 8 TB/s); append-quantize tokens/s, 1 B200"
 NOMINAL_HBM_GBS = 8000.0
 
@@ -102,7 +102,18 @@ def decode_algorithmic_bytes(plan, w, layer, length):
     return cache + w.n_q_heads * 128 * 2 + w.n_q_heads * 128 * 4
 
 
-def traffic_from_profile(kernel_file):
+DECODE_SOURCES = ("decode.cu", "decode_fast.cuh", "kvq_internal.h", "ptx.cuh", "quant.cuh")
+
+
+def kernel_source_sha256():
+    """sha256 over the decode kernel's source files (in DECODE_SOURCES order)."""
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        h.update(open(os.path.join(ROOT, "quantized_kv_cache_15_b200", "csrc", name), "rb").read())
+    return h.hexdigest()
+
+
+def traffic_from_profile(kernel_file=None):
     """dram bytes per launch recorded in profiles/decode_attention_llama8b.md, if the
     kernel source still matches the one profiled (else None)."""
     path = os.path.join(ROOT, "profiles", "decode_attention_llama8b.md")
@@ -114,8 +125,7 @@ def traffic_from_profile(kernel_file):
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
     if not m or not h:
         return None
-    src = open(kernel_file, "rb").read()
-    if hashlib.sha256(src).hexdigest() != h.group(1):
+    if kernel_source_sha256() != h.group(1):
         return None
     return float(m.group(1))
 
@@ -338,8 +348,11 @@ def run_kvq(args, world, rank, local):
     with torch.cuda.graph(g, stream=stream):
         step()
     launches_per_step = kvq.launch_count() - n0
-    for _ in range(Wm):
-        g.replay()
+    # CUDAGraph.replay() launches on the current stream: replay on `stream`, where the
+    # timing events are recorded
+    with torch.cuda.stream(stream):
+        for _ in range(Wm):
+            g.replay()
     stream.synchronize()
 
     # ---- timed region: device time of K steps
@@ -350,10 +363,11 @@ def run_kvq(args, world, rank, local):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(K):
-        g.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(K):
+            g.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
@@ -410,15 +424,15 @@ def run_kvq(args, world, rank, local):
     with torch.cuda.graph(ga, stream=stream):
         for l in range(L):
             plan.append(l, [0], [2048], ck[l], cv[l], stream)
-    for _ in range(3):
-        ga.replay()
-    stream.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     reps = 10
-    a.record(stream)
-    for _ in range(reps):
-        ga.replay()
-    b.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            ga.replay()
+        a.record(stream)
+        for _ in range(reps):
+            ga.replay()
+        b.record(stream)
     stream.synchronize()
     app_ms = a.elapsed_time(b) / reps
     append_tps = 2048 / (app_ms / 1e3)

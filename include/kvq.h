@@ -78,11 +78,14 @@ typedef enum {
  *     min(32, r) coordinates is quantized mid-rise with all 2^b levels
  *     (levels (k + 1/2) d, d = max|z| / (2^(b-1) - 1/2)); r and b per head.
  *  KVQ_F16: raw fp16 rows (unrotated).
- * Codes are stored offset-binary (u = code + 2^(b-1) for _0).  Byte layouts
- * are given in the repository's design document. */
+ * Codes are stored offset-binary (u = code + 2^(b-1) for _0).  Bit planes:
+ * 6 bits = 4-bit plane + 2-bit plane, 5 bits = 4-bit plane + 1-bit plane,
+ * 3 bits = 2-bit plane + 1-bit plane.  Byte layouts are given in the
+ * repository's design document. */
 typedef enum {
   KVQ_F16 = 0, KVQ_Q8_0 = 1, KVQ_Q6_0 = 2, KVQ_Q4_0 = 3, KVQ_Q3_0 = 4, KVQ_Q2_0 = 5,
-  KVQ_Q8_1 = 6, KVQ_Q6_1 = 7, KVQ_Q4_1 = 8, KVQ_Q3_1 = 9, KVQ_Q2_1 = 10, KVQ_RANK = 11
+  KVQ_Q8_1 = 6, KVQ_Q6_1 = 7, KVQ_Q4_1 = 8, KVQ_Q3_1 = 9, KVQ_Q2_1 = 10, KVQ_RANK = 11,
+  KVQ_Q5_0 = 12, KVQ_Q5_1 = 13
 } kvq_codec;
 
 /* Transform applied to rows before quantization (F16 rows are never

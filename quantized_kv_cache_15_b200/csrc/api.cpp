@@ -12,6 +12,8 @@
 #include <string>
 #include <vector>
 
+#include <cuda_fp16.h>
+
 #include "kvq_internal.h"
 
 using namespace kvq;
@@ -35,7 +37,7 @@ kvq_status cuda_fail(cudaError_t e, const char* what) {
   return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-bool valid_codec(int c) { return c >= KVQ_F16 && c <= KVQ_RANK; }
+bool valid_codec(int c) { return c >= KVQ_F16 && c <= KVQ_Q5_1; }
 bool valid_rank(int r) { return r == 16 || r == 32 || r == 64 || r == 96 || r == 128; }
 
 // In-place Sylvester Walsh-Hadamard transform of length n (power of two), double.
@@ -72,6 +74,7 @@ struct kvq_plan {
   float* d_sk = nullptr;    // [L][Hkv][128] 1/inv_rms of K (decode, dequantize)
   float* d_sv = nullptr;    // [L][Hkv][128] 1/inv_rms of V
   float* d_M = nullptr;     // fused projections
+  uint8_t* d_Mimg = nullptr;  // fp16 hi/lo tensor-core images of the projections
   int* d_bt = nullptr;      // block table [max_seqs][mpps]
   int* d_err = nullptr;
   std::vector<int64_t> len;           // [max_seqs][L]
@@ -83,7 +86,7 @@ struct kvq_plan {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(device);
-    cudaFree(d_inv); cudaFree(d_sk); cudaFree(d_sv); cudaFree(d_M); cudaFree(d_bt); cudaFree(d_err);
+    cudaFree(d_inv); cudaFree(d_sk); cudaFree(d_sv); cudaFree(d_M); cudaFree(d_Mimg); cudaFree(d_bt); cudaFree(d_err);
     cudaSetDevice(prev);
   }
 
@@ -160,6 +163,7 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
 
   // per-head codec info and page layout
   std::vector<float> Mhost;
+  std::vector<uint16_t> Mimg;    // per head: hi image then lo image, r x 128 fp16 each
   const double* pb = d->proj_basis;
   p->heads.resize((size_t)p->L * p->Hkv);
   p->layer_off.resize(p->L);
@@ -213,6 +217,20 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
         }
         Mhost.insert(Mhost.end(), M.begin(), M.end());
         while (Mhost.size() % 4) Mhost.push_back(0.f);
+        // tensor-core images: canonical K-major core-matrix layout, element (n, k) at
+        // ((n / 8) * 16 + k / 8) * 64 + (n % 8) * 8 + k % 8  (in fp16 elements)
+        hi.mimg_off = (uint32_t)(Mimg.size() * 2);
+        std::vector<uint16_t> img((size_t)2 * r * D);
+        for (int n = 0; n < r; ++n)
+          for (int k = 0; k < D; ++k) {
+            const float v = M[(size_t)n * D + k];
+            const __half hh = __float2half_rn(v);
+            const __half hl = __float2half_rn(v - __half2float(hh));
+            const size_t e = ((size_t)(n / 8) * 16 + k / 8) * 64 + (n % 8) * 8 + k % 8;
+            img[e] = __half_as_ushort(hh);
+            img[(size_t)r * D + e] = __half_as_ushort(hl);
+          }
+        Mimg.insert(Mimg.end(), img.begin(), img.end());
         pb += (size_t)D * r;
       }
       p->heads[i] = hi;
@@ -269,6 +287,11 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
       return fail(KVQ_ERR_OOM, "device allocation for the projections failed");
     }
     cudaMemcpy(p->d_M, Mhost.data(), Mhost.size() * 4, cudaMemcpyHostToDevice);
+    if (!dmalloc((void**)&p->d_Mimg, Mimg.size() * 2)) {
+      delete p;
+      return fail(KVQ_ERR_OOM, "device allocation for the projection images failed");
+    }
+    cudaMemcpy(p->d_Mimg, Mimg.data(), Mimg.size() * 2, cudaMemcpyHostToDevice);
   }
   p->len.assign((size_t)p->max_seqs * p->L, 0);
   p->bt.assign((size_t)p->max_seqs * p->mpps, -1);
@@ -386,7 +409,7 @@ kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* se
     ap.M = p->d_M;
     ap.err = p->d_err;
     for (int h = 0; h < p->Hkv; ++h) ap.heads[h] = p->head(layer, h);
-    int items = 0;
+    int items = 0, qitems = 0;
     for (int k = 0; k < cn; ++k) {
       const int i = c0 + k;
       const int s = seq_ids[i];
@@ -406,11 +429,29 @@ kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* se
         q.f0 = (int)f0;
         q.nF = (int)(ln - f0);
       }
+      q.qitem0 = qitems;
       items += q.nE + q.nP + q.nF;
+      qitems += q.nE + q.nP;
       row0 += n_new[i];
     }
     ap.n_seqs = cn;
     ap.total_items = items;
+    if (p->rot == KVQ_ROT_PROJECTION && qitems > 0) {
+      // tensor-core projection + quantization of the rows leaving (or bypassing) the
+      // tail; it reads evicted rows from the ring, so it runs before the ring writes
+      ProjParams pp;
+      std::memset(&pp, 0, sizeof(pp));
+      pp.pool = ap.pool; pp.page_bytes = ap.page_bytes; pp.block_table = ap.block_table;
+      pp.max_pages_per_seq = ap.max_pages_per_seq; pp.tail = ap.tail;
+      pp.T = T; pp.L = p->L; pp.layer = layer; pp.Hkv = p->Hkv;
+      pp.k_in = ap.k_in; pp.v_in = ap.v_in; pp.in_stride = p->Hkv * D;
+      pp.mimg = p->d_Mimg; pp.err = p->d_err;
+      pp.n_seqs = cn; pp.total_q = qitems;
+      std::memcpy(pp.heads, ap.heads, sizeof(pp.heads));
+      std::memcpy(pp.seqs, ap.seqs, sizeof(pp.seqs));
+      cudaError_t e = launch_project(pp, (qitems + 127) / 128, p->Hkv, st);
+      if (e != cudaSuccess) return cuda_fail(e, "projection launch");
+    }
     cudaError_t e = launch_append(ap, st);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
   }
@@ -439,18 +480,23 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
     const int64_t len = p->len[(size_t)s * p->L + layer];
     dp.seq[i] = s;
     dp.len[i] = (int)len;
-    const int64_t nq = len > p->T ? len - p->T : 0, nt = std::min<int64_t>(len, p->T);
-    const int pages = (int)((nq + PAGE - 1) / PAGE + (nt + PAGE - 1) / PAGE);
+    const SplitCounts c = split_counts((int)len, (int)p->T, 1);
+    const int pages = c.nqp + c.ntp;
     work += (int64_t)pages * p->Hkv;
     maxpages = std::max(maxpages, pages);
   }
+  // Stage ring: as deep as fits three CTAs per SM (the register limit of the kernel),
+  // at least four stages (one per consumer warp).
   dp.stage_bytes = p->stage_bytes[layer];
-  dp.n_stages = (8 * dp.stage_bytes <= 112 * 1024) ? 8 : 4;
+  dp.n_stages = 4;
+  for (int ns = 8; ns > 4; --ns)
+    if (decode_smem_bytes(dp.stage_bytes, ns, p->G) + 1024 <= (228 * 1024) / 3) { dp.n_stages = ns; break; }
   const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G);
-  const int per_sm = std::max(1, (int)((228 * 1024) / (smem + 1024)));
-  const int64_t target = (int64_t)p->num_sms * std::min(per_sm, 4);
+  // One full wave: as many CTAs as are resident at once (registers and shared memory
+  // both counted), each taking an equal share of the page-heads.
+  const int per_sm = std::max(1, decode_blocks_per_sm(p->G, smem));
+  const int64_t target = (int64_t)p->num_sms * per_sm;
   int pps = (int)std::max<int64_t>(1, (work + target - 1) / target);
-  if (pps > 2) pps = (pps + 3) & ~3;
   const int min_pps = (maxpages + MAX_SPLITS - 3) / (MAX_SPLITS - 2);
   pps = std::max(pps, min_pps);
   if (const char* env = std::getenv("KVQ_DECODE_PAGES_PER_SPLIT")) {   // fixed split size (tests, tuning)
@@ -460,11 +506,8 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   dp.pps = pps;
   int grid_x = 1;
   for (int i = 0; i < n_seqs; ++i) {
-    const int64_t len = dp.len[i];
-    const int64_t nq = len > p->T ? len - p->T : 0, nt = std::min<int64_t>(len, p->T);
-    const int qs = (int)(((nq + PAGE - 1) / PAGE + pps - 1) / pps);
-    const int ts = (int)(((nt + PAGE - 1) / PAGE + pps - 1) / pps);
-    grid_x = std::max(grid_x, qs + ts);
+    const SplitCounts c = split_counts(dp.len[i], (int)p->T, pps);
+    grid_x = std::max(grid_x, c.qsplits + c.tsplits);
   }
   if (grid_x > 1) {
     const size_t need = workspace_bytes(p, n_seqs);
@@ -573,9 +616,20 @@ kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int 
   if (layer < 0 || layer >= p->L || head < 0 || head >= p->Hkv || (kv != 0 && kv != 1) || n < 0)
     return fail(KVQ_ERR_INVALID_ARG, "argument out of range");
   const HeadInfo& h = p->head(layer, head);
+  if ((kv ? h.vcodec : h.kcodec) == KVQ_RANK) {
+    ProjParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.k_in = (const __half*)x; pp.in_stride = D;
+    pp.mimg = p->d_Mimg; pp.err = p->d_err;
+    pp.z_out = y; pp.head_override = head; pp.kv_override = kv;
+    pp.total_q = n; pp.Hkv = p->Hkv;
+    for (int hh = 0; hh < p->Hkv; ++hh) pp.heads[hh] = p->head(layer, hh);
+    cudaError_t e = launch_project(pp, (n + 127) / 128, 1, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "projection launch");
+    return KVQ_OK;
+  }
   const float* inv = p->d_inv ? p->d_inv + (((size_t)layer * p->Hkv + head) * 2 + kv) * D : nullptr;
-  const float* M = p->d_M ? p->d_M + h.m_off : nullptr;
-  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, M, n, (const __half*)x, y, (cudaStream_t)stream);
+  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, n, (const __half*)x, y, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "debug_rotate launch");
   return KVQ_OK;
 }

@@ -32,42 +32,19 @@ __device__ __forceinline__ void load_row_f16(const __half* src, float x[4]) {
 // Byte address of a tail ring row's lane piece (8 bytes = 4 fp16 values).
 __device__ __forceinline__ uint8_t* ring_lane_ptr(uint8_t* ring, int slot, int kv) {
   const int lane = threadIdx.x & 31;
-  uint8_t* tp = ring + (size_t)(slot / PAGE) * TAIL_PAGE_BYTES;
-  const int row = slot % PAGE;
-  if (kv == 0) return tp + ((lane >> 1) * PAGE + row) * 16 + (lane & 1) * 8;   // interleaved, cb = 256
-  return tp + PAGE * D * 2 + row * (D * 2) + 8 * lane;                          // row-major
+  uint8_t* tp = ring + (size_t)(slot / TAIL_TOK) * TAIL_PAGE_BYTES;
+  const int row = slot % TAIL_TOK;
+  if (kv == 0) return tp + ((lane >> 1) * TAIL_TOK + row) * 16 + (lane & 1) * 8;   // interleaved, cb = 256
+  return tp + TAIL_TOK * D * 2 + row * (D * 2) + 8 * lane;                          // row-major
 }
 
-// Transform the warp's row into the stored basis (lane: 4 values).  For the
-// projection path the output coordinates 4l..4l+3 (< r) are produced; `scratch`
-// is 128 floats of warp-private shared memory.
-__device__ __forceinline__ void transform_row(float x[4], int codec, int rot, const float* inv_s, const float* M, int r,
-                                              float* scratch) {
+// Transform the warp's row into the stored basis (lane: 4 values): the raw
+// values for F16 and unrotated plans; x * inv_s (variance normalisation) and the
+// staged Hadamard transform otherwise.  The projection (rank codec) runs on the
+// tensor cores in project.cu.
+__device__ __forceinline__ void transform_row(float x[4], int codec, int rot, const float* inv_s) {
   const int lane = threadIdx.x & 31;
-  if (codec == KVQ_F16 || rot == KVQ_ROT_NONE) return;
-  if (codec == KVQ_RANK) {
-    // z_i = sum_c M[i][c] x_c, fp32 (the tensor-core kernel replaces this)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) scratch[4 * lane + i] = x[i];
-    __syncwarp();
-    float z[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < D; c += 4) {
-      float4 xv = *reinterpret_cast<const float4*>(scratch + c);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int o = 4 * lane + i;
-        if (o < r) {
-          float4 m = *reinterpret_cast<const float4*>(M + (size_t)o * D + c);
-          z[i] = fmaf(m.x, xv.x, z[i]); z[i] = fmaf(m.y, xv.y, z[i]);
-          z[i] = fmaf(m.z, xv.z, z[i]); z[i] = fmaf(m.w, xv.w, z[i]);
-        }
-      }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = z[i];
-    return;
-  }
+  if (codec == KVQ_F16 || codec == KVQ_RANK || rot == KVQ_ROT_NONE) return;
   if (rot == KVQ_ROT_VARNORM_HADAMARD) {
     float4 s = *reinterpret_cast<const float4*>(inv_s + 4 * lane);
     x[0] = __fmul_rn(x[0], s.x); x[1] = __fmul_rn(x[1], s.y);
@@ -77,7 +54,6 @@ __device__ __forceinline__ void transform_row(float x[4], int codec, int rot, co
 }
 
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {
-  __shared__ __align__(16) float scratch_all[8][D];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const long gw = (long)blockIdx.x * 8 + wib;
@@ -101,7 +77,8 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
   uint8_t* ring = (T > 0) ? p.tail + (((size_t)sq.seq * p.L + p.layer) * p.Hkv + head) * (size_t)T * (D * 2 * 2)
                           : nullptr;
   const float* inv_s = p.inv_s ? p.inv_s + ((size_t)head * 2 + kv) * D : nullptr;
-  const float* M = p.M ? p.M + h.m_off : nullptr;
+  // rank-codec rows are quantized by the tensor-core kernel, which runs first
+  const bool quantize_here = codec != KVQ_RANK;
 
   int pos;          // position to quantize (-1: none)
   int src_row = -1; // input row index, or -1 when the source is the ring
@@ -124,7 +101,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     write_slot = slot; write_row = sq.in_row0 + (w - sq.len_old);
   }
 
-  if (pos >= 0) {
+  if (pos >= 0 && quantize_here) {
     float x[4];
     if (ring_slot >= 0) {
       uint2 v = *reinterpret_cast<const uint2*>(ring_lane_ptr(ring, ring_slot, kv));
@@ -134,7 +111,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     } else {
       load_row_f16(in + ((size_t)src_row * p.Hkv + head) * D, x);
     }
-    transform_row(x, codec, p.rot, inv_s, M, h.r, scratch_all[wib]);
+    transform_row(x, codec, p.rot, inv_s);
     const int lp = pos / PAGE;
     int pid = p.block_table[(size_t)sq.seq * p.max_pages_per_seq + lp];
     if (pid < 0) {
@@ -209,25 +186,22 @@ cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __ha
 }
 
 // ---------------------------------------------------------------- debug hooks
-__global__ void debug_rotate_kernel(HeadInfo h, int rot, int kv, const float* inv_s, const float* M, int n,
-                                    const __half* x, float* y) {
-  __shared__ __align__(16) float scratch_all[8][D];
+__global__ void debug_rotate_kernel(HeadInfo h, int rot, int kv, const float* inv_s, int n, const __half* x,
+                                    float* y) {
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int row = blockIdx.x * 8 + wib;
   if (row >= n) return;
   const int codec = kv ? h.vcodec : h.kcodec;
   float v[4];
   load_row_f16(x + (size_t)row * D, v);
-  transform_row(v, codec, rot, inv_s, M, h.r, scratch_all[wib]);
-  const int nout = codec == KVQ_RANK ? h.r : D;
+  transform_row(v, codec, rot, inv_s);
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (4 * lane + i < nout) y[(size_t)row * nout + 4 * lane + i] = v[i];
+  for (int i = 0; i < 4; ++i) y[(size_t)row * D + 4 * lane + i] = v[i];
 }
-cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, const float* M, int n,
-                                const __half* x, float* y, cudaStream_t s) {
+cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, int n, const __half* x,
+                                float* y, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  debug_rotate_kernel<<<(n + 7) / 8, 256, 0, s>>>(h, rot, kv, inv_s, M, n, x, y);
+  debug_rotate_kernel<<<(n + 7) / 8, 256, 0, s>>>(h, rot, kv, inv_s, n, x, y);
   note_launches(1);
   return cudaGetLastError();
 }

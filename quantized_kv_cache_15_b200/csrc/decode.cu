@@ -27,7 +27,11 @@
 //   q'.yhat_block = d * sum_j q'_j u_j + off * sum_j q'_j
 // with sum_j q'_j precomputed per block (qsum).
 #include <cfloat>
+#include <map>
+#include <mutex>
+#include <tuple>
 
+#include "decode_fast.cuh"
 #include "kvq_internal.h"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -72,6 +76,11 @@ __device__ __forceinline__ uint32_t kcode_generic(const uint8_t* kp, int cb, int
       uint32_t hi = (kp[kplane_off(cb, t, n / 2 + (j >> 2))] >> (2 * (j & 3))) & 3u;
       return lo | (hi << 4);
     }
+    case 5: {
+      uint32_t lo = (kp[kplane_off(cb, t, j >> 1)] >> (4 * (j & 1))) & 15u;
+      uint32_t hi = (kp[kplane_off(cb, t, n / 2 + (j >> 3))] >> (j & 7)) & 1u;
+      return lo | (hi << 4);
+    }
     case 3: {
       uint32_t lo = (kp[kplane_off(cb, t, j >> 2)] >> (2 * (j & 3))) & 3u;
       uint32_t hi = (kp[kplane_off(cb, t, n / 4 + (j >> 3))] >> (j & 7)) & 1u;
@@ -85,13 +94,14 @@ __device__ __forceinline__ uint32_t kcode_generic(const uint8_t* kp, int cb, int
 template <int G>
 __device__ __forceinline__ void score_token(int kc, int kbits, int n, int cb, int sb, const uint8_t* kp,
                                             const uint8_t* ks, int t, const float* __restrict__ qv,
-                                            const float* __restrict__ qsum, float s[G]) {
+                                            const float* __restrict__ qsum, float s[G], int rows) {
 #pragma unroll
   for (int g = 0; g < G; ++g) s[g] = 0.f;
   if (kc == KVQ_F16) {
+    if (t >= rows) return;                 // past the end of a 32-row tail tile
 #pragma unroll 2
     for (int c = 0; c < 16; ++c) {
-      uint4 v = *reinterpret_cast<const uint4*>(kp + (c * PAGE + t) * 16);
+      uint4 v = *reinterpret_cast<const uint4*>(kp + (c * rows + t) * 16);
       const __half2* hv = reinterpret_cast<const __half2*>(&v);
       float x[8];
 #pragma unroll
@@ -182,6 +192,9 @@ __device__ __forceinline__ void v_lane(int vc, int vbits, int n, int cb, int sb,
       for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> (2 * i)) & 3u) << 4); } break;
     case 3: { uint32_t lo = row[lane]; uint32_t hi = (row[n / 4 + (lane >> 1)] >> (4 * (lane & 1))) & 15u;
       for (int i = 0; i < 4; ++i) u[i] = ((lo >> (2 * i)) & 3u) | (((hi >> i) & 1u) << 2); } break;
+    case 5: { uint32_t lo = *reinterpret_cast<const uint16_t*>(row + 2 * lane);
+      uint32_t hi = (row[n / 2 + (lane >> 1)] >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> i) & 1u) << 4); } break;
     default: u[0] = u[1] = u[2] = u[3] = 0;
   }
   const int blk = n < 32 ? n : 32;
@@ -198,18 +211,24 @@ __device__ __forceinline__ void v_lane(int vc, int vbits, int n, int cb, int sb,
   for (int i = 0; i < 4; ++i) v[i] = fmaf((float)u[i], d, off);
 }
 
+// Shared memory of one CTA.  The stage ring is only read inside the tile loop;
+// afterwards the same bytes hold the warps' merge area and the final
+// accumulators ("post" region).
+__host__ __device__ inline size_t post_bytes(int G) {
+  return (size_t)4 * G * (D + 4) * 4 + (size_t)2 * G * D * 4 + (size_t)2 * G * 4 + 16;
+}
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   size_t ring = (size_t)stage_bytes * n_stages;
-  size_t merge = (size_t)4 * G * (D + 4) * sizeof(float);
-  size_t a = ring > merge ? ring : merge;
+  size_t a = ring > post_bytes(G) ? ring : post_bytes(G);
   a = (a + 127) & ~(size_t)127;
   a += (size_t)G * D * 4;            // qv
   a += (size_t)G * 4 * 4;            // qsum
-  a += (size_t)4 * PAGE * G * 4;     // pbuf
-  a += (size_t)2 * G * D * 4;        // final accumulators (quantized basis, tail)
-  a += (size_t)2 * G * 4 + 16;       // final m, l, flag
-  a += (size_t)4 * D * 4;            // per-warp scratch
+  a += (size_t)G * 4 * 4;            // qsi
+  a += (size_t)8 * 4;                // sq
+  a += (size_t)G * D * 2;            // qi16
+  a += (size_t)2 * G * 64 * 4;       // pair tables
   a = (a + 15) & ~(size_t)15;
+  a += (size_t)4 * 32 * (4 * G + 1) * 8;   // per-warp duplicated weight pairs (also the prologue scratch)
   a += (size_t)2 * 8 * 8;            // mbarriers
   return a;
 }
@@ -262,11 +281,9 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
   const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
   const int seq = p.seq[si], len = p.len[si];
   const int T = p.T;
-  const int nq = len > T ? len - T : 0;
-  const int nt = len < T ? len : T;
-  const int NQP = (nq + PAGE - 1) / PAGE, NTP = (nt + PAGE - 1) / PAGE;
-  const int qsplits = (NQP + p.pps - 1) / p.pps, tsplits = (NTP + p.pps - 1) / p.pps;
-  const int S = qsplits + tsplits;
+  const SplitCounts sc = split_counts(len, T, p.pps);
+  const int nq = sc.nq, nt = sc.nt, NQP = sc.nqp, NTP = sc.ntp, qsplits = sc.qsplits;
+  const int S = sc.qsplits + sc.tsplits;
   float* out_base = p.out + ((size_t)si * p.Hq + (size_t)head * G) * D;
   if (S == 0) {
     if (split == 0)
@@ -288,30 +305,53 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
   const int cbK = is_tail ? 2 * D : h.cbK, sbK = is_tail ? 0 : h.sbK;
   const int cbV = is_tail ? 2 * D : h.cbV, sbV = is_tail ? 0 : h.sbV;
   const uint32_t tile_bytes = is_tail ? (uint32_t)TAIL_PAGE_BYTES : h.bytes;
+  const int rows = is_tail ? TAIL_TOK : PAGE;              // token rows per tile
   const int NS = p.n_stages;
 
   // shared memory carve-up
-  size_t ring = (size_t)p.stage_bytes * NS;
-  size_t merge = (size_t)4 * G * (D + 4) * sizeof(float);
-  size_t off = ((ring > merge ? ring : merge) + 127) & ~(size_t)127;
+  const size_t ring = (size_t)p.stage_bytes * NS;
+  size_t off = ((ring > post_bytes(G) ? ring : post_bytes(G)) + 127) & ~(size_t)127;
   uint8_t* stages = smem;
-  float* mg = reinterpret_cast<float*>(smem);                 // merge area, aliases the ring after the loop
+  // post-loop region (aliases the ring)
+  float* mg = reinterpret_cast<float*>(smem);                      // [4 warps][G][D+4]
+  float* aq = mg + (size_t)4 * G * (D + 4);                        // [G][D] quantized-basis accumulator
+  float* at = aq + (size_t)G * D;                                  // [G][D] tail accumulator
+  float* fm = at + (size_t)G * D;
+  float* fl = fm + G;
+  int* flag = reinterpret_cast<int*>(fl + G);
   float* qv = reinterpret_cast<float*>(smem + off); off += (size_t)G * D * 4;
   float* qsum = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4 * 4;
-  float* pbuf = reinterpret_cast<float*>(smem + off); off += (size_t)4 * PAGE * G * 4;
-  float* aq = reinterpret_cast<float*>(smem + off); off += (size_t)G * D * 4;
-  float* at = reinterpret_cast<float*>(smem + off); off += (size_t)G * D * 4;
-  float* fm = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4;
-  float* fl = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4;
-  int* flag = reinterpret_cast<int*>(smem + off); off += 16;
-  float* scratch = reinterpret_cast<float*>(smem + off); off += (size_t)4 * D * 4;
+  int* qsi = reinterpret_cast<int*>(smem + off); off += (size_t)G * 4 * 4;
+  float* sq = reinterpret_cast<float*>(smem + off); off += (size_t)8 * 4;
+  int16_t* qi16 = reinterpret_cast<int16_t*>(smem + off); off += (size_t)G * D * 2;
+  uint32_t* tab = reinterpret_cast<uint32_t*>(smem + off); off += (size_t)2 * G * 64 * 4;
   off = (off + 15) & ~(size_t)15;
+  uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off); off += (size_t)4 * 32 * (4 * G + 1) * 8;
+  float* scratch = reinterpret_cast<float*>(pw2);                  // prologue only: [4 warps][D]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   uint64_t* empty = full + 8;
 
-  if (threadIdx.x == 0) {
+  // The producer sets up the ring and starts the first NS page loads right away,
+  // so they overlap the query preparation below.
+  const uint8_t* tail_base =
+      is_tail ? p.tail + (((size_t)seq * p.L + p.layer) * p.Hkv + head) * (size_t)T * (D * 2 * 2) : nullptr;
+  auto issue_tile = [&](int i) {
+    const int st = i % NS;
+    const uint8_t* src;
+    if (is_tail) {
+      src = tail_base + (size_t)(pg0 + i) * TAIL_PAGE_BYTES;
+    } else {
+      int pid = p.block_table[(size_t)seq * p.max_pages_per_seq + pg0 + i];
+      if (pid < 0) { atomicOr(p.err, ERR_NO_PAGE); pid = 0; }
+      src = p.pool + (size_t)pid * p.page_bytes + h.off;
+    }
+    mbar_arrive_expect_tx(&full[st], tile_bytes);
+    bulk_g2s(stages + (size_t)st * p.stage_bytes, src, tile_bytes, &full[st]);
+  };
+  if (warp == 4 && lane == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     fence_mbar_init();
+    for (int i = 0; i < NS && i < n_tiles; ++i) issue_tile(i);
   }
 
   // ---- query preparation (consumer warps): q' in the K basis, scaled to log2 units
@@ -360,6 +400,47 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
   }
   __syncthreads();
 
+  // ---- integer query for the block codecs: int16 with one scale per head, exact
+  // integer block sums, and the pair tables of the K codec's code planes
+  const bool kfast = kc != KVQ_F16 && kc != KVQ_RANK;
+  if (kfast) {
+    if (warp < 4) {
+      for (int g = warp; g < G; g += 4) {
+        float x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = qv[g * D + 4 * lane + i];
+        const float amax = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
+        const float scale = amax > 0.f ? amax * (1.0f / 32767.0f) : 1.0f;
+        const float inv = 1.0f / scale;
+        int bs = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int v = __float2int_rn(x[i] * inv);
+          v = max(-32767, min(32767, v));
+          qi16[g * D + 4 * lane + i] = (int16_t)v;
+          bs += v;
+        }
+        bs += __shfl_xor_sync(0xffffffffu, bs, 1);
+        bs += __shfl_xor_sync(0xffffffffu, bs, 2);
+        bs += __shfl_xor_sync(0xffffffffu, bs, 4);
+        if ((lane & 7) == 0) qsi[g * 4 + (lane >> 3)] = bs;
+        if (lane == 0) sq[g] = scale;
+      }
+    }
+    __syncthreads();
+    int tt0, tt1;
+    codec_tables(kc, &tt0, &tt1);
+    for (int idx = threadIdx.x; idx < 2 * G * 64; idx += blockDim.x) {
+      const int plane = idx / (G * 64), rem = idx % (G * 64), g = rem / 64, w = rem % 64;
+      const int type = plane ? tt1 : tt0;
+      if (type < 0) continue;
+      int c0, c1;
+      tab_channels(type, w, c0, c1);
+      tab[idx] = (uint32_t)(uint16_t)qi16[g * D + c0] | ((uint32_t)(uint16_t)qi16[g * D + c1] << 16);
+    }
+    __syncthreads();
+  }
+
   float m[G], l[G], acc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -368,41 +449,52 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
     for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
   }
   if (warp == 4) {
-    // ---- producer
+    // ---- producer: refill each stage once its consumer warp has released it
     if (lane == 0) {
-      const uint8_t* tail_base =
-          is_tail ? p.tail + (((size_t)seq * p.L + p.layer) * p.Hkv + head) * (size_t)T * (D * 2 * 2) : nullptr;
-      for (int i = 0; i < n_tiles; ++i) {
+      for (int i = NS; i < n_tiles; ++i) {
         const int st = i % NS;
-        if (i >= NS && !mbar_wait(&empty[st], ((i / NS) - 1) & 1)) atomicOr(p.err, ERR_TIMEOUT);
-        const uint8_t* src;
-        if (is_tail) {
-          src = tail_base + (size_t)(pg0 + i) * TAIL_PAGE_BYTES;
-        } else {
-          int pid = p.block_table[(size_t)seq * p.max_pages_per_seq + pg0 + i];
-          if (pid < 0) { atomicOr(p.err, ERR_NO_PAGE); pid = 0; }
-          src = p.pool + (size_t)pid * p.page_bytes + h.off;
-        }
-        mbar_arrive_expect_tx(&full[st], tile_bytes);
-        bulk_g2s(stages + (size_t)st * p.stage_bytes, src, tile_bytes, &full[st]);
+        if (!mbar_wait(&empty[st], ((i / NS) - 1) & 1)) atomicOr(p.err, ERR_TIMEOUT);
+        issue_tile(i);
       }
     }
   } else {
     // ---- consumers
-    float* pw = pbuf + warp * PAGE * G;
+    // [32 tokens][4 blocks][G] pairs (w, w); token rows padded by one pair so that the
+    // lanes' stores (one token each) fall in distinct banks
+    constexpr int PWR = 4 * G + 1;
+    uint64_t* pw = pw2 + (size_t)warp * 32 * PWR;
+    const int vmode = (vc == KVQ_F16 || vc == KVQ_RANK) ? 0 : (vbits == 8 || vbits == 4 || vbits == 2) ? vbits : 0;
+    const bool vasym = codec_is_asym(vc);
+    const int vhalf = (vc == KVQ_F16 || vc == KVQ_RANK) ? 0 : (1 << (vbits - 1));
+    const int blane = ((4 * lane) / (nV < 32 ? nV : 32)) & 3;
+    uint64_t A[G][2];
+    float O[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      A[g][0] = 0ull; A[g][1] = 0ull;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) O[g][b] = 0.f;
+    }
     for (int i = warp; i < n_tiles; i += 4) {
       const int st = i % NS;
       if (!mbar_wait(&full[st], (i / NS) & 1)) atomicOr(p.err, ERR_TIMEOUT);
       const uint8_t* sp = stages + (size_t)st * p.stage_bytes;
       const uint8_t* kp = sp;
-      const uint8_t* ks = kp + PAGE * cbK;
-      const uint8_t* vp = ks + PAGE * sbK;
-      const uint8_t* vs = vp + PAGE * cbV;
-      const int tok0 = (pg0 + i) * PAGE;
-      const int nvalid = min(PAGE, seg_tokens - tok0);
+      const uint8_t* ks = kp + rows * cbK;
+      const uint8_t* vp = ks + rows * sbK;
+      const uint8_t* vs = vp + rows * cbV;
+      const int tok0 = (pg0 + i) * rows;
+      const int nvalid = min(rows, seg_tokens - tok0);
       float s0[G], s1[G];
-      score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0);
-      score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1);
+      if (kfast) {
+        score2_block_codec<G>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1);
+#pragma unroll
+        for (int g = 0; g < G; ++g) { s0[g] *= sq[g]; s1[g] *= sq[g]; }
+      } else {
+        score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0, rows);
+        score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1, rows);
+      }
+      float p0[G], p1[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         if (lane >= nvalid) s0[g] = -INFINITY;
@@ -410,30 +502,81 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
         const float tmax = warp_max(fmaxf(s0[g], s1[g]));
         const float mnew = fmaxf(m[g], tmax);
         const float alpha = exp2f(m[g] - mnew);
-        const float p0 = exp2f(s0[g] - mnew), p1 = exp2f(s1[g] - mnew);
-        l[g] = l[g] * alpha + (p0 + p1);
+        p0[g] = exp2f(s0[g] - mnew);
+        p1[g] = exp2f(s1[g] - mnew);
+        l[g] = l[g] * alpha + (p0[g] + p1[g]);
+        const uint64_t a2 = pack2(alpha, alpha);
+        A[g][0] = mul2(A[g][0], a2);
+        A[g][1] = mul2(A[g][1], a2);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[g][c] *= alpha;
+        for (int b = 0; b < 4; ++b) O[g][b] *= alpha;
         m[g] = mnew;
-        pw[lane * G + g] = p0;
-        pw[(lane + 32) * G + g] = p1;
       }
-      __syncwarp();
-      for (int t = 0; t < nvalid; ++t) {
-        float v[4];
-        v_lane(vc, vbits, nV, cbV, sbV, vp, vs, t, lane, v);
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float w = pw[t * G + g];
+      for (int half = 0; half < 2; ++half) {
+        // the owner of token (lane + 32*half) publishes w = p*d per block (fast V) or p
+        const int t = lane + 32 * half;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) acc[g][c] = fmaf(w, v[c], acc[g][c]);
+        for (int b = 0; b < 4; ++b) {
+          float d = 1.f, off = 0.f;
+          if (vmode && t < nvalid) {
+            if (vasym) {
+              const __half2 dm = *reinterpret_cast<const __half2*>(vs + t * sbV + 4 * b);
+              d = __low2float(dm);
+              off = __high2float(dm);
+            } else {
+              d = __half2float(*reinterpret_cast<const __half*>(vs + t * sbV + 2 * b));
+              off = -(float)vhalf * d;
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float pg = half ? p1[g] : p0[g];
+            const float w = pg * d;
+            pw[(size_t)lane * PWR + b * G + g] = pack2(w, w);
+            O[g][b] = fmaf(pg, off, O[g][b]);
+          }
         }
+        __syncwarp();
+        const int ntok = min(32, nvalid - 32 * half);
+        for (int tt = 0; tt < ntok; ++tt) {
+          const int t2 = 32 * half + tt;
+          uint64_t u01, u23;
+          if (vmode) {
+            v_codes_fast(vmode, vp + t2 * cbV, lane, u01, u23);
+          } else {
+            float v[4];
+            v_lane(vc, vbits, nV, cbV, sbV, vp, vs, t2, lane, v);
+            u01 = pack2(v[0], v[1]);
+            u23 = pack2(v[2], v[3]);
+          }
+          const uint64_t* wrow = pw + (size_t)tt * PWR + blane * G;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint64_t w2 = wrow[g];
+            A[g][0] = fma2(w2, u01, A[g][0]);
+            A[g][1] = fma2(w2, u23, A[g][1]);
+          }
+        }
+        __syncwarp();
       }
-      __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g) l[g] = warp_sum(l[g]);
+    for (int g = 0; g < G; ++g) {
+      l[g] = warp_sum(l[g]);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) O[g][b] = warp_sum(O[g][b]);
+      float a[4];
+      unpack2(A[g][0], a[0], a[1]);
+      unpack2(A[g][1], a[2], a[3]);
+#pragma unroll
+      float ob = O[g][0];                 // O[g][blane] without a dynamic register index
+#pragma unroll
+      for (int b = 1; b < 4; ++b) ob = (b == blane) ? O[g][b] : ob;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[g][c] = a[c] * (1.0f / v_position_factor(vmode, c)) + ob;
+    }
   }
   __syncthreads();   // every stage consumed: the ring is reused as the merge area below
   if (warp < 4) {
@@ -496,30 +639,41 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
   __syncthreads();
   if (!flag[0]) return;
   __threadfence();
-  // ---- last CTA: merge every split in order
+  // ---- last CTA: merge every split (fixed order, deterministic).  One warp per
+  // head reduces the split maxima and sums with shuffles and keeps the factors
+  // 2^(m_s - M); then every thread sums its outputs' partials with independent loads.
   const float* base = p.ws + (((size_t)si * p.Hkv + head) * MAX_SPLITS) * G * PARTIAL_FLOATS;
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS));
-    float L = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float* ps = base + ((size_t)s * G + g) * PARTIAL_FLOATS;
-      const float ms = __ldcg(ps);
-      if (ms != -INFINITY) L += exp2f(ms - M) * __ldcg(ps + 1);
+  float* fsc = mg;                                                  // [G][MAX_SPLITS]
+  int* kinds = reinterpret_cast<int*>(mg + (size_t)G * MAX_SPLITS); // [MAX_SPLITS]
+  for (int g = warp; g < G; g += (int)(blockDim.x >> 5)) {
+    float ms[2], ls[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s = lane + 32 * k;
+      ms[k] = s < S ? __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS) : -INFINITY;
+      ls[k] = s < S ? __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS + 1) : 0.f;
     }
-    fm[g] = M; fl[g] = L;
+    const float M = warp_max(fmaxf(ms[0], ms[1]));
+    float part = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s = lane + 32 * k;
+      const float f = (ms[k] == -INFINITY) ? 0.f : exp2f(ms[k] - M);
+      if (s < S) fsc[g * MAX_SPLITS + s] = f;
+      part += f * ls[k];
+    }
+    const float L = warp_sum(part);
+    if (lane == 0) { fm[g] = M; fl[g] = L; }
   }
+  for (int s = threadIdx.x; s < S; s += blockDim.x) kinds[s] = __ldcg(base + (size_t)s * G * PARTIAL_FLOATS + 2) != 0.f;
   __syncthreads();
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
     const int g = idx / D, c = idx % D;
-    const float M = fm[g];
     float Aq = 0.f, At = 0.f;
+#pragma unroll 8
     for (int s = 0; s < S; ++s) {
-      const float* ps = base + ((size_t)s * G + g) * PARTIAL_FLOATS;
-      const float ms = __ldcg(ps);
-      if (ms == -INFINITY) continue;
-      const float f = exp2f(ms - M) * __ldcg(ps + 4 + c);
-      if (__ldcg(ps + 2) != 0.f) At += f; else Aq += f;
+      const float v = __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS + 4 + c) * fsc[g * MAX_SPLITS + s];
+      if (kinds[s]) At += v; else Aq += v;
     }
     aq[idx] = Aq;
     at[idx] = At;
@@ -535,16 +689,51 @@ int decode_max_smem() { return 227 * 1024; }
 template <int G>
 static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
   const size_t smem = decode_smem_bytes(p.stage_bytes, p.n_stages, G);
-  static size_t configured = 0;
-  if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = smem;
-  }
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(grid_x, p.Hkv, p.n_seqs);
   decode_kernel<G><<<grid, 160, smem, s>>>(p);
   note_launches(1);
   return cudaGetLastError();
+}
+
+// Resident CTAs per SM of the kernel for G heads with `smem` dynamic bytes (registers,
+// shared memory and the thread limit all counted), 0 on error.
+template <int G>
+static int blocks_per_sm_g(size_t smem) {
+  if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G>, 160, smem) != cudaSuccess) return 0;
+  return n;
+}
+
+static int blocks_per_sm_uncached(int G, size_t smem) {
+  switch (G) {
+    case 1: return blocks_per_sm_g<1>(smem);
+    case 2: return blocks_per_sm_g<2>(smem);
+    case 3: return blocks_per_sm_g<3>(smem);
+    case 4: return blocks_per_sm_g<4>(smem);
+    case 5: return blocks_per_sm_g<5>(smem);
+    case 6: return blocks_per_sm_g<6>(smem);
+    case 7: return blocks_per_sm_g<7>(smem);
+    case 8: return blocks_per_sm_g<8>(smem);
+    default: return 0;
+  }
+}
+
+int decode_blocks_per_sm(int G, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, size_t>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(dev, G, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  const int n = blocks_per_sm_uncached(G, smem);
+  if (n > 0) cache[key] = n;
+  return n;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int grid_x, cudaStream_t s) {

@@ -26,6 +26,9 @@ __device__ __forceinline__ void lane_codes(const uint8_t* plane, int cb, int t, 
       for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> (2 * i)) & 3u) << 4); } break;
     case 3: { uint32_t lo = at(lane); uint32_t hi = (at(n / 4 + (lane >> 1)) >> (4 * (lane & 1))) & 15u;
       for (int i = 0; i < 4; ++i) u[i] = ((lo >> (2 * i)) & 3u) | (((hi >> i) & 1u) << 2); } break;
+    case 5: { uint32_t lo = at(2 * lane) | (at(2 * lane + 1) << 8);
+      uint32_t hi = (at(n / 2 + (lane >> 1)) >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> i) & 1u) << 4); } break;
     default: u[0] = u[1] = u[2] = u[3] = 0;
   }
 }
@@ -50,9 +53,10 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
     // tail ring, raw fp16
     const uint8_t* ring = p.tail + (((size_t)seq * p.L + p.layer) * p.Hkv + head) * (size_t)T * (D * 2 * 2);
     const int slot = (int)(pos % T);
-    const uint8_t* tp = ring + (size_t)(slot / PAGE) * TAIL_PAGE_BYTES;
-    const int r = slot % PAGE;
-    const uint8_t* src = kv == 0 ? tp + ((lane >> 1) * PAGE + r) * 16 + (lane & 1) * 8 : tp + PAGE * D * 2 + r * (D * 2) + 8 * lane;
+    const uint8_t* tp = ring + (size_t)(slot / TAIL_TOK) * TAIL_PAGE_BYTES;
+    const int r = slot % TAIL_TOK;
+    const uint8_t* src = kv == 0 ? tp + ((lane >> 1) * TAIL_TOK + r) * 16 + (lane & 1) * 8
+                                 : tp + TAIL_TOK * D * 2 + r * (D * 2) + 8 * lane;
     uint2 w = *reinterpret_cast<const uint2*>(src);
     float2 a = __half22float2(*reinterpret_cast<__half2*>(&w.x));
     float2 b = __half22float2(*reinterpret_cast<__half2*>(&w.y));

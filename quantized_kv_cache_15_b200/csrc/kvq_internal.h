@@ -13,8 +13,9 @@
 //   V codes : 64 rows of cbV bytes, row-major (lanes split one row's channels).
 //   V scales: 64 rows of sbV bytes, row-major.
 // Canonical packed rows (codes then scales) are defined by the quantizer: see
-// quant.cuh.  The tail ring of (seq, layer, kv head) is T/64 tail pages of
-// 32 KiB: [K fp16, interleaved as above with cb = 256][V fp16 row-major];
+// quant.cuh.  The tail ring of (seq, layer, kv head) is T/32 tail pages of
+// 16 KiB, each 32 token slots: [K fp16, interleaved as above but with 32 rows:
+// byte i of slot t at ((i / 16) * 32 + t) * 16 + i % 16][V fp16 row-major];
 // token position p lives in ring slot p % T.
 #pragma once
 
@@ -32,8 +33,24 @@ constexpr int MAX_HKV = KVQ_MAX_KV_HEADS;
 constexpr int MAX_G = KVQ_MAX_GQA;
 constexpr int MAX_BATCH = KVQ_MAX_BATCH;
 constexpr int MAX_SPLITS = 64;            // split-K pieces per (sequence, kv head)
-constexpr int TAIL_PAGE_BYTES = PAGE * D * 2 * 2;
+constexpr int TAIL_TOK = 32;                 // token slots per tail page
+constexpr int TAIL_PAGE_BYTES = TAIL_TOK * D * 2 * 2;   // 16 KiB: K fp16 (interleaved) then V fp16
 constexpr int PARTIAL_FLOATS = 4 + D;     // m, l, kind, pad, acc[128]
+
+// Split-K layout of one sequence of `len` tokens, shared by the host (grid size)
+// and the decode kernel: the quantized segment in 64-token pages, the tail
+// segment in 32-token tail pages, each cut into splits of `pps` pages.
+struct SplitCounts { int nq, nt, nqp, ntp, qsplits, tsplits; };
+__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps) {
+  SplitCounts c;
+  c.nq = len > T ? len - T : 0;
+  c.nt = len < T ? len : T;
+  c.nqp = (c.nq + PAGE - 1) / PAGE;
+  c.ntp = (c.nt + TAIL_TOK - 1) / TAIL_TOK;
+  c.qsplits = (c.nqp + pps - 1) / pps;
+  c.tsplits = (c.ntp + pps - 1) / pps;
+  return c;
+}
 
 // Device error word bits.
 constexpr int ERR_NO_PAGE = 1;
@@ -49,20 +66,21 @@ struct HeadInfo {                // one (layer, kv head); 32 bytes
   uint32_t off;                  // region offset inside a page
   uint32_t bytes;                // region bytes = 64 * (cbK + sbK + cbV + sbV)
   uint32_t m_off;                // float offset of M_h (r x 128) in the projection table
-  uint32_t pad2;
+  uint32_t mimg_off;             // byte offset of M_h's fp16 hi/lo tensor-core images
 };
 
 __host__ __device__ inline int codec_bits(int c) {
   switch (c) {
     case KVQ_Q8_0: case KVQ_Q8_1: return 8;
     case KVQ_Q6_0: case KVQ_Q6_1: return 6;
+    case KVQ_Q5_0: case KVQ_Q5_1: return 5;
     case KVQ_Q4_0: case KVQ_Q4_1: return 4;
     case KVQ_Q3_0: case KVQ_Q3_1: return 3;
     case KVQ_Q2_0: case KVQ_Q2_1: return 2;
     default: return 16;
   }
 }
-__host__ __device__ inline bool codec_is_asym(int c) { return c >= KVQ_Q8_1 && c <= KVQ_Q2_1; }
+__host__ __device__ inline bool codec_is_asym(int c) { return (c >= KVQ_Q8_1 && c <= KVQ_Q2_1) || c == KVQ_Q5_1; }
 __host__ __device__ inline int interleave_w(int cb) {
   return (cb % 16 == 0) ? 16 : (cb % 8 == 0) ? 8 : (cb % 4 == 0) ? 4 : 2;
 }
@@ -84,6 +102,7 @@ struct AppendSeq {
   int len_old;    // tokens in this layer before the call
   int in_row0;    // first input row of this sequence
   int item0;      // first work item of this sequence
+  int qitem0;     // first quantize item (E or P) of this sequence, over all sequences
   int nE, nP, nF; // evicted-from-tail, pass-through, final-tail-occupant counts
   int e0, f0;     // first evicted position, first final tail position
 };
@@ -104,6 +123,28 @@ struct AppendParams {
   int* err;
   int n_seqs;
   int total_items;
+  HeadInfo heads[MAX_HKV];
+  AppendSeq seqs[MAX_APPEND_SEQS];
+};
+
+// Projection path (tcgen05): quantize items E and P of an append, or (z_out set)
+// export z = M_h x for rows of k_in.
+struct ProjParams {
+  uint8_t* pool;
+  uint32_t page_bytes;
+  const int* block_table;
+  int max_pages_per_seq;
+  uint8_t* tail;
+  int T, L, layer, Hkv;
+  const __half* k_in;
+  const __half* v_in;
+  int in_stride;                 // halves between consecutive input rows
+  const uint8_t* mimg;           // hi/lo fp16 images of every head
+  int* err;
+  float* z_out;                  // inspection: z rows [total_q][r] (one head, one kv)
+  int head_override, kv_override;
+  int n_seqs;
+  int total_q;                   // quantize items over all sequences
   HeadInfo heads[MAX_HKV];
   AppendSeq seqs[MAX_APPEND_SEQS];
 };
@@ -138,14 +179,16 @@ struct DecodeParams {
 // ---------------------------------------------------------------- launchers (host)
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_block_table_update(int* table, int n, const int* idx_host, const int* val_host, cudaStream_t s);
+int decode_blocks_per_sm(int G, size_t smem_bytes);
 cudaError_t launch_decode(const DecodeParams& p, int grid_x, cudaStream_t s);
 cudaError_t launch_dequantize(const DecodeParams& p, int seq, int64_t t0, int64_t t1, float* k_out, float* v_out,
                               cudaStream_t s);
 cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t t1, int kv, uint8_t* codes,
                              uint8_t* scales, cudaStream_t s);
+cudaError_t launch_project(const ProjParams& p, int n_tiles, int n_heads, cudaStream_t s);
 cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __half* x, float* inv, cudaStream_t s);
-cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, const float* M, int n,
-                                const __half* x, float* y, cudaStream_t s);
+cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, int n, const __half* x,
+                                float* y, cudaStream_t s);
 cudaError_t launch_debug_quantize(int codec, int r, int b, int n, const float* y, uint8_t* codes, uint8_t* scales,
                                   cudaStream_t s);
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G);

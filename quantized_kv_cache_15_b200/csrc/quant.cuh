@@ -21,7 +21,8 @@
 //   rank : d = fp16_rn(min(amax / (2^(b-1) - 1/2), 65504));
 //          u = clamp(floor(x * (1/d)), -2^(b-1), 2^(b-1)-1) + 2^(b-1); d == 0 -> u = 2^(b-1).
 // Canonical packed row: b = 8 one byte per value; 4, 2, 1 bit fields LSB-first;
-// 6 bits = 4-bit plane (n/2 bytes) then 2-bit plane (n/4); 3 bits = 2-bit plane
+// 6 bits = 4-bit plane (n/2 bytes) then 2-bit plane (n/4); 5 bits = 4-bit plane
+// then 1-bit plane (n/8); 3 bits = 2-bit plane
 // (n/4) then 1-bit plane (n/8).  Scales: _0 and rank d_0..d_{nb-1}; _1 pairs
 // (d_k, m_k).  F16: the fp16 values.
 #pragma once
@@ -159,6 +160,13 @@ __device__ __forceinline__ LanePieces pack_lane(uint32_t u, int bits, int n, int
     p.val[0] = (u0 & 15) | ((u1 & 15) << 4) | ((u2 & 15) << 8) | ((u3 & 15) << 12);
     p.off[1] = n / 2 + lane; p.len[1] = 1;
     p.val[1] = (u0 >> 4) | ((u1 >> 4) << 2) | ((u2 >> 4) << 4) | ((u3 >> 4) << 6);
+  } else if (bits == 5) {
+    p.n = 2;
+    p.off[0] = 2 * lane; p.len[0] = 2;
+    p.val[0] = (u0 & 15) | ((u1 & 15) << 4) | ((u2 & 15) << 8) | ((u3 & 15) << 12);
+    uint32_t nib = nib1(u0 >> 4, u1 >> 4, u2 >> 4, u3 >> 4);
+    uint32_t other = __shfl_xor_sync(0xffffffffu, nib, 1);
+    p.off[1] = n / 2 + (lane >> 1); p.len[1] = (lane & 1) ? 0 : 1; p.val[1] = nib | (other << 4);
   } else if (bits == 3) {
     p.n = 2;
     p.off[0] = lane; p.len[0] = 1;

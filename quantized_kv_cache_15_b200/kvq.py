@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
-F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK = range(12)
+F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK, Q5_0, Q5_1 = range(14)
 ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION = range(4)
 HEAD_DIM = 128
 PAGE_TOKENS = 64

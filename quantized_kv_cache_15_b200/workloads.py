@@ -26,7 +26,7 @@ D = 128
 M32 = 0xFFFFFFFF
 
 # codec ids (same numbering as include/kvq.h)
-F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK = range(12)
+F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK, Q5_0, Q5_1 = range(14)
 ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION = range(4)
 
 RANKS = (16, 32, 64, 96, 128)
