@@ -167,6 +167,30 @@ kvq_status kvq_decode_attention(kvq_plan* plan, int layer, int n_seqs, const int
                                 const void* q, float* out, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
+/* Decode attention without any allocation, for callers that cannot allocate
+ * device memory (no counterpart in the pages: this is a deployment variant of
+ * kvq_decode_attention).  Some callers cannot supply a workspace: runtimes
+ * without an allocator, hosts whose memory pool owns every byte of device
+ * memory and cannot lend a slice to a library, and loops that must never call
+ * cudaMalloc because it can synchronise the device.  This entry point computes
+ * exactly what kvq_decode_attention computes, with the same arguments except the
+ * workspace: its split-K scratch is a fixed device array of
+ * KVQ_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *  - Calls needing more scratch than that (kvq_plan_workspace_bytes(plan, n_seqs)
+ *    above the limit) return KVQ_ERR_CAPACITY before enqueueing anything.
+ *  - The first call on a device looks the array's device address up (with that
+ *    device current); make that first call before any stream capture.
+ *  - The entry point allocates nothing (no cudaMalloc/cudaFree, no allocating
+ *    library routine); it zeroes the array's merge counters with an async
+ *    memset on `stream` at every call.
+ *  - Every call shares the one array: calls that may overlap on the GPU (other
+ *    streams, other threads, other plans on the same device) race and must be
+ *    serialised by the caller. */
+#define KVQ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+kvq_status kvq_decode_attention_noalloc(kvq_plan* plan, int layer, int n_seqs, const int* seq_ids /*host*/,
+                                        const void* q, float* out, void* stream);
+
 /* Reconstruct cached rows t0 .. t1-1 of one sequence and layer in the ORIGINAL
  * basis (inverse rotation / projection applied; tail rows copied).
  *  k_out, v_out: device fp32 [t1-t0][n_kv_heads][128] (either may be NULL). */

@@ -522,6 +522,26 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   return KVQ_OK;
 }
 
+kvq_status kvq_decode_attention_noalloc(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const void* q,
+                                        float* out, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
+  const size_t need = workspace_bytes(p, n_seqs);
+  if (need > NOALLOC_SCRATCH_BYTES)
+    return fail(KVQ_ERR_CAPACITY, "decode of %d sequences needs %zu bytes of scratch; the built-in array holds %zu "
+                "(use kvq_decode_attention with a workspace)", n_seqs, need, NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "scratch address lookup");
+  // merge counters must start at zero (partials are written before they are read)
+  const size_t tickets = (size_t)n_seqs * p->Hkv * sizeof(int);
+  if (tickets) {
+    e = cudaMemsetAsync((char*)scratch + (need - tickets), 0, tickets, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "scratch counter reset");
+  }
+  return kvq_decode_attention(p, layer, n_seqs, seq_ids, q, out, scratch, NOALLOC_SCRATCH_BYTES, stream);
+}
+
 kvq_status kvq_dequantize(const kvq_plan* p, int layer, int seq_id, int64_t t0, int64_t t1, float* k_out,
                           float* v_out, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");

@@ -192,6 +192,8 @@ cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float*
 cudaError_t launch_debug_quantize(int codec, int r, int b, int n, const float* y, uint8_t* codes, uint8_t* scales,
                                   cudaStream_t s);
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G);
+constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)16 << 20;   // = KVQ_NOALLOC_SCRATCH_BYTES
+cudaError_t noalloc_scratch(void** out);
 void note_launches(int n);   // counts kernel launches made by the library
 int decode_max_smem();
 

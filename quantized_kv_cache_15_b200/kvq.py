@@ -21,6 +21,7 @@ F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK, Q5_0, Q5_
 ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION = range(4)
 HEAD_DIM = 128
 PAGE_TOKENS = 64
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED", 3: "KVQ_ERR_CAPACITY",
           4: "KVQ_ERR_OOM", 5: "KVQ_ERR_CUDA", 6: "KVQ_ERR_DEVICE", 7: "KVQ_ERR_TIMEOUT", 8: "KVQ_ERR_STATE"}
@@ -36,6 +37,7 @@ SIGNATURES = {
     "kvq_cache_bind": (_I, [_P, _P, _SZ]),
     "kvq_append_quantize": (_I, [_P, _I, _I, _IP, _IP, _P, _P, _P]),
     "kvq_decode_attention": (_I, [_P, _I, _I, _IP, _P, _P, _P, _SZ, _P]),
+    "kvq_decode_attention_noalloc": (_I, [_P, _I, _I, _IP, _P, _P, _P]),
     "kvq_dequantize": (_I, [_P, _I, _I, _I64, _I64, _P, _P, _P]),
     "kvq_row_bytes": (_I, [_P, _I, _I, _I, _IP, _IP]),
     "kvq_read_rows": (_I, [_P, _I, _I, _I64, _I64, _I, _P, _P, _P]),
@@ -182,6 +184,11 @@ class Plan:
         _check(lib().kvq_decode_attention(self._h, layer, len(seq_ids), _ints(seq_ids), _ptr(q), _ptr(out),
                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _stream(stream)))
+
+    def decode_noalloc(self, layer: int, seq_ids, q: torch.Tensor, out: torch.Tensor, stream=None):
+        """Decode attention using the library's built-in scratch array (no workspace)."""
+        _check(lib().kvq_decode_attention_noalloc(self._h, layer, len(seq_ids), _ints(seq_ids), _ptr(q), _ptr(out),
+                                                  _stream(stream)))
 
     def dequantize(self, layer: int, seq: int, t0: int, t1: int, k_out=None, v_out=None, stream=None):
         _check(lib().kvq_dequantize(self._h, layer, seq, t0, t1, _ptr(k_out), _ptr(v_out), _stream(stream)))
