@@ -223,6 +223,21 @@ kvq_status kvq_seq_reset(kvq_plan* plan, int seq_id);
 kvq_status kvq_calibrate_varnorm(int64_t n_tokens, int n_channels, int64_t row_stride, const void* x,
                                  float* inv_rms, void* stream);
 
+/* KV-COBRA rank/bit allocation, run once at calibration [KV-COBRA explainer,
+ * §The news: steps C1 and C2; §Where the bits actually go].  For each head the
+ * error of keeping rank r at b bits is the variance of the dropped directions
+ * plus eps[b-1] times the variance of the kept ones (eps: relative rounding
+ * noise of the b-bit rank quantizer, b = 1..4, measured by the caller).  Every
+ * head starts at (16, 1); the budget of round(bpd * 128 * n_heads) bits is then
+ * handed out one upgrade at a time to the head whose affordable upgrade removes
+ * the most error per extra bit (ties: lower head index, then fewer bits).
+ *  lambdas: host [n_heads][128] direction variances, each row non-increasing.
+ *  ranks, bits: host [n_heads] outputs (r in {16,32,64,96,128}, b in 1..4).
+ *  bits_used: host, may be NULL.  Host-only: touches no device.
+ * KVQ_ERR_CAPACITY if the budget is below 16 bits per head. */
+kvq_status kvq_cobra_allocate(int n_heads, const double* lambdas, double bpd, const double* eps, int* ranks,
+                              int* bits, int* bits_used);
+
 /* Synchronise `stream`, read and clear the plan's device error word. */
 kvq_status kvq_check_device_error(kvq_plan* plan, void* stream);
 

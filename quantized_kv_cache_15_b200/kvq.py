@@ -47,6 +47,7 @@ SIGNATURES = {
     "kvq_check_device_error": (_I, [_P, _P]),
     "kvq_last_error": (ctypes.c_char_p, []),
     "kvq_launch_count": (_I, [ctypes.POINTER(ctypes.c_uint64)]),
+    "kvq_cobra_allocate": (_I, [_I, _P, ctypes.c_double, _P, _IP, _IP, _IP]),
     "kvq_debug_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "kvq_debug_quantize_f32": (_I, [_I, _I, _I, _I, _P, _P, _P, _P]),
 }
@@ -215,6 +216,21 @@ class Plan:
 
     def debug_rotate(self, layer: int, head: int, kv: int, x: torch.Tensor, y: torch.Tensor, stream=None):
         _check(lib().kvq_debug_rotate(self._h, layer, head, kv, x.shape[0], _ptr(x), _ptr(y), _stream(stream)))
+
+
+def cobra_allocate(lambdas: np.ndarray, bpd: float, eps) -> tuple:
+    """Per-head (ranks, bits, bits used) for direction variances lambdas [n][128]."""
+    lam = np.ascontiguousarray(lambdas, np.float64)
+    e = np.ascontiguousarray(eps, np.float64)
+    n = lam.shape[0]
+    r = np.zeros(n, np.int32)
+    b = np.zeros(n, np.int32)
+    used = ctypes.c_int()
+    st = lib().kvq_cobra_allocate(n, lam.ctypes.data_as(_P), float(bpd), e.ctypes.data_as(_P),
+                                  r.ctypes.data_as(_IP), b.ctypes.data_as(_IP), ctypes.byref(used))
+    if st != 0:
+        raise KVQError(st, "kvq_cobra_allocate: invalid spectra, bpd or budget")
+    return r, b, used.value
 
 
 def launch_count() -> int:
