@@ -219,7 +219,10 @@ __host__ __device__ inline size_t post_bytes(int G) {
 }
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   size_t ring = (size_t)stage_bytes * n_stages;
-  size_t a = ring > post_bytes(G) ? ring : post_bytes(G);
+  // after the loop the ring's bytes hold the post region and at least one head's
+  // staged partials (MAX_SPLITS of them) for the last CTA's merge
+  const size_t post_and_stage = ((post_bytes(G) + 127) & ~(size_t)127) + (size_t)MAX_SPLITS * PARTIAL_FLOATS * 4;
+  size_t a = ring > post_and_stage ? ring : post_and_stage;
   a = (a + 127) & ~(size_t)127;
   a += (size_t)G * D * 4;            // qv
   a += (size_t)G * 4 * 4;            // qsum
@@ -229,7 +232,7 @@ size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   a += (size_t)2 * G * 64 * 4;       // pair tables
   a = (a + 15) & ~(size_t)15;
   a += (size_t)4 * 32 * (4 * G + 1) * 8;   // per-warp duplicated weight pairs (also the prologue scratch)
-  a += (size_t)2 * 8 * 8;            // mbarriers
+  a += (size_t)(2 * 8 + 2) * 8;      // mbarriers: ring full / empty, merge staging
   return a;
 }
 
@@ -275,7 +278,7 @@ __device__ void finalize(const DecodeParams& p, const HeadInfo& h, int vbasis, i
 }
 
 template <int G>
-__global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
@@ -310,7 +313,8 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
 
   // shared memory carve-up
   const size_t ring = (size_t)p.stage_bytes * NS;
-  size_t off = ((ring > post_bytes(G) ? ring : post_bytes(G)) + 127) & ~(size_t)127;
+  const size_t post_and_stage = ((post_bytes(G) + 127) & ~(size_t)127) + (size_t)MAX_SPLITS * PARTIAL_FLOATS * 4;
+  size_t off = ((ring > post_and_stage ? ring : post_and_stage) + 127) & ~(size_t)127;
   uint8_t* stages = smem;
   // post-loop region (aliases the ring)
   float* mg = reinterpret_cast<float*>(smem);                      // [4 warps][G][D+4]
@@ -330,6 +334,7 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
   float* scratch = reinterpret_cast<float*>(pw2);                  // prologue only: [4 warps][D]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   uint64_t* empty = full + 8;
+  uint64_t* mmerge = full + 16;                                    // the merge's two staging buffers
 
   // The producer sets up the ring and starts the first NS page loads right away,
   // so they overlap the query preparation below.
@@ -350,10 +355,13 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
   };
   if (warp == 4 && lane == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(&mmerge[0], 1);
+    mbar_init(&mmerge[1], 1);
     fence_mbar_init();
     for (int i = 0; i < NS && i < n_tiles; ++i) issue_tile(i);
   }
 
+  const bool kfast = kc != KVQ_F16 && kc != KVQ_RANK;
   // ---- query preparation (consumer warps): q' in the K basis, scaled to log2 units
   if (warp < 4) {
     float* tmp = scratch + warp * D;
@@ -396,19 +404,9 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
       float ssum = (x[0] + x[1]) + (x[2] + x[3]);
       for (int m = 1; m < blk / 4; m <<= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, m);
       if (4 * lane < nK && ((4 * lane) % blk) == 0) qsum[g * 4 + (4 * lane) / blk] = ssum;
-    }
-  }
-  __syncthreads();
-
-  // ---- integer query for the block codecs: int16 with one scale per head, exact
-  // integer block sums, and the pair tables of the K codec's code planes
-  const bool kfast = kc != KVQ_F16 && kc != KVQ_RANK;
-  if (kfast) {
-    if (warp < 4) {
-      for (int g = warp; g < G; g += 4) {
-        float x[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = qv[g * D + 4 * lane + i];
+      if (kfast) {
+        // integer query for the block codecs: int16 with one scale per head and
+        // exact integer block sums
         const float amax = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
         const float scale = amax > 0.f ? amax * (1.0f / 32767.0f) : 1.0f;
         const float inv = 1.0f / scale;
@@ -427,7 +425,11 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
         if (lane == 0) sq[g] = scale;
       }
     }
-    __syncthreads();
+  }
+  __syncthreads();
+
+  // ---- pair tables of the K codec's code planes (block codecs)
+  if (kfast) {
     int tt0, tt1;
     codec_tables(kc, &tt0, &tt1);
     for (int idx = threadIdx.x; idx < 2 * G * 64; idx += blockDim.x) {
@@ -459,22 +461,30 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
     }
   } else {
     // ---- consumers
-    // [32 tokens][4 blocks][G] pairs (w, w); token rows padded by one pair so that the
-    // lanes' stores (one token each) fall in distinct banks
-    constexpr int PWR = 4 * G + 1;
-    uint64_t* pw = pw2 + (size_t)warp * 32 * PWR;
-    const int vmode = (vc == KVQ_F16 || vc == KVQ_RANK) ? 0 : (vbits == 8 || vbits == 4 || vbits == 2) ? vbits : 0;
-    const bool vasym = codec_is_asym(vc);
-    const int vhalf = (vc == KVQ_F16 || vc == KVQ_RANK) ? 0 : (1 << (vbits - 1));
-    const int blane = ((4 * lane) / (nV < 32 ? nV : 32)) & 3;
-    uint64_t A[G][2];
-    float O[G][4];
+    // Per warp: online-softmax state (m, l per head) and the fp32 value accumulators
+    // of the lane's 4 channels 4*lane .. 4*lane+3, as two packed pairs per head.  On
+    // the integer value path the block offsets of the lane's own tokens (weight x
+    // (-2^(b-1) d) or weight x m) go into off[g][block] and are summed over the warp
+    // after the last tile.
+    uint64_t O2[G][2];
+    float off[G][4];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      A[g][0] = 0ull; A[g][1] = 0ull;
+      O2[g][0] = 0ull; O2[g][1] = 0ull;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) O[g][b] = 0.f;
+      for (int b = 0; b < 4; ++b) off[g][b] = 0.f;
     }
+    const bool vblock = vc != KVQ_F16 && vc != KVQ_RANK;
+    const int vclass = (vblock && (vbits == 8 || vbits == 4 || vbits == 2)) ? vbits : 0;
+    const bool vasym = codec_is_asym(vc);
+    const float vhalf = vblock ? (float)(1 << (vbits - 1)) : 0.f;
+    const int blane = ((4 * lane) / (nV < 32 ? nV : 32)) & 3;
+    const int kclass = kfast ? (kbits == 8 ? 8 : (kbits >= 4 ? 4 : 2)) : 0;
+    // This warp's weight table: (w, w) pairs per token on the fp32 path, int16 pairs
+    // per token pair and block on the integer path (same bytes).
+    constexpr int PWG = G + 1;                          // fp32 path row: G pairs + pad
+    uint64_t* pw = pw2 + (size_t)warp * 32 * (4 * G + 1);
+    uint32_t* wq = reinterpret_cast<uint32_t*>(pw);
     for (int i = warp; i < n_tiles; i += 4) {
       const int st = i % NS;
       if (!mbar_wait(&full[st], (i / NS) & 1)) atomicOr(p.err, ERR_TIMEOUT);
@@ -486,96 +496,84 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
       const int tok0 = (pg0 + i) * rows;
       const int nvalid = min(rows, seg_tokens - tok0);
       float s0[G], s1[G];
-      if (kfast) {
-        score2_block_codec<G>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1);
+      switch (kclass) {
+        case 8: score2_block_codec<G, 8>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        case 4: score2_block_codec<G, 4>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        case 2: score2_block_codec<G, 2>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        default:
+          score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0, rows);
+          score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1, rows);
+      }
+      if (kclass) {
 #pragma unroll
         for (int g = 0; g < G; ++g) { s0[g] *= sq[g]; s1[g] *= sq[g]; }
-      } else {
-        score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0, rows);
-        score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1, rows);
       }
-      float p0[G], p1[G];
+      float p0[G], p1[G], pm[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         if (lane >= nvalid) s0[g] = -INFINITY;
         if (lane + 32 >= nvalid) s1[g] = -INFINITY;
         const float tmax = warp_max(fmaxf(s0[g], s1[g]));
         const float mnew = fmaxf(m[g], tmax);
-        const float alpha = exp2f(m[g] - mnew);
-        p0[g] = exp2f(s0[g] - mnew);
-        p1[g] = exp2f(s1[g] - mnew);
+        const float alpha = ex2_approx(m[g] - mnew);
+        p0[g] = ex2_approx(s0[g] - mnew);
+        p1[g] = ex2_approx(s1[g] - mnew);
+        pm[g] = ex2_approx(tmax - mnew);
         l[g] = l[g] * alpha + (p0[g] + p1[g]);
         const uint64_t a2 = pack2(alpha, alpha);
-        A[g][0] = mul2(A[g][0], a2);
-        A[g][1] = mul2(A[g][1], a2);
+        O2[g][0] = mul2(O2[g][0], a2);
+        O2[g][1] = mul2(O2[g][1], a2);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) O[g][b] *= alpha;
+        for (int b = 0; b < 4; ++b) off[g][b] *= alpha;
         m[g] = mnew;
       }
+      switch (vclass) {
+        case 8: value_tile_int<G, 8>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
+        case 4: value_tile_int<G, 4>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
+        case 2: value_tile_int<G, 2>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
+        default:
+          // fp32 path: dequantized values times the softmax numerator, packed FMAs
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // the owner of token (lane + 32*half) publishes w = p*d per block (fast V) or p
-        const int t = lane + 32 * half;
+          for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          float d = 1.f, off = 0.f;
-          if (vmode && t < nvalid) {
-            if (vasym) {
-              const __half2 dm = *reinterpret_cast<const __half2*>(vs + t * sbV + 4 * b);
-              d = __low2float(dm);
-              off = __high2float(dm);
-            } else {
-              d = __half2float(*reinterpret_cast<const __half*>(vs + t * sbV + 2 * b));
-              off = -(float)vhalf * d;
+            for (int g = 0; g < G; ++g) {
+              const float pg = half ? p1[g] : p0[g];
+              pw[(size_t)lane * PWG + g] = pack2(pg, pg);
             }
-          }
+            __syncwarp();
+            const int ntok = min(32, nvalid - 32 * half);
+            for (int tt = 0; tt < ntok; ++tt) {
+              float v[4];
+              v_lane(vc, vbits, nV, cbV, sbV, vp, vs, 32 * half + tt, lane, v);
+              const uint64_t u01 = pack2(v[0], v[1]), u23 = pack2(v[2], v[3]);
+              const uint64_t* wrow = pw + (size_t)tt * PWG;
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float pg = half ? p1[g] : p0[g];
-            const float w = pg * d;
-            pw[(size_t)lane * PWR + b * G + g] = pack2(w, w);
-            O[g][b] = fmaf(pg, off, O[g][b]);
+              for (int g = 0; g < G; ++g) {
+                const uint64_t w2 = wrow[g];
+                O2[g][0] = fma2(w2, u01, O2[g][0]);
+                O2[g][1] = fma2(w2, u23, O2[g][1]);
+              }
+            }
+            __syncwarp();
           }
-        }
-        __syncwarp();
-        const int ntok = min(32, nvalid - 32 * half);
-        for (int tt = 0; tt < ntok; ++tt) {
-          const int t2 = 32 * half + tt;
-          uint64_t u01, u23;
-          if (vmode) {
-            v_codes_fast(vmode, vp + t2 * cbV, lane, u01, u23);
-          } else {
-            float v[4];
-            v_lane(vc, vbits, nV, cbV, sbV, vp, vs, t2, lane, v);
-            u01 = pack2(v[0], v[1]);
-            u23 = pack2(v[2], v[3]);
-          }
-          const uint64_t* wrow = pw + (size_t)tt * PWR + blane * G;
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const uint64_t w2 = wrow[g];
-            A[g][0] = fma2(w2, u01, A[g][0]);
-            A[g][1] = fma2(w2, u23, A[g][1]);
-          }
-        }
-        __syncwarp();
       }
+      __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       l[g] = warp_sum(l[g]);
+      float ob = 0.f;                     // the lane's block's offset sum, no dynamic register index
 #pragma unroll
-      for (int b = 0; b < 4; ++b) O[g][b] = warp_sum(O[g][b]);
+      for (int b = 0; b < 4; ++b) {
+        const float sb = warp_sum(off[g][b]);
+        ob = (b == blane) ? sb : ob;
+      }
       float a[4];
-      unpack2(A[g][0], a[0], a[1]);
-      unpack2(A[g][1], a[2], a[3]);
+      unpack2(O2[g][0], a[0], a[1]);
+      unpack2(O2[g][1], a[2], a[3]);
 #pragma unroll
-      float ob = O[g][0];                 // O[g][blane] without a dynamic register index
-#pragma unroll
-      for (int b = 1; b < 4; ++b) ob = (b == blane) ? O[g][b] : ob;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[g][c] = a[c] * (1.0f / v_position_factor(vmode, c)) + ob;
+      for (int c = 0; c < 4; ++c) acc[g][c] = a[c] + ob;
     }
   }
   __syncthreads();   // every stage consumed: the ring is reused as the merge area below
@@ -619,64 +617,84 @@ __global__ void __launch_bounds__(160) decode_kernel(const __grid_constant__ Dec
     finalize<G>(p, h, vbasis, head, aq, at, fl, out_base);
     return;
   }
-  // ---- publish the partial, take a ticket
-  float* part = p.ws + (((size_t)si * p.Hkv + head) * MAX_SPLITS + split) * G * PARTIAL_FLOATS;
+  // ---- publish the partial, take a ticket.  Partials are laid out
+  // [sequence, kv head][G][MAX_SPLITS][PARTIAL_FLOATS], so one head's splits are
+  // one contiguous block for the merge below.
+  float* pbase = p.ws + ((size_t)si * p.Hkv + head) * G * MAX_SPLITS * PARTIAL_FLOATS;
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
     const int g = idx / D, c = idx % D;
-    part[(size_t)g * PARTIAL_FLOATS + 4 + c] = is_tail ? at[idx] : aq[idx];
+    pbase[((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS + 4 + c] = is_tail ? at[idx] : aq[idx];
   }
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    part[(size_t)g * PARTIAL_FLOATS + 0] = fm[g];
-    part[(size_t)g * PARTIAL_FLOATS + 1] = fl[g];
-    part[(size_t)g * PARTIAL_FLOATS + 2] = is_tail ? 1.f : 0.f;
+    pbase[((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS + 0] = fm[g];
+    pbase[((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS + 1] = fl[g];
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    const int old = atomicAdd(&p.tickets[si * p.Hkv + head], 1);
+    // release: this CTA's partial (ordered before by the barrier) becomes visible
+    // to whichever CTA draws the last ticket; acquire: that CTA sees all others'.
+    const int old = atom_add_acq_rel_gpu(&p.tickets[si * p.Hkv + head], 1);
     flag[0] = (old == S - 1);
   }
   __syncthreads();
   if (!flag[0]) return;
-  __threadfence();
-  // ---- last CTA: merge every split (fixed order, deterministic).  One warp per
-  // head reduces the split maxima and sums with shuffles and keeps the factors
-  // 2^(m_s - M); then every thread sums its outputs' partials with independent loads.
-  const float* base = p.ws + (((size_t)si * p.Hkv + head) * MAX_SPLITS) * G * PARTIAL_FLOATS;
-  float* fsc = mg;                                                  // [G][MAX_SPLITS]
-  int* kinds = reinterpret_cast<int*>(mg + (size_t)G * MAX_SPLITS); // [MAX_SPLITS]
-  for (int g = warp; g < G; g += (int)(blockDim.x >> 5)) {
-    float ms[2], ls[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int s = lane + 32 * k;
-      ms[k] = s < S ? __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS) : -INFINITY;
-      ls[k] = s < S ? __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS + 1) : 0.f;
+  // ---- last CTA: merge every split in a fixed order (deterministic).  Each head's
+  // S partials are pulled into shared memory with one bulk copy (double-buffered
+  // over the heads when room allows); one warp reduces the split maxima and sums,
+  // then one thread per channel sums the rescaled partials.
+  const uint32_t per_g = (uint32_t)S * PARTIAL_FLOATS * 4;
+  const size_t stage_off = (post_bytes(G) + 127) & ~(size_t)127;
+  const size_t stage_room = (size_t)(reinterpret_cast<uint8_t*>(full) - smem) - stage_off;   // all dead after the loop
+  const int nbuf = min(min(G, 2), (int)(stage_room / per_g));      // >= 1: see decode_smem_bytes
+  float* fsc = mg;                                                  // [MAX_SPLITS] factors of the current head
+  if (threadIdx.x == 0) {
+    fence_proxy_async_global();          // the acquired partials, read through the bulk-copy path
+    fence_proxy_async_shared();          // the staging area was last used by ordinary loads and stores
+    for (int b = 0; b < nbuf; ++b) {
+      mbar_arrive_expect_tx(&mmerge[b], per_g);
+      bulk_g2s(smem + stage_off + (size_t)b * per_g, pbase + (size_t)b * MAX_SPLITS * PARTIAL_FLOATS, per_g,
+               &mmerge[b]);
     }
-    const float M = warp_max(fmaxf(ms[0], ms[1]));
-    float part = 0.f;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int s = lane + 32 * k;
-      const float f = (ms[k] == -INFINITY) ? 0.f : exp2f(ms[k] - M);
-      if (s < S) fsc[g * MAX_SPLITS + s] = f;
-      part += f * ls[k];
-    }
-    const float L = warp_sum(part);
-    if (lane == 0) { fm[g] = M; fl[g] = L; }
   }
-  for (int s = threadIdx.x; s < S; s += blockDim.x) kinds[s] = __ldcg(base + (size_t)s * G * PARTIAL_FLOATS + 2) != 0.f;
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int g = idx / D, c = idx % D;
-    float Aq = 0.f, At = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < S; ++s) {
-      const float v = __ldcg(base + ((size_t)s * G + g) * PARTIAL_FLOATS + 4 + c) * fsc[g * MAX_SPLITS + s];
-      if (kinds[s]) At += v; else Aq += v;
+  for (int g = 0; g < G; ++g) {
+    const int b = g % nbuf;
+    if (!mbar_wait(&mmerge[b], (g / nbuf) & 1)) atomicOr(p.err, ERR_TIMEOUT);
+    const float* pg = reinterpret_cast<const float*>(smem + stage_off + (size_t)b * per_g);
+    if (warp == 0) {
+      float ms[2], ls[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int s = lane + 32 * k;
+        ms[k] = s < S ? pg[(size_t)s * PARTIAL_FLOATS] : -INFINITY;
+        ls[k] = s < S ? pg[(size_t)s * PARTIAL_FLOATS + 1] : 0.f;
+      }
+      const float M = warp_max(fmaxf(ms[0], ms[1]));
+      float part = 0.f;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int s = lane + 32 * k;
+        const float f = (ms[k] == -INFINITY) ? 0.f : exp2f(ms[k] - M);
+        if (s < S) fsc[s] = f;
+        part += f * ls[k];
+      }
+      const float L = warp_sum(part);
+      if (lane == 0) { fm[g] = M; fl[g] = L; }
     }
-    aq[idx] = Aq;
-    at[idx] = At;
+    __syncthreads();
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+      float A = 0.f, B = 0.f;
+      for (int s2 = 0; s2 < qsplits; ++s2) A = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fsc[s2], A);
+      for (int s2 = qsplits; s2 < S; ++s2) B = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fsc[s2], B);
+      aq[g * D + c] = A;
+      at[g * D + c] = B;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && g + nbuf < G) {
+      fence_proxy_async_shared();
+      mbar_arrive_expect_tx(&mmerge[b], per_g);
+      bulk_g2s(smem + stage_off + (size_t)b * per_g, pbase + (size_t)(g + nbuf) * MAX_SPLITS * PARTIAL_FLOATS, per_g,
+               &mmerge[b]);
+    }
   }
   if (threadIdx.x == 0) p.tickets[si * p.Hkv + head] = 0;
   __syncthreads();

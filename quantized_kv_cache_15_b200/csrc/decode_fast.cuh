@@ -13,14 +13,9 @@
 // The 16-bit query carries a relative error of at most 2^-16 of its largest
 // element, far inside the 2e-3 output tolerance.
 //
-// Value accumulation runs as packed fp32 FMAs (fma.rn.f32x2: two FMAs per
-// issue slot).  Codes are turned into exact floats with one ALU op each (a
-// byte permute or a mask OR-ed into the exponent of 2^23) plus one packed
-// subtract per pair.  A code at bit position 4k (nibbles) or 2k (2-bit fields)
-// comes out multiplied by 16^k or 4^k; that power of two is carried by the
-// channel's accumulator and divided out exactly after the last tile.  The block
-// scale is folded into the softmax weight (w = p * d) and the block offset
-// (-2^(b-1) d, or the minimum m) into one accumulator per block.
+// Values run as integer dot products too (value_tile_int below) for the 8-, 4-
+// and 2-bit code planes; the other value codecs (F16 pages and tail, rank, 6-,
+// 5- and 3-bit) use packed fp32 FMAs (fma.rn.f32x2) on dequantized floats.
 #pragma once
 
 #include "kvq_internal.h"
@@ -36,6 +31,29 @@ __device__ __forceinline__ int dp2a_hi(uint32_t q, uint32_t b, int c) {
   int d;
   asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(q), "r"(b), "r"(c));
   return d;
+}
+// Signed-byte forms (centred value codes).
+__device__ __forceinline__ int dp2a_lo_s(uint32_t w, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi_s(uint32_t w, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(b), "r"(c));
+  return d;
+}
+
+// 2^x and 1/x with the SFU's approximate instructions (relative error ~2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ---- packed fp32 helpers (a pair lives in one 64-bit register)
@@ -129,7 +147,10 @@ __device__ __forceinline__ void score_block_epilogue(const uint8_t* ks, int sb, 
 
 // Unscaled integer-domain scores of tokens t0 and t0+32 for the block codecs.
 // tab0/tab1: pair tables [G][64] of the code planes; qsi: [G][4] block sums.
-template <int G>
+// KCLASS selects the code planes compiled in: 8 (q8), 4 (a nibble plane, plus a
+// 2-bit or 1-bit high plane for 6 / 5 bits), 2 (a 2-bit plane, plus a 1-bit high
+// plane for 3 bits).
+template <int G, int KCLASS>
 __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, const uint8_t* ks, int sb, int t0,
                                                    const uint32_t* tab0, const uint32_t* tab1, const int* qsi,
                                                    float s0[G], float s1[G]) {
@@ -143,7 +164,7 @@ __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, co
     int a0[G], a1[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) { a0[g] = 0; a1[g] = 0; }
-    if (bits == 8) {
+    if (KCLASS == 8) {
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const uint4 k0 = *reinterpret_cast<const uint4*>(kp + ((2 * b + ch) * PAGE + t0) * 16);
@@ -161,7 +182,7 @@ __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, co
           }
         }
       }
-    } else if (bits == 4 || bits == 6 || bits == 5) {
+    } else if (KCLASS == 4) {
       // nibble plane: chunk b holds the block's 32 low nibbles
       const uint4 k0 = *reinterpret_cast<const uint4*>(kp + (b * PAGE + t0) * 16);
       const uint4 k1 = *reinterpret_cast<const uint4*>(kp + (b * PAGE + t0 + 32) * 16);
@@ -275,30 +296,186 @@ __host__ __device__ inline void codec_tables(int kc, int* t0, int* t1) {
   }
 }
 
-// V fast modes: the lane's 4 channels of token row t as two exact-value pairs
-// (position factors 1 / 16^k / 4^k folded into the accumulators).
-// mode 8: 4 code bytes; mode 4: 4 nibbles; mode 2: 4 two-bit fields.
-__device__ __forceinline__ void v_codes_fast(int mode, const uint8_t* row, int lane, uint64_t& u01, uint64_t& u23) {
-  const uint32_t magic = 0x4B000000u;
-  if (mode == 8) {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + 4 * lane);
-    u01 = demagic2(prmt(w, magic, 0x7540u), prmt(w, magic, 0x7541u));
-    u23 = demagic2(prmt(w, magic, 0x7542u), prmt(w, magic, 0x7543u));
-  } else if (mode == 4) {
-    const uint32_t w = *reinterpret_cast<const uint16_t*>(row + 2 * lane);
-    u01 = demagic2((w & 0x000Fu) | magic, (w & 0x00F0u) | magic);
-    u23 = demagic2((w & 0x0F00u) | magic, (w & 0xF000u) | magic);
+// ---- values as integer dot products
+//
+// Per 64-token tile the softmax weight of token t for block b and head g,
+// w = p_tg * d_tb (p: softmax numerator, d: the block's fp16 scale), is rounded to
+// an integer W = rint(w / sigma_g) with sigma_g = (max_t p_tg) * (max_tb d_tb) / WMAX,
+// so 0 <= W <= WMAX < 2^15.  Lane j owns the token pair (j, j + 32): it packs
+// (W_j, W_j+32) as two int16 and publishes them per block and head.  Every lane then
+// walks the 32 pairs for its 4 channels: byte permutes put the two tokens' codes of
+// a channel side by side, centred (u - 2^(b-1), moved to the top bits of the byte
+// and sign-flipped, so a constant power-of-two factor rides along), and signed
+// dp2a adds W_j u_j + W_j+32 u_j+32 exactly in int32.  At the end of the tile the
+// integer sums are converted once, scaled by sigma_g / factor and added to the
+// fp32 accumulators.  Centring matters: W's rounding error (at most sigma_g / 2)
+// then multiplies a centred code, so the per-token errors do not add up to a
+// constant vector that the inverse Hadamard transform would concentrate into one
+// channel.  For the _1 codecs the rest of the value, m + 2^(b-1) d, is accumulated
+// separately in fp32 from the exact weights.
+constexpr float WMAX = 32000.0f;                   // below 2^15 with room for rounding
+constexpr float RINT_MAGIC = 12582912.0f;          // 1.5 * 2^23: x + MAGIC holds rint(x) in its low bits
+
+template <int G>
+__host__ __device__ constexpr int wq_row_words() { return 4 * G + 4; }  // token-pair row: [4 blocks][G] words + pad
+
+// One row of G words of the integer weight table.
+template <int G>
+__device__ __forceinline__ void load_wrow(const uint32_t* w, uint32_t out[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int g = 0; g < G; g += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(w + g);
+      out[g] = v.x; out[g + 1] = v.y; out[g + 2] = v.z; out[g + 3] = v.w;
+    }
+  } else if constexpr (G % 2 == 0) {
+#pragma unroll
+    for (int g = 0; g < G; g += 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(w + g);
+      out[g] = v.x; out[g + 1] = v.y;
+    }
   } else {
-    const uint32_t w = row[lane];
-    u01 = demagic2((w & 0x03u) | magic, (w & 0x0Cu) | magic);
-    u23 = demagic2((w & 0x30u) | magic, (w & 0xC0u) | magic);
+#pragma unroll
+    for (int g = 0; g < G; ++g) out[g] = w[g];
   }
 }
-// Factor carried by channel position k (0..3) of the lane in fast mode `mode`.
-__device__ __forceinline__ float v_position_factor(int mode, int k) {
-  if (mode == 4) return (float)(1 << (4 * k));
-  if (mode == 2) return (float)(1 << (2 * k));
-  return 1.0f;
+
+// Integer value sums of one tile for the lane's 4 channels (slot order of the
+// class, see slot_channel): acc[g][k] += sum_j W_j c_j + W_j+32 c_j+32 with c the
+// centred code times the class factor.
+// VB 8: slots = channels 0,1,2,3, factor 1.  VB 4: slots = channels 0, 2, 1, 3,
+// factor 16.  VB 2: slots = channels 0,1,2,3, factor 64.
+template <int G, int VB>
+__device__ __forceinline__ void value_dots(const uint8_t* vp, int cbV, int lane, const uint32_t* wr, int acc[G][4]) {
+  constexpr int WRS = wq_row_words<G>();
+#pragma unroll 4
+  for (int j = 0; j < 32; ++j) {
+    uint32_t X, Y;
+    if (VB == 8) {
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(vp + j * cbV + 4 * lane);
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(vp + (j + 32) * cbV + 4 * lane);
+      X = prmt(a, b, 0x5140u) ^ 0x80808080u;          // u - 128 as a signed byte
+      Y = prmt(a, b, 0x7362u) ^ 0x80808080u;
+    } else if (VB == 4) {
+      const uint32_t a = *reinterpret_cast<const uint16_t*>(vp + j * cbV + 2 * lane);
+      const uint32_t b = *reinterpret_cast<const uint16_t*>(vp + (j + 32) * cbV + 2 * lane);
+      const uint32_t z = prmt(a, b, 0x5140u);
+      X = ((z << 4) & 0xF0F0F0F0u) ^ 0x80808080u;     // 16 (u - 8): low nibbles moved up
+      Y = (z & 0xF0F0F0F0u) ^ 0x80808080u;            // 16 (u - 8): high nibbles
+    } else {
+      const uint32_t a = vp[j * cbV + lane];
+      const uint32_t b = vp[(j + 32) * cbV + lane];
+      const uint32_t z = prmt(a, b, 0x4040u);          // [a, b, a, b]
+      X = (((z << 6) & 0x0000C0C0u) | ((z << 4) & 0xC0C00000u)) ^ 0x80808080u;   // 64 (u - 2), fields 0, 1
+      Y = (((z << 2) & 0x0000C0C0u) | (z & 0xC0C00000u)) ^ 0x80808080u;          // fields 2, 3
+    }
+    uint32_t w[G];
+    load_wrow<G>(wr + j * WRS, w);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      acc[g][0] = dp2a_lo_s(w[g], X, acc[g][0]);
+      acc[g][1] = dp2a_hi_s(w[g], X, acc[g][1]);
+      acc[g][2] = dp2a_lo_s(w[g], Y, acc[g][2]);
+      acc[g][3] = dp2a_hi_s(w[g], Y, acc[g][3]);
+    }
+  }
+}
+
+// Channel (0..3 within the lane) and reciprocal position factor of slot k.
+template <int VB>
+__device__ __forceinline__ void slot_channel(int k, int& ch, float& inv_factor) {
+  if (VB == 8) { ch = k; inv_factor = 1.0f; }
+  else if (VB == 4) { ch = (k == 1) ? 2 : (k == 2) ? 1 : k; inv_factor = 1.0f / 16.0f; }
+  else { ch = k; inv_factor = 1.0f / 64.0f; }
+}
+
+// One 64-token tile of the value accumulation on the integer path.
+//  p0/p1: softmax numerators of the lane's tokens (lane, lane + 32); pm: the
+//  tile's largest numerator per head.  O2: packed fp32 accumulators of the
+//  lane's channels (already rescaled for this tile); off: per-block offsets.
+template <int G, int VB>
+__device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const uint8_t* vp, const uint8_t* vs, int cbV,
+                                               int sbV, int nvalid, int lane, int blane, uint32_t* wq,
+                                               const float p0[G], const float p1[G], const float pm[G],
+                                               uint64_t O2[G][2], float off[G][4]) {
+  constexpr int WRS = wq_row_words<G>();
+  float d0[4], d1[4], f0[4], f1[4];
+  float dm = 0.f;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    d0[b] = 0.f; d1[b] = 0.f; f0[b] = 0.f; f1[b] = 0.f;
+    if (lane < nvalid) {
+      if (vasym) {
+        const __half2 x = *reinterpret_cast<const __half2*>(vs + lane * sbV + 4 * b);
+        d0[b] = __low2float(x); f0[b] = fmaf(vhalf, d0[b], __high2float(x));
+      } else {
+        d0[b] = __half2float(*reinterpret_cast<const __half*>(vs + lane * sbV + 2 * b));
+      }
+    }
+    if (lane + 32 < nvalid) {
+      if (vasym) {
+        const __half2 x = *reinterpret_cast<const __half2*>(vs + (lane + 32) * sbV + 4 * b);
+        d1[b] = __low2float(x); f1[b] = fmaf(vhalf, d1[b], __high2float(x));
+      } else {
+        d1[b] = __half2float(*reinterpret_cast<const __half*>(vs + (lane + 32) * sbV + 2 * b));
+      }
+    }
+    dm = fmaxf(dm, fmaxf(d0[b], d1[b]));
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) dm = fmaxf(dm, __shfl_xor_sync(0xffffffffu, dm, m));
+
+  float sg[G];
+  uint32_t wv[4][G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float top = pm[g] * dm;                      // largest p * d of the tile
+    const float inv = top > 0.f ? WMAX * rcp_approx(top) : 0.f;
+    sg[g] = top * (1.0f / WMAX);
+    const float q0 = p0[g] * inv, q1 = p1[g] * inv;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const float w0 = fmaf(q0, d0[b], RINT_MAGIC), w1 = fmaf(q1, d1[b], RINT_MAGIC);
+      wv[b][g] = prmt(__float_as_uint(w0), __float_as_uint(w1), 0x5410u);
+      if (vasym) off[g][b] = fmaf(p0[g], f0[b], fmaf(p1[g], f1[b], off[g][b]));
+    }
+  }
+  uint32_t* row = wq + lane * WRS;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    if constexpr (G % 4 == 0) {
+#pragma unroll
+      for (int g = 0; g < G; g += 4)
+        *reinterpret_cast<uint4*>(row + b * G + g) = make_uint4(wv[b][g], wv[b][g + 1], wv[b][g + 2], wv[b][g + 3]);
+    } else if constexpr (G % 2 == 0) {
+#pragma unroll
+      for (int g = 0; g < G; g += 2) *reinterpret_cast<uint2*>(row + b * G + g) = make_uint2(wv[b][g], wv[b][g + 1]);
+    } else {
+#pragma unroll
+      for (int g = 0; g < G; ++g) row[b * G + g] = wv[b][g];
+    }
+  }
+  __syncwarp();
+  int acc[G][4];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[g][k] = 0;
+  value_dots<G, VB>(vp, cbV, lane, wq + blane * G, acc);
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float v[4], f[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      int ch; float inv_f;
+      slot_channel<VB>(k, ch, inv_f);
+      v[ch] = (float)acc[g][k];
+      f[ch] = sg[g] * inv_f;
+    }
+    O2[g][0] = fma2(pack2(v[0], v[1]), pack2(f[0], f[1]), O2[g][0]);
+    O2[g][1] = fma2(pack2(v[2], v[3]), pack2(f[2], f[3]), O2[g][1]);
+  }
 }
 
 }  // namespace kvq
