@@ -158,7 +158,9 @@ kvq_status kvq_append_quantize(kvq_plan* plan, int layer, int n_seqs, const int*
  * [forum thread on KV compression: dot, softmax, weighted average of values].
  *  q:   device fp16 [n_seqs][n_q_heads][128]
  *  out: device fp32 [n_seqs][n_q_heads][128]
- *  workspace: device, kvq_plan_workspace_bytes(plan, n_seqs), zeroed before first use.
+ *  workspace: device, kvq_plan_workspace_bytes(plan, n_seqs), zeroed before first use;
+ *    may be NULL when no sequence needs more than one split and the plan has no
+ *    projection (KVQ_ROT_PROJECTION plans keep their projected queries there).
  * Query head h attends with kv head h / (n_q_heads / n_kv_heads) over every
  * cached token of the sequence in this layer (quantized rows dequantized in
  * registers, tail rows in F16).  Split-K over pages; partial softmax states

@@ -312,9 +312,15 @@ kvq_status kvq_plan_cache_bytes(const kvq_plan* p, size_t* bytes) {
   return KVQ_OK;
 }
 
+// Decode workspace: [split partials][projected queries (projection plans)][merge counters]
+static size_t partial_bytes(const kvq_plan* p, int n_seqs) {
+  return (size_t)n_seqs * p->Hkv * MAX_SPLITS * p->G * PARTIAL_FLOATS * sizeof(float);
+}
+static size_t qproj_bytes(const kvq_plan* p, int n_seqs) {
+  return p->rot == KVQ_ROT_PROJECTION ? (size_t)n_seqs * p->Hq * D * sizeof(float) : 0;
+}
 static size_t workspace_bytes(const kvq_plan* p, int n_seqs) {
-  return (size_t)n_seqs * p->Hkv * MAX_SPLITS * p->G * PARTIAL_FLOATS * sizeof(float) +
-         (size_t)n_seqs * p->Hkv * sizeof(int);
+  return partial_bytes(p, n_seqs) + qproj_bytes(p, n_seqs) + (size_t)n_seqs * p->Hkv * sizeof(int);
 }
 
 kvq_status kvq_plan_workspace_bytes(const kvq_plan* p, int n_seqs, size_t* bytes) {
@@ -509,13 +515,19 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
     const SplitCounts c = split_counts(dp.len[i], (int)p->T, pps);
     grid_x = std::max(grid_x, c.qsplits + c.tsplits);
   }
-  if (grid_x > 1) {
+  const bool proj = p->rot == KVQ_ROT_PROJECTION;
+  if (grid_x > 1 || proj) {
     const size_t need = workspace_bytes(p, n_seqs);
     if (!workspace || workspace_bytes_given < need)
       return fail(KVQ_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes_given);
     if ((uintptr_t)workspace % 16) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
     dp.ws = (float*)workspace;
-    dp.tickets = (int*)((char*)workspace + (size_t)n_seqs * p->Hkv * MAX_SPLITS * p->G * PARTIAL_FLOATS * sizeof(float));
+    dp.qproj = (float*)((char*)workspace + partial_bytes(p, n_seqs));
+    dp.tickets = (int*)((char*)workspace + partial_bytes(p, n_seqs) + qproj_bytes(p, n_seqs));
+  }
+  if (proj) {
+    cudaError_t e = launch_project_query(dp, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "query projection launch");
   }
   cudaError_t e = launch_decode(dp, grid_x, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");

@@ -16,6 +16,7 @@
 //   F (final tail occupants): positions [f0, f0+nF) are copied into the ring,
 //                unless their slot belongs to an E warp.
 #include "kvq_internal.h"
+#include "ptx.cuh"
 #include "quant.cuh"
 
 namespace kvq {
@@ -54,6 +55,10 @@ __device__ __forceinline__ void transform_row(float x[4], int codec, int rot, co
 }
 
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {
+  // launched as a programmatic dependent (see ptx.cuh): set up while the previous
+  // kernel drains, then wait for it before touching global data
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const long gw = (long)blockIdx.x * 8 + wib;
@@ -134,9 +139,19 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
   if (p.total_items <= 0) return cudaSuccess;
   const long warps = (long)p.total_items * p.Hkv * 2;
   const long blocks = (warps + 7) / 8;
-  append_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, append_kernel, p);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 // ---------------------------------------------------------------- block table

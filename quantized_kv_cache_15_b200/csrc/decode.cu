@@ -231,7 +231,7 @@ size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   a += (size_t)G * D * 2;            // qi16
   a += (size_t)2 * G * 64 * 4;       // pair tables
   a = (a + 15) & ~(size_t)15;
-  a += (size_t)4 * 32 * (4 * G + 1) * 8;   // per-warp duplicated weight pairs (also the prologue scratch)
+  a += (size_t)4 * 32 * (4 * G + 1) * 8;   // per-warp weight tables
   a += (size_t)(2 * 8 + 2) * 8;      // mbarriers: ring full / empty, merge staging
   return a;
 }
@@ -280,6 +280,10 @@ __device__ void finalize(const DecodeParams& p, const HeadInfo& h, int vbasis, i
 template <int G>
 __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // launched as a programmatic dependent: the grid is set up while the previous
+  // kernel drains, and waits for it before reading or writing any global data
+  griddep_launch_dependents();
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
   const int seq = p.seq[si], len = p.len[si];
@@ -331,7 +335,6 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + off); off += (size_t)2 * G * 64 * 4;
   off = (off + 15) & ~(size_t)15;
   uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off); off += (size_t)4 * 32 * (4 * G + 1) * 8;
-  float* scratch = reinterpret_cast<float*>(pw2);                  // prologue only: [4 warps][D]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   uint64_t* empty = full + 8;
   uint64_t* mmerge = full + 16;                                    // the merge's two staging buffers
@@ -361,10 +364,9 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
     for (int i = 0; i < NS && i < n_tiles; ++i) issue_tile(i);
   }
 
-  const bool kfast = kc != KVQ_F16 && kc != KVQ_RANK;
+  const bool kfast = kc != KVQ_F16;                 // integer key scores (block and rank codecs)
   // ---- query preparation (consumer warps): q' in the K basis, scaled to log2 units
   if (warp < 4) {
-    float* tmp = scratch + warp * D;
     for (int g = warp; g < G; g += 4) {
       const __half* qsrc = p.q + ((size_t)si * p.Hq + (size_t)head * G + g) * D;
       uint2 raw = *reinterpret_cast<const uint2*>(qsrc + 4 * lane);
@@ -379,20 +381,10 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
         }
         fwht_row(x);
       } else if (kbasis == BASIS_PROJ) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tmp[4 * lane + i] = x[i];
-        __syncwarp();
-        const float* M = p.M + h.m_off;
-        float z[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int c = 0; c < D; ++c) {
-          const float xc = tmp[c];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (4 * lane + i < h.r) z[i] = fmaf(M[(size_t)(4 * lane + i) * D + c], xc, z[i]);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = z[i];
+        // M_h q, computed once per (sequence, kv head) by project_query_kernel
+        const float4 z = *reinterpret_cast<const float4*>(p.qproj + ((size_t)si * p.Hq + (size_t)head * G + g) * D +
+                                                          4 * lane);
+        x[0] = z.x; x[1] = z.y; x[2] = z.z; x[3] = z.w;
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -431,7 +423,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
   // ---- pair tables of the K codec's code planes (block codecs)
   if (kfast) {
     int tt0, tt1;
-    codec_tables(kc, &tt0, &tt1);
+    codec_tables(kbits, &tt0, &tt1);
     for (int idx = threadIdx.x; idx < 2 * G * 64; idx += blockDim.x) {
       const int plane = idx / (G * 64), rem = idx % (G * 64), g = rem / 64, w = rem % 64;
       const int type = plane ? tt1 : tt0;
@@ -475,11 +467,22 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
       for (int b = 0; b < 4; ++b) off[g][b] = 0.f;
     }
     const bool vblock = vc != KVQ_F16 && vc != KVQ_RANK;
-    const int vclass = (vblock && (vbits == 8 || vbits == 4 || vbits == 2)) ? vbits : 0;
+    // value path: centred integer (8/4/2-bit planes), two unsigned planes (LO*10 + HI),
+    // or 0 = fp32 (F16)
+    int vclass = 0;
+    if (vblock) vclass = (vbits == 8 || vbits == 4 || vbits == 2) ? vbits : (vbits == 6) ? 42 : (vbits == 5) ? 41 : 21;
+    else if (vc == KVQ_RANK) vclass = (vbits == 4) ? 40 : (vbits == 3) ? 21 : (vbits == 2) ? 20 : 10;
     const bool vasym = codec_is_asym(vc);
     const float vhalf = vblock ? (float)(1 << (vbits - 1)) : 0.f;
+    // the codes' centre on the plane path, the byte offset of the high plane, the
+    // blocks per row and the lanes per token pair
+    const float vcen = (vc == KVQ_RANK) ? 0.5f * (float)((1 << vbits) - 1) : vhalf;
+    const int voffB = (vc == KVQ_RANK) ? nV / 4 : (vbits == 3 ? 32 : 64);
+    const int blkV = nV < 32 ? nV : 32;
+    const int nbV = nV / blkV;
+    const int vcl = (nV == 16 || nV == 32 || nV == 64) ? nV / 4 : 32;
     const int blane = ((4 * lane) / (nV < 32 ? nV : 32)) & 3;
-    const int kclass = kfast ? (kbits == 8 ? 8 : (kbits >= 4 ? 4 : 2)) : 0;
+    const int kclass = !kfast ? 0 : (kc == KVQ_RANK) ? 10 + kbits : (kbits == 8 ? 8 : (kbits >= 4 ? 4 : 2));
     // This warp's weight table: (w, w) pairs per token on the fp32 path, int16 pairs
     // per token pair and block on the integer path (same bytes).
     constexpr int PWG = G + 1;                          // fp32 path row: G pairs + pad
@@ -500,6 +503,10 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
         case 8: score2_block_codec<G, 8>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         case 4: score2_block_codec<G, 4>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         case 2: score2_block_codec<G, 2>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        case 11: score2_rank<G, 1>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        case 12: score2_rank<G, 2>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        case 13: score2_rank<G, 3>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+        case 14: score2_rank<G, 4>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         default:
           score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0, rows);
           score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1, rows);
@@ -531,6 +538,30 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
         case 8: value_tile_int<G, 8>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
         case 4: value_tile_int<G, 4>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
         case 2: value_tile_int<G, 2>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
+        case 42:
+          value_tile_planes<G, 4, 2>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
+                                          pm, O2, off);
+          break;
+        case 41:
+          value_tile_planes<G, 4, 1>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
+                                          pm, O2, off);
+          break;
+        case 21:
+          value_tile_planes<G, 2, 1>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
+                                          pm, O2, off);
+          break;
+        case 40:
+          value_tile_planes<G, 4, 0>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
+                                          pm, O2, off);
+          break;
+        case 20:
+          value_tile_planes<G, 2, 0>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
+                                          pm, O2, off);
+          break;
+        case 10:
+          value_tile_planes<G, 1, 0>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
+                                          pm, O2, off);
+          break;
         default:
           // fp32 path: dequantized values times the softmax numerator, packed FMAs
 #pragma unroll
@@ -702,6 +733,46 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
   finalize<G>(p, h, vb_final, head, aq, at, fl, out_base);
 }
 
+// Projected queries of the rank variant: z = M_h q for the G query heads of every
+// (sequence, kv head), one thread per row of M_h (r <= 128), written to
+// p.qproj[seq][q head][0..127] (zeros past r).  Runs before decode_kernel.
+__global__ void __launch_bounds__(128) project_query_kernel(const __grid_constant__ DecodeParams p) {
+  __shared__ __align__(16) float qs[MAX_G][D];
+  const int head = blockIdx.x, si = blockIdx.y, i = threadIdx.x;
+  const HeadInfo h = p.heads[head];
+  for (int idx = threadIdx.x; idx < p.G * D; idx += blockDim.x) {
+    const int g = idx / D, c = idx % D;
+    qs[g][c] = __half2float(p.q[((size_t)si * p.Hq + (size_t)head * p.G + g) * D + c]);
+  }
+  __syncthreads();
+  float z[MAX_G];
+#pragma unroll
+  for (int g = 0; g < MAX_G; ++g) z[g] = 0.f;
+  if (h.kcodec == KVQ_RANK && i < h.r) {
+    const float4* row = reinterpret_cast<const float4*>(p.M + h.m_off + (size_t)i * D);
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+      const float4 m = __ldg(row + c4);
+#pragma unroll
+      for (int g = 0; g < MAX_G; ++g) {
+        if (g < p.G) {
+          z[g] = fmaf(m.x, qs[g][4 * c4 + 0], z[g]);
+          z[g] = fmaf(m.y, qs[g][4 * c4 + 1], z[g]);
+          z[g] = fmaf(m.z, qs[g][4 * c4 + 2], z[g]);
+          z[g] = fmaf(m.w, qs[g][4 * c4 + 3], z[g]);
+        }
+      }
+    }
+  }
+  for (int g = 0; g < p.G; ++g) p.qproj[((size_t)si * p.Hq + (size_t)head * p.G + g) * D + i] = z[g];
+}
+
+cudaError_t launch_project_query(const DecodeParams& p, cudaStream_t s) {
+  project_query_kernel<<<dim3(p.Hkv, p.n_seqs), 128, 0, s>>>(p);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 int decode_max_smem() { return 227 * 1024; }
 
 template <int G>
@@ -709,10 +780,19 @@ static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
   const size_t smem = decode_smem_bytes(p.stage_bytes, p.n_stages, G);
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(grid_x, p.Hkv, p.n_seqs);
-  decode_kernel<G><<<grid, 160, smem, s>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_x, p.Hkv, p.n_seqs);
+  cfg.blockDim = dim3(160, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<G>, p);
   note_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 // Resident CTAs per SM of the kernel for G heads with `smem` dynamic bytes (registers,

@@ -283,15 +283,120 @@ __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, co
   }
 }
 
-// Pair-table layouts the K codec uses (plane 0, plane 1; -1 = none).
-__host__ __device__ inline void codec_tables(int kc, int* t0, int* t1) {
-  switch (codec_bits(kc)) {
+// ---- rank codec keys: the projected row z (r values, b bits) of a KV-COBRA head.
+// Word k (4 bytes) of token t's code row in an interleaved K plane of chunk width w.
+// Bytes past the row are other data of the tile; the pair tables hold zeros for
+// channels >= r, so they contribute nothing.
+__device__ __forceinline__ uint32_t kword(const uint8_t* kp, int w, int t, int k) {
+  const int lw = __ffs(w) - 1;                     // w is a power of two
+  if (w >= 4) return *reinterpret_cast<const uint32_t*>(kp + ((((4 * k) >> lw) * PAGE + t) << lw) + ((4 * k) & (w - 1)));
+  const uint32_t lo = *reinterpret_cast<const uint16_t*>(kp + ((2 * k) * PAGE + t) * 2);
+  const uint32_t hi = *reinterpret_cast<const uint16_t*>(kp + ((2 * k + 1) * PAGE + t) * 2);
+  return lo | (hi << 16);
+}
+
+// Unscaled-to-log2 scores of tokens t0, t0+32 for a rank head with B-bit codes.
+// Block b (min(32, r) channels): s += d_b * (A_b - c * qsum_b), c = (2^B - 1) / 2,
+// taken exactly as (2 A_b - (2^B - 1) qsum_b) / 2.
+template <int G, int B>
+__device__ __forceinline__ void score2_rank(int r, const uint8_t* kp, const uint8_t* ks, int cbK, int sbK, int t0,
+                                            const uint32_t* tab0, const uint32_t* tab1, const int* qsi,
+                                            float s0[G], float s1[G]) {
+  const int w = interleave_w(cbK);
+  const int blk = r < 32 ? r : 32, nb = r / blk;
+#pragma unroll
+  for (int g = 0; g < G; ++g) { s0[g] = 0.f; s1[g] = 0.f; }
+#pragma unroll 1
+  for (int b = 0; b < nb; ++b) {
+    int a0[G], a1[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) { a0[g] = 0; a1[g] = 0; }
+    if (B == 4) {
+      const int nw = blk / 8;                        // 4 words per block (2 when r = 16)
+#pragma unroll 4
+      for (int i = 0; i < nw; ++i) {
+        const int k = 4 * b + i;
+        const uint32_t x0 = kword(kp, w, t0, k), x1 = kword(kp, w, t0 + 32, k);
+        const uint32_t lo0 = x0 & 0x0F0F0F0Fu, hi0 = (x0 >> 4) & 0x0F0F0F0Fu;
+        const uint32_t lo1 = x1 & 0x0F0F0F0Fu, hi1 = (x1 >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const uint4 q = *reinterpret_cast<const uint4*>(tab0 + g * 64 + 4 * k);
+          a0[g] = dp2a_hi(q.w, hi0, dp2a_lo(q.z, hi0, dp2a_hi(q.y, lo0, dp2a_lo(q.x, lo0, a0[g]))));
+          a1[g] = dp2a_hi(q.w, hi1, dp2a_lo(q.z, hi1, dp2a_hi(q.y, lo1, dp2a_lo(q.x, lo1, a1[g]))));
+        }
+      }
+    } else if (B == 2 || B == 3) {
+      const int nw = blk / 16;                       // 2 words per block (1 when r = 16)
+#pragma unroll 2
+      for (int i = 0; i < nw; ++i) {
+        const int k = 2 * b + i;
+        const uint32_t x0 = kword(kp, w, t0, k), x1 = kword(kp, w, t0 + 32, k);
+#pragma unroll
+        for (int sft = 0; sft < 4; ++sft) {
+          const uint32_t y0 = (x0 >> (2 * sft)) & 0x03030303u, y1 = (x1 >> (2 * sft)) & 0x03030303u;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint2 q = *reinterpret_cast<const uint2*>(tab0 + g * 64 + 8 * k + 2 * sft);
+            a0[g] = dp2a_hi(q.y, y0, dp2a_lo(q.x, y0, a0[g]));
+            a1[g] = dp2a_hi(q.y, y1, dp2a_lo(q.x, y1, a1[g]));
+          }
+        }
+      }
+      if (B == 3) {                                  // 1-bit high plane, weight 4, after r/4 bytes
+        const int k = r / 16 + b;
+        const uint32_t z0 = kword(kp, w, t0, k), z1 = kword(kp, w, t0 + 32, k);
+        int e0[G], e1[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) { e0[g] = 0; e1[g] = 0; }
+#pragma unroll
+        for (int sft = 0; sft < 8; ++sft) {
+          const uint32_t y0 = (z0 >> sft) & 0x01010101u, y1 = (z1 >> sft) & 0x01010101u;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const uint2 q = *reinterpret_cast<const uint2*>(tab1 + g * 64 + 16 * b + 2 * sft);
+            e0[g] = dp2a_hi(q.y, y0, dp2a_lo(q.x, y0, e0[g]));
+            e1[g] = dp2a_hi(q.y, y1, dp2a_lo(q.x, y1, e1[g]));
+          }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) { a0[g] += 4 * e0[g]; a1[g] += 4 * e1[g]; }
+      }
+    } else {                                         // B == 1: one word per block
+      const uint32_t z0 = kword(kp, w, t0, b), z1 = kword(kp, w, t0 + 32, b);
+#pragma unroll
+      for (int sft = 0; sft < 8; ++sft) {
+        const uint32_t y0 = (z0 >> sft) & 0x01010101u, y1 = (z1 >> sft) & 0x01010101u;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const uint2 q = *reinterpret_cast<const uint2*>(tab0 + g * 64 + 16 * b + 2 * sft);
+          a0[g] = dp2a_hi(q.y, y0, dp2a_lo(q.x, y0, a0[g]));
+          a1[g] = dp2a_hi(q.y, y1, dp2a_lo(q.x, y1, a1[g]));
+        }
+      }
+    }
+    const float d0 = 0.5f * __half2float(*reinterpret_cast<const __half*>(ks + t0 * sbK + 2 * b));
+    const float d1 = 0.5f * __half2float(*reinterpret_cast<const __half*>(ks + (t0 + 32) * sbK + 2 * b));
+    constexpr int C2 = (1 << B) - 1;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int qs = C2 * qsi[g * 4 + b];
+      s0[g] = fmaf((float)(2 * a0[g] - qs), d0, s0[g]);
+      s1[g] = fmaf((float)(2 * a1[g] - qs), d1, s1[g]);
+    }
+  }
+}
+
+// Pair-table layouts of a key codec with `bits` code bits (plane 0, plane 1; -1 = none).
+__host__ __device__ inline void codec_tables(int bits, int* t0, int* t1) {
+  switch (bits) {
     case 8: *t0 = TAB_NAT; *t1 = -1; break;
     case 6: *t0 = TAB_Q4; *t1 = TAB_Q2; break;
     case 5: *t0 = TAB_Q4; *t1 = TAB_Q1; break;
     case 4: *t0 = TAB_Q4; *t1 = -1; break;
     case 3: *t0 = TAB_Q2; *t1 = TAB_Q1; break;
     case 2: *t0 = TAB_Q2; *t1 = -1; break;
+    case 1: *t0 = TAB_Q1; *t1 = -1; break;
     default: *t0 = -1; *t1 = -1; break;
   }
 }
@@ -389,33 +494,32 @@ __device__ __forceinline__ void slot_channel(int k, int& ch, float& inv_factor) 
   else { ch = k; inv_factor = 1.0f / 64.0f; }
 }
 
-// One 64-token tile of the value accumulation on the integer path.
-//  p0/p1: softmax numerators of the lane's tokens (lane, lane + 32); pm: the
-//  tile's largest numerator per head.  O2: packed fp32 accumulators of the
-//  lane's channels (already rescaled for this tile); off: per-block offsets.
-template <int G, int VB>
-__device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const uint8_t* vp, const uint8_t* vs, int cbV,
-                                               int sbV, int nvalid, int lane, int blane, uint32_t* wq,
-                                               const float p0[G], const float p1[G], const float pm[G],
-                                               uint64_t O2[G][2], float off[G][4]) {
+// Softmax weights of one 64-token tile as int16 pairs: lane j publishes row j of
+// the warp's table ([4 blocks][G] words of (W_j, W_j+32)) and sigma_g is returned.
+// nb: blocks per row (absent blocks get weight 0).  For the _1 codecs
+// off[g][b] += p * (m + fcoef * d) per own token.
+template <int G>
+__device__ __forceinline__ void tile_weights(int nb, bool vasym, float fcoef, const uint8_t* vs, int sbV, int nvalid,
+                                             int lane, uint32_t* wq, const float p0[G], const float p1[G],
+                                             const float pm[G], float sg[G], float off[G][4]) {
   constexpr int WRS = wq_row_words<G>();
   float d0[4], d1[4], f0[4], f1[4];
   float dm = 0.f;
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     d0[b] = 0.f; d1[b] = 0.f; f0[b] = 0.f; f1[b] = 0.f;
-    if (lane < nvalid) {
+    if (b < nb && lane < nvalid) {
       if (vasym) {
         const __half2 x = *reinterpret_cast<const __half2*>(vs + lane * sbV + 4 * b);
-        d0[b] = __low2float(x); f0[b] = fmaf(vhalf, d0[b], __high2float(x));
+        d0[b] = __low2float(x); f0[b] = fmaf(fcoef, d0[b], __high2float(x));
       } else {
         d0[b] = __half2float(*reinterpret_cast<const __half*>(vs + lane * sbV + 2 * b));
       }
     }
-    if (lane + 32 < nvalid) {
+    if (b < nb && lane + 32 < nvalid) {
       if (vasym) {
         const __half2 x = *reinterpret_cast<const __half2*>(vs + (lane + 32) * sbV + 4 * b);
-        d1[b] = __low2float(x); f1[b] = fmaf(vhalf, d1[b], __high2float(x));
+        d1[b] = __low2float(x); f1[b] = fmaf(fcoef, d1[b], __high2float(x));
       } else {
         d1[b] = __half2float(*reinterpret_cast<const __half*>(vs + (lane + 32) * sbV + 2 * b));
       }
@@ -424,8 +528,6 @@ __device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const ui
   }
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) dm = fmaxf(dm, __shfl_xor_sync(0xffffffffu, dm, m));
-
-  float sg[G];
   uint32_t wv[4][G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -456,6 +558,20 @@ __device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const ui
     }
   }
   __syncwarp();
+}
+
+// One 64-token tile of the value accumulation on the centred integer path
+// (8-, 4- and 2-bit planes).  p0/p1: softmax numerators of the lane's tokens
+// (lane, lane + 32); pm: the tile's largest numerator per head.  O2: packed fp32
+// accumulators of the lane's channels (already rescaled for this tile); off:
+// per-block offsets of the _1 codecs.
+template <int G, int VB>
+__device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const uint8_t* vp, const uint8_t* vs, int cbV,
+                                               int sbV, int nvalid, int lane, int blane, uint32_t* wq,
+                                               const float p0[G], const float p1[G], const float pm[G],
+                                               uint64_t O2[G][2], float off[G][4]) {
+  float sg[G];
+  tile_weights<G>(4, vasym, vhalf, vs, sbV, nvalid, lane, wq, p0, p1, pm, sg, off);
   int acc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g)
@@ -475,6 +591,126 @@ __device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const ui
     }
     O2[g][0] = fma2(pack2(v[0], v[1]), pack2(f[0], f[1]), O2[g][0]);
     O2[g][1] = fma2(pack2(v[2], v[3]), pack2(f[2], f[3]), O2[g][1]);
+  }
+}
+
+// ---- values as unsigned code planes with an exact weight sum
+//
+// For the codecs whose codes span two bit planes (6 = 4 + 2, 5 = 4 + 1, 3 = 2 + 1
+// bits) and for the rank codec (1..4 bits, mid-rise levels (u - (2^b - 1)/2) d), the
+// codes enter dp2a unsigned, plane by plane, and the weights' exact integer sum
+// SW = sum_t W_t is accumulated beside them (one more dp2a per pair and head), so
+// sum_t W_t (u_t - c) = sum_t W_t u_t - c SW is exact for any centre c: W's rounding
+// errors still multiply centred codes.
+// Plane words of the two tokens (rows r0, r1) for the lane's 4 channels, and the
+// slot layout: BITS 4: (ch0, ch2, 16 ch1, 16 ch3); 2: (ch0, 4 ch1, 16 ch2, 64 ch3);
+// 1: (ch0, 2 ch1, 4 ch2, 8 ch3).
+template <int BITS>
+__device__ __forceinline__ void plane_words(const uint8_t* r0, const uint8_t* r1, int lane, uint32_t& X, uint32_t& Y) {
+  if (BITS == 4) {
+    const uint32_t a = *reinterpret_cast<const uint16_t*>(r0 + 2 * lane);
+    const uint32_t b = *reinterpret_cast<const uint16_t*>(r1 + 2 * lane);
+    const uint32_t z = prmt(a, b, 0x5140u);
+    X = z & 0x0F0F0F0Fu;
+    Y = z & 0xF0F0F0F0u;
+  } else if (BITS == 2) {
+    const uint32_t z = prmt(r0[lane], r1[lane], 0x4040u);
+    X = z & 0x0C0C0303u;
+    Y = z & 0xC0C03030u;
+  } else {
+    const uint32_t a = (r0[lane >> 1] >> (4 * (lane & 1))) & 15u;
+    const uint32_t b = (r1[lane >> 1] >> (4 * (lane & 1))) & 15u;
+    const uint32_t z = prmt(a, b, 0x4040u);
+    X = z & 0x02020101u;
+    Y = z & 0x08080404u;
+  }
+}
+template <int BITS>
+__device__ __forceinline__ void plane_slot(int k, int& ch, double& inv_f) {
+  if (BITS == 4) { ch = (k == 1) ? 2 : (k == 2) ? 1 : k; inv_f = (k < 2) ? 1.0 : 1.0 / 16.0; }
+  else if (BITS == 2) { ch = k; inv_f = (k == 0) ? 1.0 : (k == 1) ? 0.25 : (k == 2) ? 1.0 / 16.0 : 1.0 / 64.0; }
+  else { ch = k; inv_f = (k == 0) ? 1.0 : (k == 1) ? 0.5 : (k == 2) ? 0.25 : 0.125; }
+}
+
+// LO: bits of the low plane (4, 2, 1); HI: bits of the high plane (2, 1) or 0;
+// offB: byte offset of the high plane in a row; cen: the codes' centre (the _1
+// codecs' rest m + cen d goes to off); nb: blocks of blk channels per row.
+// Rows of fewer than 128 channels (rank heads) use cl = n/4 lanes per token pair
+// and 32/cl pairs side by side, summed over the lane groups at the end of the tile;
+// lane cg < cl then holds channels 4cg .. 4cg+3 (the other lanes hold copies for
+// channels that do not exist).
+template <int G, int LO, int HI>
+__device__ __forceinline__ void value_tile_planes(int nb, int blk, int cl, bool vasym, float cen, int offB,
+                                                  const uint8_t* vp, const uint8_t* vs, int cbV, int sbV, int nvalid,
+                                                  int lane, uint32_t* wq, const float p0[G], const float p1[G],
+                                                  const float pm[G], uint64_t O2[G][2], float off[G][4]) {
+  constexpr int WRS = wq_row_words<G>();
+  float sg[G];
+  tile_weights<G>(nb, vasym, cen, vs, sbV, nvalid, lane, wq, p0, p1, pm, sg, off);
+  const int grp = lane / cl, cg = lane - grp * cl, ngrp = 32 / cl;
+  const int blane = ((4 * cg) / blk) & 3;
+  int accA[G][4], accB[G][4], sw[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    sw[g] = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { accA[g][k] = 0; accB[g][k] = 0; }
+  }
+  const uint32_t* wr = wq + blane * G;
+#pragma unroll 4
+  for (int j = grp; j < 32; j += ngrp) {
+    const uint8_t* r0 = vp + j * cbV;
+    const uint8_t* r1 = vp + (j + 32) * cbV;
+    uint32_t XA, YA, XB = 0u, YB = 0u;
+    plane_words<LO>(r0, r1, cg, XA, YA);
+    if (HI) plane_words<HI ? HI : 1>(r0 + offB, r1 + offB, cg, XB, YB);
+    uint32_t w[G];
+    load_wrow<G>(wr + j * WRS, w);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      accA[g][0] = dp2a_lo(w[g], XA, accA[g][0]);
+      accA[g][1] = dp2a_hi(w[g], XA, accA[g][1]);
+      accA[g][2] = dp2a_lo(w[g], YA, accA[g][2]);
+      accA[g][3] = dp2a_hi(w[g], YA, accA[g][3]);
+      if (HI) {
+        accB[g][0] = dp2a_lo(w[g], XB, accB[g][0]);
+        accB[g][1] = dp2a_hi(w[g], XB, accB[g][1]);
+        accB[g][2] = dp2a_lo(w[g], YB, accB[g][2]);
+        accB[g][3] = dp2a_hi(w[g], YB, accB[g][3]);
+      }
+      sw[g] = dp2a_lo(w[g], 0x00000101u, sw[g]);
+    }
+  }
+  for (int m = cl; m < 32; m <<= 1) {                // sum over the lane groups
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      sw[g] += __shfl_xor_sync(0xffffffffu, sw[g], m);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        accA[g][k] += __shfl_xor_sync(0xffffffffu, accA[g][k], m);
+        if (HI) accB[g][k] += __shfl_xor_sync(0xffffffffu, accB[g][k], m);
+      }
+    }
+  }
+  __syncwarp();
+  // exact in double: sums of integers below 2^31 times powers of two
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    double v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = -(double)cen * (double)sw[g];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      int ch; double inv_f;
+      plane_slot<LO>(k, ch, inv_f);
+      v[ch] += (double)accA[g][k] * inv_f;
+      if (HI) {
+        plane_slot<HI ? HI : 1>(k, ch, inv_f);
+        v[ch] += (double)accB[g][k] * inv_f * (double)(1 << LO);
+      }
+    }
+    O2[g][0] = fma2(pack2((float)v[0], (float)v[1]), pack2(sg[g], sg[g]), O2[g][0]);
+    O2[g][1] = fma2(pack2((float)v[2], (float)v[3]), pack2(sg[g], sg[g]), O2[g][1]);
   }
 }
 

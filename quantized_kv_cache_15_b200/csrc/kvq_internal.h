@@ -167,7 +167,8 @@ struct DecodeParams {
   int pps;                       // pages per split
   int stage_bytes;               // bytes of one pipeline stage
   int n_stages;                  // 4 or 8
-  float* ws;                     // partials [n_seqs*Hkv][MAX_SPLITS][G][PARTIAL_FLOATS]
+  float* ws;                     // partials [n_seqs*Hkv][G][MAX_SPLITS][PARTIAL_FLOATS]
+  float* qproj;                  // projected queries M_h q [n_seqs][Hq][128] (projection plans)
   int* tickets;                  // [n_seqs*Hkv]
   int* err;
   int n_seqs;
@@ -181,6 +182,7 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t launch_block_table_update(int* table, int n, const int* idx_host, const int* val_host, cudaStream_t s);
 int decode_blocks_per_sm(int G, size_t smem_bytes);
 cudaError_t launch_decode(const DecodeParams& p, int grid_x, cudaStream_t s);
+cudaError_t launch_project_query(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_dequantize(const DecodeParams& p, int seq, int64_t t0, int64_t t1, float* k_out, float* v_out,
                               cudaStream_t s);
 cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t t1, int kv, uint8_t* codes,

@@ -68,4 +68,12 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Programmatic dependent launch (kernels launched with the programmatic
+// stream-serialization attribute).  launch_dependents lets the next kernel in the
+// stream be scheduled before this grid finishes; wait blocks until every
+// prerequisite grid has completed and its memory is visible.  A kernel calls wait
+// before touching anything an earlier kernel may write.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace kvq
