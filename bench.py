@@ -375,20 +375,27 @@ def run_kvq(args, world, rank, local):
     step_ms = ms / K
     plan.check_device_error(stream)
 
-    # ---- per-launch decode durations: the step's L decode launches, each between two
-    # events, enqueued behind a GPU sleep so they run back to back (no host gaps)
-    dec = []
-    ev_pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+    # ---- per-launch decode durations: a CUDA graph of the step's L decode calls
+    # (back to back, every layer's cache read once: far more than L2), replayed
+    # between two events on the launching stream; duration = elapsed / L
+    gd = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gd, stream=stream):
+        for l in range(L):
+            plan.decode(l, seqs, qall[l], out[l], ws, stream)
+    dec_reps = max(3, K // 4)
     with torch.cuda.stream(stream):
-        for _ in range(max(3, K // 4)):
-            torch.cuda._sleep(20_000_000 if B > 1 else 4_000_000)
-            for l in range(L):
-                ev_pairs[l][0].record(stream)
-                plan.decode(l, seqs, qall[l], out[l], ws, stream)
-                ev_pairs[l][1].record(stream)
-            stream.synchronize()
-            dec.extend(a.elapsed_time(b) for a, b in ev_pairs)
-    dec_ms = statistics.mean(dec)
+        for _ in range(2):
+            gd.replay()
+    stream.synchronize()
+    da, db = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        da.record(stream)
+        for _ in range(dec_reps):
+            gd.replay()
+        db.record(stream)
+    stream.synchronize()
+    dec_ms = max_over_ranks(da.elapsed_time(db) / (dec_reps * L), world, dev)
+    plan.check_device_error(stream)
 
     # ---- e2e through the public API: host buffers in, host buffers out
     kh, vh, qh = knew.cpu().pin_memory(), vnew.cpu().pin_memory(), qall.cpu().pin_memory()

@@ -491,12 +491,13 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
     work += (int64_t)pages * p->Hkv;
     maxpages = std::max(maxpages, pages);
   }
-  // Stage ring: as deep as fits three CTAs per SM (the register limit of the kernel),
-  // at least four stages (one per consumer warp).
   dp.stage_bytes = p->stage_bytes[layer];
-  dp.n_stages = 4;
-  for (int ns = 8; ns > 4; --ns)
-    if (decode_smem_bytes(dp.stage_bytes, ns, p->G) + 1024 <= (228 * 1024) / 3) { dp.n_stages = ns; break; }
+  // Stage ring: one stage per consumer warp at least, deeper while the CTAs per SM
+  // that the register allocation aims at still fit in shared memory.
+  const int want_ctas = NCW <= 4 ? 3 : 2;
+  dp.n_stages = NCW;
+  for (int ns = 8; ns > NCW; --ns)
+    if (decode_smem_bytes(dp.stage_bytes, ns, p->G) + 1024 <= (228 * 1024) / want_ctas) { dp.n_stages = ns; break; }
   const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G);
   // One full wave: as many CTAs as are resident at once (registers and shared memory
   // both counted), each taking an equal share of the page-heads.

@@ -215,7 +215,7 @@ __device__ __forceinline__ void v_lane(int vc, int vbits, int n, int cb, int sb,
 // afterwards the same bytes hold the warps' merge area and the final
 // accumulators ("post" region).
 __host__ __device__ inline size_t post_bytes(int G) {
-  return (size_t)4 * G * (D + 4) * 4 + (size_t)2 * G * D * 4 + (size_t)2 * G * 4 + 16;
+  return (size_t)NCW * G * (D + 4) * 4 + (size_t)2 * G * D * 4 + (size_t)2 * G * 4 + 16;
 }
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   size_t ring = (size_t)stage_bytes * n_stages;
@@ -231,7 +231,7 @@ size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   a += (size_t)G * D * 2;            // qi16
   a += (size_t)2 * G * 64 * 4;       // pair tables
   a = (a + 15) & ~(size_t)15;
-  a += (size_t)4 * 32 * (4 * G + 1) * 8;   // per-warp weight tables
+  a += (size_t)NCW * 32 * (4 * G + 1) * 8;   // per-warp weight tables
   a += (size_t)(2 * 8 + 2) * 8;      // mbarriers: ring full / empty, merge staging
   return a;
 }
@@ -278,7 +278,7 @@ __device__ void finalize(const DecodeParams& p, const HeadInfo& h, int vbasis, i
 }
 
 template <int G>
-__global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   // launched as a programmatic dependent: the grid is set up while the previous
   // kernel drains, and waits for it before reading or writing any global data
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
   uint8_t* stages = smem;
   // post-loop region (aliases the ring)
   float* mg = reinterpret_cast<float*>(smem);                      // [4 warps][G][D+4]
-  float* aq = mg + (size_t)4 * G * (D + 4);                        // [G][D] quantized-basis accumulator
+  float* aq = mg + (size_t)NCW * G * (D + 4);                      // [G][D] quantized-basis accumulator
   float* at = aq + (size_t)G * D;                                  // [G][D] tail accumulator
   float* fm = at + (size_t)G * D;
   float* fl = fm + G;
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
   int16_t* qi16 = reinterpret_cast<int16_t*>(smem + off); off += (size_t)G * D * 2;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + off); off += (size_t)2 * G * 64 * 4;
   off = (off + 15) & ~(size_t)15;
-  uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off); off += (size_t)4 * 32 * (4 * G + 1) * 8;
+  uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off); off += (size_t)NCW * 32 * (4 * G + 1) * 8;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   uint64_t* empty = full + 8;
   uint64_t* mmerge = full + 16;                                    // the merge's two staging buffers
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
     mbar_arrive_expect_tx(&full[st], tile_bytes);
     bulk_g2s(stages + (size_t)st * p.stage_bytes, src, tile_bytes, &full[st]);
   };
-  if (warp == 4 && lane == 0) {
+  if (warp == NCW && lane == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(&mmerge[0], 1);
     mbar_init(&mmerge[1], 1);
@@ -366,8 +366,8 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
 
   const bool kfast = kc != KVQ_F16;                 // integer key scores (block and rank codecs)
   // ---- query preparation (consumer warps): q' in the K basis, scaled to log2 units
-  if (warp < 4) {
-    for (int g = warp; g < G; g += 4) {
+  if (warp < NCW) {
+    for (int g = warp; g < G; g += NCW) {
       const __half* qsrc = p.q + ((size_t)si * p.Hq + (size_t)head * G + g) * D;
       uint2 raw = *reinterpret_cast<const uint2*>(qsrc + 4 * lane);
       float2 a = __half22float2(*reinterpret_cast<__half2*>(&raw.x));
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[g][i] = 0.f;
   }
-  if (warp == 4) {
+  if (warp == NCW) {
     // ---- producer: refill each stage once its consumer warp has released it
     if (lane == 0) {
       for (int i = NS; i < n_tiles; ++i) {
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
     constexpr int PWG = G + 1;                          // fp32 path row: G pairs + pad
     uint64_t* pw = pw2 + (size_t)warp * 32 * (4 * G + 1);
     uint32_t* wq = reinterpret_cast<uint32_t*>(pw);
-    for (int i = warp; i < n_tiles; i += 4) {
+    for (int i = warp; i < n_tiles; i += NCW) {
       const int st = i % NS;
       if (!mbar_wait(&full[st], (i / NS) & 1)) atomicOr(p.err, ERR_TIMEOUT);
       const uint8_t* sp = stages + (size_t)st * p.stage_bytes;
@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
     }
   }
   __syncthreads();   // every stage consumed: the ring is reused as the merge area below
-  if (warp < 4) {
+  if (warp < NCW) {
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float* dst = mg + ((size_t)warp * G + g) * (D + 4);
@@ -622,9 +622,9 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
   // ---- merge the four warps' states
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
     float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, mg[((size_t)w * G + g) * (D + 4)]);
+    for (int w = 0; w < NCW; ++w) M = fmaxf(M, mg[((size_t)w * G + g) * (D + 4)]);
     float L = 0.f;
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < NCW; ++w) {
       const float mw = mg[((size_t)w * G + g) * (D + 4)];
       L += (mw == -INFINITY) ? 0.f : exp2f(mw - M) * mg[((size_t)w * G + g) * (D + 4) + 1];
     }
@@ -635,7 +635,7 @@ __global__ void __launch_bounds__(160, G <= 4 ? 3 : 2) decode_kernel(const __gri
     const int g = idx / D, c = idx % D;
     const float M = fm[g];
     float A = 0.f;
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < NCW; ++w) {
       const float mw = mg[((size_t)w * G + g) * (D + 4)];
       if (mw != -INFINITY) A += exp2f(mw - M) * mg[((size_t)w * G + g) * (D + 4) + 4 + c];
     }
@@ -782,7 +782,7 @@ static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid_x, p.Hkv, p.n_seqs);
-  cfg.blockDim = dim3(160, 1, 1);
+  cfg.blockDim = dim3(DECODE_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -802,7 +802,7 @@ static int blocks_per_sm_g(size_t smem) {
   if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G>, 160, smem) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G>, DECODE_THREADS, smem) != cudaSuccess) return 0;
   return n;
 }
 

@@ -36,6 +36,14 @@ constexpr int MAX_SPLITS = 64;            // split-K pieces per (sequence, kv he
 constexpr int TAIL_TOK = 32;                 // token slots per tail page
 constexpr int TAIL_PAGE_BYTES = TAIL_TOK * D * 2 * 2;   // 16 KiB: K fp16 (interleaved) then V fp16
 constexpr int PARTIAL_FLOATS = 4 + D;     // m, l, kind, pad, acc[128]
+// Decode CTA shape: NCW consumer warps and one producer warp.
+#ifndef KVQ_DECODE_CONSUMER_WARPS
+#define KVQ_DECODE_CONSUMER_WARPS 4
+#endif
+constexpr int NCW = KVQ_DECODE_CONSUMER_WARPS;
+constexpr int DECODE_THREADS = 32 * (NCW + 1);
+// resident CTAs per SM the register allocation aims at
+#define DECODE_MIN_CTAS(G) ((NCW <= 4) ? ((G) <= 4 ? 3 : 2) : ((G) <= 4 ? 2 : 1))
 
 // Split-K layout of one sequence of `len` tokens, shared by the host (grid size)
 // and the decode kernel: the quantized segment in 64-token pages, the tail
