@@ -499,13 +499,29 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   for (int ns = 8; ns > NCW; --ns)
     if (decode_smem_bytes(dp.stage_bytes, ns, p->G) + 1024 <= (228 * 1024) / want_ctas) { dp.n_stages = ns; break; }
   const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G);
-  // One full wave: as many CTAs as are resident at once (registers and shared memory
-  // both counted), each taking an equal share of the page-heads.
+  // Split size: the candidate with the smallest estimated makespan, counted in waves
+  // of resident CTAs (registers and shared memory both counted) times the pages of
+  // a split plus a fixed cost of about three pages (query preparation, publishing
+  // the partial).  One full wave of equal shares suits one long sequence; a batch of
+  // ragged sequences does better with short splits over many waves.
   const int per_sm = std::max(1, decode_blocks_per_sm(p->G, smem));
   const int64_t target = (int64_t)p->num_sms * per_sm;
-  int pps = (int)std::max<int64_t>(1, (work + target - 1) / target);
   const int min_pps = (maxpages + MAX_SPLITS - 3) / (MAX_SPLITS - 2);
-  pps = std::max(pps, min_pps);
+  auto makespan = [&](int pp) {
+    int64_t ctas = 0;
+    for (int i = 0; i < n_seqs; ++i) {
+      const SplitCounts c = split_counts(dp.len[i], (int)p->T, pp);
+      ctas += (int64_t)(c.qsplits + c.tsplits) * p->Hkv;
+    }
+    return ((ctas + target - 1) / target) * (int64_t)(pp + 3);
+  };
+  int pps = std::max<int>(min_pps, (int)std::max<int64_t>(1, (work + target - 1) / target));
+  int64_t best = makespan(pps);
+  for (int cand : {8, 16, 32, 64}) {
+    if (cand < min_pps || cand >= pps) continue;
+    const int64_t m = makespan(cand);
+    if (m < best) { best = m; pps = cand; }
+  }
   if (const char* env = std::getenv("KVQ_DECODE_PAGES_PER_SPLIT")) {   // fixed split size (tests, tuning)
     const int v = std::atoi(env);
     if (v > 0) pps = std::max(v, min_pps);
