@@ -98,7 +98,7 @@ __device__ __forceinline__ void score_token(int kc, int kbits, int n, int cb, in
 #pragma unroll
   for (int g = 0; g < G; ++g) s[g] = 0.f;
   if (kc == KVQ_F16) {
-    if (t >= rows) return;                 // past the end of a 32-row tail tile
+    if (t >= rows) return;                 // past the end of a tail tile (TAIL_TOK rows)
 #pragma unroll 2
     for (int c = 0; c < 16; ++c) {
       uint4 v = *reinterpret_cast<const uint4*>(kp + (c * rows + t) * 16);

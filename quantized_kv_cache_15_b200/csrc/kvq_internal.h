@@ -13,10 +13,12 @@
 //   V codes : 64 rows of cbV bytes, row-major (lanes split one row's channels).
 //   V scales: 64 rows of sbV bytes, row-major.
 // Canonical packed rows (codes then scales) are defined by the quantizer: see
-// quant.cuh.  The tail ring of (seq, layer, kv head) is T/32 tail pages of
-// 16 KiB, each 32 token slots: [K fp16, interleaved as above but with 32 rows:
-// byte i of slot t at ((i / 16) * 32 + t) * 16 + i % 16][V fp16 row-major];
-// token position p lives in ring slot p % T.
+// quant.cuh.  The tail ring of (seq, layer, kv head) is T/TAIL_TOK tail pages of
+// 8 KiB, each TAIL_TOK = 16 token slots: [K fp16, interleaved as above but with
+// 16 rows: byte i of slot t at ((i / 16) * 16 + t) * 16 + i % 16][V fp16
+// row-major]; token position p lives in ring slot p % T.  A tail page is one
+// decode tile no larger than a quantized page-head of the common codecs, so a
+// tail does not enlarge the decode kernel's stage ring.
 #pragma once
 
 #include <cstdint>
@@ -33,8 +35,8 @@ constexpr int MAX_HKV = KVQ_MAX_KV_HEADS;
 constexpr int MAX_G = KVQ_MAX_GQA;
 constexpr int MAX_BATCH = KVQ_MAX_BATCH;
 constexpr int MAX_SPLITS = 64;            // split-K pieces per (sequence, kv head)
-constexpr int TAIL_TOK = 32;                 // token slots per tail page
-constexpr int TAIL_PAGE_BYTES = TAIL_TOK * D * 2 * 2;   // 16 KiB: K fp16 (interleaved) then V fp16
+constexpr int TAIL_TOK = 16;                 // token slots per tail page
+constexpr int TAIL_PAGE_BYTES = TAIL_TOK * D * 2 * 2;   // 8 KiB: K fp16 (interleaved) then V fp16
 constexpr int PARTIAL_FLOATS = 4 + D;     // m, l, kind, pad, acc[128]
 // Decode CTA shape: NCW consumer warps and one producer warp.
 #ifndef KVQ_DECODE_CONSUMER_WARPS
@@ -47,7 +49,7 @@ constexpr int DECODE_THREADS = 32 * (NCW + 1);
 
 // Split-K layout of one sequence of `len` tokens, shared by the host (grid size)
 // and the decode kernel: the quantized segment in 64-token pages, the tail
-// segment in 32-token tail pages, each cut into splits of `pps` pages.
+// segment in TAIL_TOK-token tail pages, each cut into splits of `pps` pages.
 struct SplitCounts { int nq, nt, nqp, ntp, qsplits, tsplits; };
 __host__ __device__ inline SplitCounts split_counts(int len, int T, int pps) {
   SplitCounts c;

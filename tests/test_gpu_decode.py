@@ -65,7 +65,7 @@ def test_workloads_small(cfg):
 
 def test_tail_covering_context_equals_f16_cache():
     """A tail that covers the whole context gives F16 attention: the same raw rows,
-    read from 32-row tail pages instead of 64-row F16 pages, so only the order of
+    read from 16-row tail pages instead of 64-row F16 pages, so only the order of
     the fp32 softmax merges differs (the oracle checks the bit-for-bit form)."""
     a = W.make_workload(1, "full", ctx=[768], tail=1024, k_codec=[[W.Q2_0] * 2], v_codec=[[W.Q2_0] * 2])
     b = W.make_workload(1, "full", ctx=[768], tail=0, k_codec=[[W.F16] * 2], v_codec=[[W.F16] * 2])
