@@ -193,6 +193,42 @@ kvq_status kvq_decode_attention(kvq_plan* plan, int layer, int n_seqs, const int
 kvq_status kvq_decode_attention_noalloc(kvq_plan* plan, int layer, int n_seqs, const int* seq_ids /*host*/,
                                         const void* q, float* out, void* stream);
 
+/* VBR regrade ["Introducing a new KV format: VBR (Variable Bit Rate)", first post:
+ * the cache is quantized layer by layer as the session grows, within a VRAM
+ * budget and above a quality floor].  Requantize every cached row of one layer
+ * below the F16 tail, for every sequence, to new per-kv-head codecs:
+ *  k_codec, v_codec: host [n_kv_heads]; block codecs (q8_0 .. q5_1) or F16 where
+ *    the head's rows are F16 already.  Rows are brought to the stored basis
+ *    (F16 rows through the layer's variance normalisation and Hadamard rotation,
+ *    block rows dequantized exactly) and quantized with the new codec; the tail
+ *    stays raw.  Later appends and decodes of the layer use the new codecs.
+ *  scratch: device, kvq_plan_regrade_bytes() bytes, 16-byte aligned: the layer's
+ *    pages are written there in the new layout and then copied over the layer's
+ *    pool on `stream`.
+ * KVQ_ERR_UNSUPPORTED for projection plans, rank targets, or a quantized row
+ * regraded to F16; KVQ_ERR_CAPACITY if the new pages would be larger than the
+ * layer's current pages (a regrade only moves to poorer codecs overall). */
+kvq_status kvq_plan_regrade_bytes(const kvq_plan* plan, int layer, const int* k_codec /*host*/,
+                                  const int* v_codec /*host*/, size_t* bytes);
+kvq_status kvq_regrade_layer(kvq_plan* plan, int layer, const int* k_codec /*host*/, const int* v_codec /*host*/,
+                             void* scratch, size_t scratch_bytes, void* stream);
+
+/* VBR policy step (host only) ["Introducing a new KV format: VBR (Variable Bit
+ * Rate)": quantize layer by layer as the session grows, within --vbr-vram and
+ * above --vbr-floor].  The pages fix no ladder or order; this reading uses the
+ * rungs F16 > q8_0 > q6_0 > q4_1 > q2_1 with V on a rung and K one rung richer.
+ * If bytes_in_use > budget, *layer is the deepest layer on the richest rung above
+ * floor_codec (a rung of the ladder) and new_k_codec / new_v_codec (host
+ * [n_kv_heads]) its codecs one rung down; else, or when every layer sits at the
+ * floor, *layer = -1.  k_codec, v_codec: host [n_layers][n_kv_heads], every head
+ * of a layer on the same V rung.  KVQ_ERR_UNSUPPORTED for codecs off the ladder. */
+kvq_status kvq_vbr_next(int n_layers, int n_kv_heads, const int* k_codec, const int* v_codec, int64_t bytes_in_use,
+                        int64_t budget, int floor_codec, int* layer, int* new_k_codec, int* new_v_codec);
+
+/* Device bytes the plan's cache uses now: every layer's pages held by sequences at
+ * the layer's current page size, plus the F16 tail rings. */
+kvq_status kvq_plan_bytes_in_use(const kvq_plan* plan, int64_t* bytes);
+
 /* Reconstruct cached rows t0 .. t1-1 of one sequence and layer in the ORIGINAL
  * basis (inverse rotation / projection applied; tail rows copied).
  *  k_out, v_out: device fp32 [t1-t0][n_kv_heads][128] (either may be NULL). */

@@ -235,6 +235,19 @@ def encode_rows(codec, rot, x_f16, inv_s=None, M=None, r=D, b=0):
     return codes, scales[:, : sb // 2]
 
 
+def regrade_rows(old_codec, new_codec, rot, codes, scales, inv_s=None):
+    """VBR regrade of packed rows ("Introducing a new KV format: VBR (Variable Bit
+    Rate)", first post: the cache is requantized layer by layer as the session
+    grows).  F16 rows (their codes are the raw fp16 values) are encoded with the
+    new codec exactly as an append would; block-codec rows are dequantized in the
+    stored basis and quantized again with the new codec.  Returns (codes, scales)."""
+    if old_codec == F16:
+        raw = _c(codes, np.uint8).reshape(-1, 2 * D).view(np.uint16)
+        return encode_rows(new_codec, rot, raw, inv_s=inv_s)
+    y = dequantize_rows(old_codec, codes, scales)
+    return quantize_rows(new_codec, y)
+
+
 def decode_rows_original(codec, rot, codes, scales, inv_s=None, M=None, r=D, b=0):
     cb, sb = row_bytes(codec, r, b)
     codes = _c(codes, np.uint8).reshape(-1, cb)

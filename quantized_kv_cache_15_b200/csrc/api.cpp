@@ -614,6 +614,121 @@ kvq_status kvq_read_rows(const kvq_plan* p, int layer, int seq_id, int64_t t0, i
   return KVQ_OK;
 }
 
+// New layout of one layer for the codecs kc[h], vc[h] (block codecs or F16, not the
+// rank codec): head infos with region offsets, the page bytes and the stage bytes.
+static kvq_status regrade_layout(const kvq_plan* p, int layer, const int* kc, const int* vc,
+                                 std::vector<HeadInfo>& heads, uint32_t& page_bytes, int& stage) {
+  if (p->rot == KVQ_ROT_PROJECTION) return fail(KVQ_ERR_UNSUPPORTED, "regrade of projection plans is not supported");
+  heads.assign(p->Hkv, HeadInfo{});
+  uint32_t poff = 0;
+  stage = 0;
+  for (int h = 0; h < p->Hkv; ++h) {
+    const HeadInfo& old = p->head(layer, h);
+    const int nk = kc[h], nv = vc[h];
+    if (!valid_codec(nk) || !valid_codec(nv) || nk == KVQ_RANK || nv == KVQ_RANK)
+      return fail(KVQ_ERR_UNSUPPORTED, "head %d: regrade targets must be block codecs or F16", h);
+    if ((nk == KVQ_F16 && old.kcodec != KVQ_F16) || (nv == KVQ_F16 && old.vcodec != KVQ_F16))
+      return fail(KVQ_ERR_UNSUPPORTED, "head %d: a quantized row cannot be regraded to F16", h);
+    HeadInfo hi;
+    std::memset(&hi, 0, sizeof(hi));
+    hi.kcodec = (uint8_t)nk; hi.vcodec = (uint8_t)nv; hi.r = (uint8_t)D;
+    hi.kbits = (uint8_t)codec_bits(nk); hi.vbits = (uint8_t)codec_bits(nv);
+    int cbK, sbK, cbV, sbV;
+    row_bytes(nk, D, 0, &cbK, &sbK);
+    row_bytes(nv, D, 0, &cbV, &sbV);
+    hi.cbK = (uint16_t)cbK; hi.sbK = (uint16_t)sbK; hi.cbV = (uint16_t)cbV; hi.sbV = (uint16_t)sbV;
+    hi.off = poff;
+    hi.bytes = (uint32_t)(PAGE * (cbK + sbK + cbV + sbV));
+    poff += hi.bytes;
+    stage = std::max(stage, (int)hi.bytes);
+    heads[h] = hi;
+  }
+  if (p->T > 0) stage = std::max(stage, TAIL_PAGE_BYTES);
+  stage = (stage + 127) & ~127;
+  page_bytes = poff;
+  if (page_bytes > p->page_bytes[layer])
+    return fail(KVQ_ERR_CAPACITY, "regrade must not grow the layer's pages (%u -> %u bytes)", p->page_bytes[layer],
+                page_bytes);
+  return KVQ_OK;
+}
+
+kvq_status kvq_plan_regrade_bytes(const kvq_plan* p, int layer, const int* k_codec, const int* v_codec, size_t* bytes) {
+  if (!p || !k_codec || !v_codec || !bytes) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  std::vector<HeadInfo> heads;
+  uint32_t pb = 0;
+  int stage = 0;
+  const kvq_status st = regrade_layout(p, layer, k_codec, v_codec, heads, pb, stage);
+  if (st != KVQ_OK) return st;
+  *bytes = (size_t)pb * (size_t)p->n_pages;
+  return KVQ_OK;
+}
+
+kvq_status kvq_regrade_layer(kvq_plan* p, int layer, const int* k_codec, const int* v_codec, void* scratch,
+                             size_t scratch_bytes, void* stream) {
+  if (!p || !k_codec || !v_codec) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
+  if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  std::vector<HeadInfo> heads;
+  uint32_t pb = 0;
+  int stage = 0;
+  kvq_status st = regrade_layout(p, layer, k_codec, v_codec, heads, pb, stage);
+  if (st != KVQ_OK) return st;
+  const size_t need = (size_t)pb * (size_t)p->n_pages;
+  if (need && (!scratch || scratch_bytes < need))
+    return fail(KVQ_ERR_INVALID_ARG, "scratch of %zu bytes needed (got %zu)", need, scratch_bytes);
+  if ((uintptr_t)scratch % 16) return fail(KVQ_ERR_INVALID_ARG, "scratch must be 16-byte aligned");
+  const cudaStream_t s = (cudaStream_t)stream;
+  RegradeParams rp;
+  std::memset(&rp, 0, sizeof(rp));
+  rp.src_pool = p->cache + p->layer_off[layer];
+  rp.src_page_bytes = p->page_bytes[layer];
+  rp.dst_pool = (uint8_t*)scratch;
+  rp.dst_page_bytes = pb;
+  rp.block_table = p->d_bt;
+  rp.max_pages_per_seq = p->mpps;
+  rp.Hkv = p->Hkv;
+  rp.rot = p->rot;
+  rp.inv_s = p->d_inv ? p->d_inv + (size_t)layer * p->Hkv * 2 * D : nullptr;
+  rp.err = p->d_err;
+  for (int h = 0; h < p->Hkv; ++h) { rp.src[h] = p->head(layer, h); rp.dst[h] = heads[h]; }
+  // every sequence's quantized rows, MAX_REGRADE_SEQS sequences per launch
+  for (int s0 = 0; s0 < p->max_seqs; s0 += MAX_REGRADE_SEQS) {
+    rp.n_seqs = 0;
+    rp.total_rows = 0;
+    for (int sq = s0; sq < std::min(p->max_seqs, s0 + MAX_REGRADE_SEQS); ++sq) {
+      const int64_t len = p->len[(size_t)sq * p->L + layer];
+      const int64_t nq = len > p->T ? len - p->T : 0;
+      if (nq <= 0) continue;
+      rp.seq[rp.n_seqs] = sq;
+      rp.row0[rp.n_seqs] = rp.total_rows;
+      rp.total_rows += nq;
+      ++rp.n_seqs;
+    }
+    rp.row0[rp.n_seqs] = rp.total_rows;
+    const cudaError_t e = launch_regrade(rp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "regrade launch");
+  }
+  if (need) {
+    const cudaError_t e = cudaMemcpyAsync(p->cache + p->layer_off[layer], scratch, need, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "regrade copy-back");
+  }
+  for (int h = 0; h < p->Hkv; ++h) p->heads[(size_t)layer * p->Hkv + h] = heads[h];
+  p->page_bytes[layer] = pb;
+  p->stage_bytes[layer] = stage;
+  return KVQ_OK;
+}
+
+kvq_status kvq_plan_bytes_in_use(const kvq_plan* p, int64_t* bytes) {
+  if (!p || !bytes) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  int64_t pages = 0;
+  for (int s = 0; s < p->max_seqs; ++s) pages += p->npages[s];
+  int64_t b = 0;
+  for (int l = 0; l < p->L; ++l) b += pages * (int64_t)p->page_bytes[l];
+  *bytes = b + (int64_t)(p->cache_bytes - p->tail_off);
+  return KVQ_OK;
+}
+
 kvq_status kvq_seq_length(const kvq_plan* p, int seq_id, int layer, int64_t* len) {
   if (!p || !len) return fail(KVQ_ERR_INVALID_ARG, "null argument");
   if (seq_id < 0 || seq_id >= p->max_seqs || layer < 0 || layer >= p->L)

@@ -21,15 +21,6 @@
 
 namespace kvq {
 
-__device__ __forceinline__ void load_row_f16(const __half* src, float x[4]) {
-  const int lane = threadIdx.x & 31;
-  uint2 v = *reinterpret_cast<const uint2*>(src + 4 * lane);
-  __half2 a = *reinterpret_cast<__half2*>(&v.x);
-  __half2 b = *reinterpret_cast<__half2*>(&v.y);
-  float2 fa = __half22float2(a), fb = __half22float2(b);
-  x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
-}
-
 // Byte address of a tail ring row's lane piece (8 bytes = 4 fp16 values).
 __device__ __forceinline__ uint8_t* ring_lane_ptr(uint8_t* ring, int slot, int kv) {
   const int lane = threadIdx.x & 31;
@@ -37,21 +28,6 @@ __device__ __forceinline__ uint8_t* ring_lane_ptr(uint8_t* ring, int slot, int k
   const int row = slot % TAIL_TOK;
   if (kv == 0) return tp + ((lane >> 1) * TAIL_TOK + row) * 16 + (lane & 1) * 8;   // interleaved, cb = 256
   return tp + TAIL_TOK * D * 2 + row * (D * 2) + 8 * lane;                          // row-major
-}
-
-// Transform the warp's row into the stored basis (lane: 4 values): the raw
-// values for F16 and unrotated plans; x * inv_s (variance normalisation) and the
-// staged Hadamard transform otherwise.  The projection (rank codec) runs on the
-// tensor cores in project.cu.
-__device__ __forceinline__ void transform_row(float x[4], int codec, int rot, const float* inv_s) {
-  const int lane = threadIdx.x & 31;
-  if (codec == KVQ_F16 || codec == KVQ_RANK || rot == KVQ_ROT_NONE) return;
-  if (rot == KVQ_ROT_VARNORM_HADAMARD) {
-    float4 s = *reinterpret_cast<const float4*>(inv_s + 4 * lane);
-    x[0] = __fmul_rn(x[0], s.x); x[1] = __fmul_rn(x[1], s.y);
-    x[2] = __fmul_rn(x[2], s.z); x[3] = __fmul_rn(x[3], s.w);
-  }
-  fwht_row(x);
 }
 
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendParams p) {

@@ -11,28 +11,6 @@
 
 namespace kvq {
 
-// The lane's 4 codes (values 4l .. 4l+3 of a row of n values) from a code plane.
-__device__ __forceinline__ void lane_codes(const uint8_t* plane, int cb, int t, bool interleaved, int bits, int n,
-                                           int lane, uint32_t u[4]) {
-  auto at = [&](int i) -> uint32_t { return plane[interleaved ? kplane_off(cb, t, i) : t * cb + i]; };
-  switch (bits) {
-    case 8: for (int i = 0; i < 4; ++i) u[i] = at(4 * lane + i); break;
-    case 4: { uint32_t w = at(2 * lane) | (at(2 * lane + 1) << 8);
-      for (int i = 0; i < 4; ++i) u[i] = (w >> (4 * i)) & 15u; } break;
-    case 2: { uint32_t w = at(lane); for (int i = 0; i < 4; ++i) u[i] = (w >> (2 * i)) & 3u; } break;
-    case 1: { uint32_t w = (at(lane >> 1) >> (4 * (lane & 1))) & 15u;
-      for (int i = 0; i < 4; ++i) u[i] = (w >> i) & 1u; } break;
-    case 6: { uint32_t lo = at(2 * lane) | (at(2 * lane + 1) << 8); uint32_t hi = at(n / 2 + lane);
-      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> (2 * i)) & 3u) << 4); } break;
-    case 3: { uint32_t lo = at(lane); uint32_t hi = (at(n / 4 + (lane >> 1)) >> (4 * (lane & 1))) & 15u;
-      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (2 * i)) & 3u) | (((hi >> i) & 1u) << 2); } break;
-    case 5: { uint32_t lo = at(2 * lane) | (at(2 * lane + 1) << 8);
-      uint32_t hi = (at(n / 2 + (lane >> 1)) >> (4 * (lane & 1))) & 15u;
-      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> i) & 1u) << 4); } break;
-    default: u[0] = u[1] = u[2] = u[3] = 0;
-  }
-}
-
 __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ DecodeParams p, int seq, int len,
                                                       long t0, long n_rows, float* k_out, float* v_out) {
   __shared__ __align__(16) float zs[8][D];

@@ -193,6 +193,27 @@ cudaError_t launch_block_table_update(int* table, int n, const int* idx_host, co
 int decode_blocks_per_sm(int G, size_t smem_bytes);
 cudaError_t launch_decode(const DecodeParams& p, int grid_x, cudaStream_t s);
 cudaError_t launch_project_query(const DecodeParams& p, cudaStream_t s);
+// ---------------------------------------------------------------- VBR regrade
+constexpr int MAX_REGRADE_SEQS = 128;
+struct RegradeParams {
+  const uint8_t* src_pool;       // the layer's page pool in its current layout
+  uint32_t src_page_bytes;
+  uint8_t* dst_pool;             // scratch: every page of the layer in the new layout
+  uint32_t dst_page_bytes;
+  const int* block_table;
+  int max_pages_per_seq;
+  int Hkv, rot;
+  const float* inv_s;            // [Hkv][2][128] of this layer, or null
+  int* err;
+  int n_seqs;
+  long total_rows;
+  int seq[MAX_REGRADE_SEQS];
+  long row0[MAX_REGRADE_SEQS + 1];   // prefix sums of the sequences' quantized rows
+  HeadInfo src[MAX_HKV];
+  HeadInfo dst[MAX_HKV];
+};
+cudaError_t launch_regrade(const RegradeParams& p, cudaStream_t s);
+
 cudaError_t launch_dequantize(const DecodeParams& p, int seq, int64_t t0, int64_t t1, float* k_out, float* v_out,
                               cudaStream_t s);
 cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t t1, int kv, uint8_t* codes,

@@ -243,4 +243,51 @@ __device__ __forceinline__ void quantize_store_row(const float x[4], int codec, 
   }
 }
 
+// The warp's fp16 row (lane: 4 values) as fp32.
+__device__ __forceinline__ void load_row_f16(const __half* src, float x[4]) {
+  const int lane = threadIdx.x & 31;
+  uint2 v = *reinterpret_cast<const uint2*>(src + 4 * lane);
+  __half2 a = *reinterpret_cast<__half2*>(&v.x);
+  __half2 b = *reinterpret_cast<__half2*>(&v.y);
+  float2 fa = __half22float2(a), fb = __half22float2(b);
+  x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
+}
+
+// Transform the warp's row into the stored basis (lane: 4 values): the raw
+// values for F16 and unrotated plans; x * inv_s (variance normalisation) and the
+// staged Hadamard transform otherwise.  The projection (rank codec) runs on the
+// tensor cores in project.cu.
+__device__ __forceinline__ void transform_row(float x[4], int codec, int rot, const float* inv_s) {
+  const int lane = threadIdx.x & 31;
+  if (codec == KVQ_F16 || codec == KVQ_RANK || rot == KVQ_ROT_NONE) return;
+  if (rot == KVQ_ROT_VARNORM_HADAMARD) {
+    float4 s = *reinterpret_cast<const float4*>(inv_s + 4 * lane);
+    x[0] = __fmul_rn(x[0], s.x); x[1] = __fmul_rn(x[1], s.y);
+    x[2] = __fmul_rn(x[2], s.z); x[3] = __fmul_rn(x[3], s.w);
+  }
+  fwht_row(x);
+}
+
+// The lane's 4 codes (values 4l .. 4l+3 of a row of n values) from a code plane.
+__device__ __forceinline__ void lane_codes(const uint8_t* plane, int cb, int t, bool interleaved, int bits, int n,
+                                           int lane, uint32_t u[4]) {
+  auto at = [&](int i) -> uint32_t { return plane[interleaved ? kplane_off(cb, t, i) : t * cb + i]; };
+  switch (bits) {
+    case 8: for (int i = 0; i < 4; ++i) u[i] = at(4 * lane + i); break;
+    case 4: { uint32_t w = at(2 * lane) | (at(2 * lane + 1) << 8);
+      for (int i = 0; i < 4; ++i) u[i] = (w >> (4 * i)) & 15u; } break;
+    case 2: { uint32_t w = at(lane); for (int i = 0; i < 4; ++i) u[i] = (w >> (2 * i)) & 3u; } break;
+    case 1: { uint32_t w = (at(lane >> 1) >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = (w >> i) & 1u; } break;
+    case 6: { uint32_t lo = at(2 * lane) | (at(2 * lane + 1) << 8); uint32_t hi = at(n / 2 + lane);
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> (2 * i)) & 3u) << 4); } break;
+    case 3: { uint32_t lo = at(lane); uint32_t hi = (at(n / 4 + (lane >> 1)) >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (2 * i)) & 3u) | (((hi >> i) & 1u) << 2); } break;
+    case 5: { uint32_t lo = at(2 * lane) | (at(2 * lane + 1) << 8);
+      uint32_t hi = (at(n / 2 + (lane >> 1)) >> (4 * (lane & 1))) & 15u;
+      for (int i = 0; i < 4; ++i) u[i] = ((lo >> (4 * i)) & 15u) | (((hi >> i) & 1u) << 4); } break;
+    default: u[0] = u[1] = u[2] = u[3] = 0;
+  }
+}
+
 }  // namespace kvq

@@ -38,6 +38,10 @@ SIGNATURES = {
     "kvq_append_quantize": (_I, [_P, _I, _I, _IP, _IP, _P, _P, _P]),
     "kvq_decode_attention": (_I, [_P, _I, _I, _IP, _P, _P, _P, _SZ, _P]),
     "kvq_decode_attention_noalloc": (_I, [_P, _I, _I, _IP, _P, _P, _P]),
+    "kvq_plan_regrade_bytes": (_I, [_P, _I, _IP, _IP, ctypes.POINTER(ctypes.c_size_t)]),
+    "kvq_regrade_layer": (_I, [_P, _I, _IP, _IP, _P, ctypes.c_size_t, _P]),
+    "kvq_vbr_next": (_I, [_I, _I, _IP, _IP, ctypes.c_int64, ctypes.c_int64, _I, _IP, _IP, _IP]),
+    "kvq_plan_bytes_in_use": (_I, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "kvq_dequantize": (_I, [_P, _I, _I, _I64, _I64, _P, _P, _P]),
     "kvq_row_bytes": (_I, [_P, _I, _I, _I, _IP, _IP]),
     "kvq_read_rows": (_I, [_P, _I, _I, _I64, _I64, _I, _P, _P, _P]),
@@ -191,6 +195,21 @@ class Plan:
         _check(lib().kvq_decode_attention_noalloc(self._h, layer, len(seq_ids), _ints(seq_ids), _ptr(q), _ptr(out),
                                                   _stream(stream)))
 
+    def regrade_bytes(self, layer: int, k_codec, v_codec) -> int:
+        v = ctypes.c_size_t()
+        _check(lib().kvq_plan_regrade_bytes(self._h, layer, _ints(k_codec), _ints(v_codec), ctypes.byref(v)))
+        return v.value
+
+    def regrade(self, layer: int, k_codec, v_codec, scratch: torch.Tensor, stream=None):
+        """Requantize layer `layer` to new per-kv-head codecs (VBR regrade)."""
+        _check(lib().kvq_regrade_layer(self._h, layer, _ints(k_codec), _ints(v_codec), _ptr(scratch),
+                                       scratch.numel() * scratch.element_size(), _stream(stream)))
+
+    def bytes_in_use(self) -> int:
+        v = ctypes.c_int64()
+        _check(lib().kvq_plan_bytes_in_use(self._h, ctypes.byref(v)))
+        return v.value
+
     def dequantize(self, layer: int, seq: int, t0: int, t1: int, k_out=None, v_out=None, stream=None):
         _check(lib().kvq_dequantize(self._h, layer, seq, t0, t1, _ptr(k_out), _ptr(v_out), _stream(stream)))
 
@@ -231,6 +250,22 @@ def cobra_allocate(lambdas: np.ndarray, bpd: float, eps) -> tuple:
     if st != 0:
         raise KVQError(st, "kvq_cobra_allocate: invalid spectra, bpd or budget")
     return r, b, used.value
+
+
+def vbr_next(k_codec, v_codec, bytes_in_use: int, budget: int, floor_codec: int):
+    """VBR policy step: (layer, new K codecs, new V codecs), layer -1 if nothing to do.
+    k_codec, v_codec: [n_layers][n_kv_heads]."""
+    kc = np.ascontiguousarray(k_codec, np.int32)
+    vc = np.ascontiguousarray(v_codec, np.int32)
+    L, H = kc.shape
+    layer = ctypes.c_int()
+    nk = np.zeros(H, np.int32)
+    nv = np.zeros(H, np.int32)
+    st = lib().kvq_vbr_next(L, H, kc.ctypes.data_as(_IP), vc.ctypes.data_as(_IP), int(bytes_in_use), int(budget),
+                            int(floor_codec), ctypes.byref(layer), nk.ctypes.data_as(_IP), nv.ctypes.data_as(_IP))
+    if st != 0:
+        raise KVQError(st, "kvq_vbr_next: codecs off the ladder or bad arguments")
+    return layer.value, nk.tolist(), nv.tolist()
 
 
 def launch_count() -> int:
