@@ -481,8 +481,38 @@ def run_kvq(args, world, rank, local):
 
     dec_bytes_all = [layer_decode_bytes(l) for l in range(L)]
     dec_bytes = statistics.mean(dec_bytes_all)
+
     app_step_bytes = sum(n_app * n_app_seqs * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, l, Hkv)) for l in range(L))
     step_bytes = sum(dec_bytes_all) + app_step_bytes
+    # ---- VBR regrade of one layer (last, since it changes that layer's codecs):
+    # K to q4_0 and V to q2_0 where that does not grow the pages
+    regrade = None
+    if w.rot != W.ROT_PROJECTION:
+        rl = L // 2
+        nk, nv = [W.Q4_0] * Hkv, [W.Q2_0] * Hkv
+        try:
+            rbytes = plan.regrade_bytes(rl, nk, nv)
+        except kvq.KVQError:
+            rbytes = None
+        if rbytes:
+            rows = sum(max(0, lengths[rl][s] - w.tail) for s in seqs) * Hkv
+            old_b = rows * bytes_per_token_head(plan, rl, Hkv) / Hkv
+            scratch = torch.empty(rbytes, dtype=torch.uint8, device=dev)
+            ra, rb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                ra.record(stream)
+                plan.regrade(rl, nk, nv, scratch, stream)
+                rb.record(stream)
+            stream.synchronize()
+            plan.check_device_error(stream)
+            new_b = rows * bytes_per_token_head(plan, rl, Hkv) / Hkv
+            r_ms = ra.elapsed_time(rb)
+            moved = old_b + new_b + 2 * rbytes                 # read old rows, write scratch, copy back
+            regrade = {"layer": rl, "ms": r_ms, "rows": rows, "to": ["q4_0", "q2_0"],
+                       "gb_s": moved / (r_ms / 1e3) / 1e9,
+                       "note": "kernel + copy-back of the whole layer pool; bytes = old rows read + new rows "
+                               "written + scratch copied back"}
+
     peaks = measured_peaks()
     peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
@@ -507,6 +537,7 @@ def run_kvq(args, world, rank, local):
         "append_tokens_per_s": append_tps,
         "append_note": f"2048-token chunk appended to all {L} layers (K and V quantized): {app_ms:.3f} ms, "
                        f"{app_bytes / (app_ms / 1e3) / 1e9:.0f} GB/s algorithmic",
+        "regrade": regrade,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "kernel": f"decode_kernel<{w.G}>",
                      "bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
