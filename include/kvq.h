@@ -288,20 +288,30 @@ kvq_status kvq_launch_count(uint64_t* count);
 
 /* --- inspection entry points (used by the parity tests) ------------------ */
 
+/* Row layouts of the append and regrade kernels (the inspection entry points
+ * below run either): KVQ_ROWS_WARP one warp per row (4 values per lane; small
+ * appends, the projection path), KVQ_ROWS_QUAD four threads per row (one
+ * 32-value block each; chunk appends, regrade).  Both must produce the same
+ * bytes. */
+enum kvq_row_layout { KVQ_ROWS_WARP = 0, KVQ_ROWS_QUAD = 1 };
+
 /* Rows in the stored basis, fp32, exactly as the append path computes them
  * before quantization: the staged Hadamard transform (after variance
  * normalisation) for rotated codecs, z = M_h x on the tensor cores for the
  * projection path, the raw values for F16.
- *  x: device fp16 [n][128];  y: device fp32 [n][128] (or [n][r]). */
+ *  x: device fp16 [n][128];  y: device fp32 [n][128] (or [n][r]).
+ *  layout: kvq_row_layout (ignored for the projection path). */
 kvq_status kvq_debug_rotate(const kvq_plan* plan, int layer, int head, int kv, int n, const void* x,
-                            float* y, void* stream);
+                            float* y, int layout, void* stream);
 
 /* The block quantizer alone: fp32 rows in the stored basis -> canonical packed
  * rows.  codec: kvq_codec; r, b: rank and bits (KVQ_RANK only, else ignored).
  *  y: device fp32 [n_rows][128 or r]; codes: device [n_rows][code_bytes];
- *  scales: device [n_rows][scale_bytes]. */
+ *  scales: device [n_rows][scale_bytes].
+ *  layout: kvq_row_layout (KVQ_RANK: KVQ_ROWS_WARP only, else
+ *  KVQ_ERR_UNSUPPORTED). */
 kvq_status kvq_debug_quantize_f32(int codec, int r, int b, int n_rows, const float* y, void* codes,
-                                  void* scales, void* stream);
+                                  void* scales, int layout, void* stream);
 
 #ifdef __cplusplus
 }

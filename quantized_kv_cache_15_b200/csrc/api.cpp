@@ -775,8 +775,9 @@ kvq_status kvq_check_device_error(kvq_plan* p, void* stream) {
 }
 
 kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int n, const void* x, float* y,
-                            void* stream) {
+                            int layout, void* stream) {
   if (!p || !x || !y) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (layout != KVQ_ROWS_WARP && layout != KVQ_ROWS_QUAD) return fail(KVQ_ERR_INVALID_ARG, "bad row layout");
   if (layer < 0 || layer >= p->L || head < 0 || head >= p->Hkv || (kv != 0 && kv != 1) || n < 0)
     return fail(KVQ_ERR_INVALID_ARG, "argument out of range");
   const HeadInfo& h = p->head(layer, head);
@@ -793,18 +794,22 @@ kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int 
     return KVQ_OK;
   }
   const float* inv = p->d_inv ? p->d_inv + (((size_t)layer * p->Hkv + head) * 2 + kv) * D : nullptr;
-  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, n, (const __half*)x, y, (cudaStream_t)stream);
+  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, n, (const __half*)x, y, layout == KVQ_ROWS_QUAD,
+                                      (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "debug_rotate launch");
   return KVQ_OK;
 }
 
 kvq_status kvq_debug_quantize_f32(int codec, int r, int b, int n_rows, const float* y, void* codes, void* scales,
-                                  void* stream) {
+                                  int layout, void* stream) {
   if (!valid_codec(codec)) return fail(KVQ_ERR_UNSUPPORTED, "bad codec");
+  if (layout != KVQ_ROWS_WARP && layout != KVQ_ROWS_QUAD) return fail(KVQ_ERR_INVALID_ARG, "bad row layout");
+  if (layout == KVQ_ROWS_QUAD && codec == KVQ_RANK) return fail(KVQ_ERR_UNSUPPORTED, "rank rows are warp rows");
   if (codec == KVQ_RANK && (!valid_rank(r) || b < 1 || b > 4)) return fail(KVQ_ERR_UNSUPPORTED, "bad rank or bits");
   if (n_rows < 0 || !y || !codes || (!scales && codec != KVQ_F16)) return fail(KVQ_ERR_INVALID_ARG, "bad argument");
   if (codec != KVQ_RANK) r = D;
-  cudaError_t e = launch_debug_quantize(codec, r, b, n_rows, y, (uint8_t*)codes, (uint8_t*)scales, (cudaStream_t)stream);
+  cudaError_t e = launch_debug_quantize(codec, r, b, n_rows, y, (uint8_t*)codes, (uint8_t*)scales,
+                                        layout == KVQ_ROWS_QUAD, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "debug_quantize launch");
   return KVQ_OK;
 }

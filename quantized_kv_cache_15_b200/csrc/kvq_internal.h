@@ -221,9 +221,9 @@ cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t
 cudaError_t launch_project(const ProjParams& p, int n_tiles, int n_heads, cudaStream_t s);
 cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __half* x, float* inv, cudaStream_t s);
 cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, int n, const __half* x,
-                                float* y, cudaStream_t s);
+                                float* y, bool quad, cudaStream_t s);
 cudaError_t launch_debug_quantize(int codec, int r, int b, int n, const float* y, uint8_t* codes, uint8_t* scales,
-                                  cudaStream_t s);
+                                  bool quad, cudaStream_t s);
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G);
 constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)16 << 20;   // = KVQ_NOALLOC_SCRATCH_BYTES
 cudaError_t noalloc_scratch(void** out);

@@ -290,4 +290,278 @@ __device__ __forceinline__ void lane_codes(const uint8_t* plane, int cb, int t, 
   }
 }
 
+// ---- four threads per row, one 32-value block each
+//
+// Lane q = threadIdx.x & 3 of an aligned group of four ("quad") holds values
+// 32q .. 32q+31 of the row in registers.  The Hadamard stages h = 1 .. 16 stay
+// inside the thread, h = 32 and 64 pair the quad's lanes through shuffles, and a
+// block's scale, codes and packing need no communication at all.  Every value
+// goes through the same correctly rounded binary32 operations in the same order as
+// in the warp quantizer above (fwht_row, quantize4), so the stored bytes are the
+// same.  Neighbouring quads own consecutive tokens of one (kv head, K|V), so the
+// interleaved K planes and the row-major V planes are written in coalesced runs.
+
+// The quad's lanes within the warp (shuffle member mask); all four lanes of a
+// quad always take the same path.
+__device__ __forceinline__ unsigned quad_mask() { return 0xfu << (threadIdx.x & 28); }
+
+// Staged Hadamard transform (h = 1, 2, ..., 64, then x c) of the quad's row.
+__device__ __forceinline__ void fwht_quad(float v[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+  const unsigned mask = quad_mask();
+  const int q = threadIdx.x & 3;
+#pragma unroll
+  for (int m = 1; m < 4; m <<= 1) {  // h = 32 m
+    const bool upper = (q & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float o = __shfl_xor_sync(mask, v[i], m);
+      v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+    }
+  }
+  const float c = hadamard_c();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], c);
+}
+
+// The stored basis of the quad's raw row: x * inv_s (variance normalisation) and
+// the staged Hadamard transform, as transform_row above.  inv_s: the row's 128
+// factors.
+__device__ __forceinline__ void transform_row_quad(float v[32], int rot, const float* inv_s) {
+  if (rot == KVQ_ROT_NONE) return;
+  if (rot == KVQ_ROT_VARNORM_HADAMARD) {
+    const float4* s4 = reinterpret_cast<const float4*>(inv_s) + 8 * (threadIdx.x & 3);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 s = s4[c];
+      v[4 * c] = __fmul_rn(v[4 * c], s.x); v[4 * c + 1] = __fmul_rn(v[4 * c + 1], s.y);
+      v[4 * c + 2] = __fmul_rn(v[4 * c + 2], s.z); v[4 * c + 3] = __fmul_rn(v[4 * c + 3], s.w);
+    }
+  }
+  fwht_quad(v);
+}
+
+// 16 bytes of raw fp16 values -> 8 floats.
+__device__ __forceinline__ void chunk_to_float(const uint4 w, float* x) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+    x[2 * k] = f.x; x[2 * k + 1] = f.y;
+  }
+}
+
+// Address of word wi of the canonical packed row of token row t: K planes are
+// interleaved in 16-byte chunks, V planes row-major (cb bytes per row).
+__device__ __forceinline__ uint8_t* row_word_ptr(uint8_t* codes, bool kplane, int cb, int t, int wi) {
+  return kplane ? codes + ((wi / 4) * PAGE + t) * 16 + 4 * (wi % 4) : codes + t * cb + 4 * wi;
+}
+__device__ __forceinline__ const uint8_t* row_word_ptr(const uint8_t* codes, bool kplane, int cb, int t, int wi) {
+  return kplane ? codes + ((wi / 4) * PAGE + t) * 16 + 4 * (wi % 4) : codes + t * cb + 4 * wi;
+}
+
+// Store / load words [first + W b, first + W (b + 1)) of a row: the block's share
+// of a plane of W-bit fields (W words per 32-value block; 8 words = two chunks).
+template <int W>
+__device__ __forceinline__ void store_plane(uint8_t* codes, bool kplane, int cb, int t, int first, int b,
+                                            const uint32_t w[W]) {
+  const int wi = first + W * b;
+  if constexpr (W == 8) {
+    *reinterpret_cast<uint4*>(row_word_ptr(codes, kplane, cb, t, wi)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(row_word_ptr(codes, kplane, cb, t, wi + 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+  } else if constexpr (W == 4) {
+    *reinterpret_cast<uint4*>(row_word_ptr(codes, kplane, cb, t, wi)) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (W == 2) {
+    *reinterpret_cast<uint2*>(row_word_ptr(codes, kplane, cb, t, wi)) = make_uint2(w[0], w[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(row_word_ptr(codes, kplane, cb, t, wi)) = w[0];
+  }
+}
+template <int W>
+__device__ __forceinline__ void load_plane(const uint8_t* codes, bool kplane, int cb, int t, int first, int b,
+                                           uint32_t w[W]) {
+  const int wi = first + W * b;
+  if constexpr (W == 8 || W == 4) {
+#pragma unroll
+    for (int h = 0; h < W / 4; ++h) {
+      const uint4 x = *reinterpret_cast<const uint4*>(row_word_ptr(codes, kplane, cb, t, wi + 4 * h));
+      w[4 * h] = x.x; w[4 * h + 1] = x.y; w[4 * h + 2] = x.z; w[4 * h + 3] = x.w;
+    }
+  } else if constexpr (W == 2) {
+    const uint2 x = *reinterpret_cast<const uint2*>(row_word_ptr(codes, kplane, cb, t, wi));
+    w[0] = x.x; w[1] = x.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t*>(row_word_ptr(codes, kplane, cb, t, wi));
+  }
+}
+
+// The low / high planes of a BITS-bit codec: 8, 4, 2 one plane; 6 = 4 + 2,
+// 5 = 4 + 1, 3 = 2 + 1 (the high plane after the 128 * LO / 8 bytes of the low).
+template <int BITS> struct Planes {
+  static constexpr int LO = (BITS == 6 || BITS == 5) ? 4 : (BITS == 3 ? 2 : BITS);
+  static constexpr int HI = BITS - LO;
+};
+
+// Quantize this lane's block b = q (values v[0..31] in the stored basis) with a
+// _0 (KIND 0) or _1 (KIND 1) codec of BITS bits and write its codes to token row
+// t; returns the block's scale word (_0: d in the low half; _1: d | m << 16).
+template <int KIND, int BITS>
+__device__ __forceinline__ uint32_t quantize_block_quad(const float v[32], uint8_t* codes, int t, bool kplane,
+                                                        int cb) {
+  constexpr int LO = Planes<BITS>::LO, HI = Planes<BITS>::HI;
+  const int b = threadIdx.x & 3;
+  uint32_t u[32];
+  uint32_t sc;
+  if constexpr (KIND == 1) {
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int j = 1; j < 32; ++j) { mn = fminf(mn, v[j]); mx = fmaxf(mx, v[j]); }
+    mn = fminf(fmaxf(mn, -65504.0f), 65504.0f);
+    const __half mh = __float2half_rd(mn);
+    const float mf = __half2float(mh);
+    constexpr int umax = (1 << BITS) - 1;
+    float d = __fdiv_rn(__fsub_rn(mx, mf), (float)umax);
+    d = fminf(d, 65504.0f);
+    const __half dh = __float2half_rn(d);
+    const float df = __half2float(dh);
+    sc = (uint32_t)__half_as_ushort(dh) | ((uint32_t)__half_as_ushort(mh) << 16);
+    const float inv = __fdiv_rn(1.0f, df);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float r = rintf(__fmul_rn(__fsub_rn(v[j], mf), inv));
+      r = fminf(fmaxf(r, 0.0f), (float)umax);
+      u[j] = df == 0.0f ? 0u : (uint32_t)(int)r;
+    }
+  } else {
+    float amax = fabsf(v[0]);
+#pragma unroll
+    for (int j = 1; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    constexpr int half = 1 << (BITS - 1);
+    float d = __fdiv_rn(amax, (float)(half - 1));
+    d = fminf(d, 65504.0f);
+    const __half dh = __float2half_rn(d);
+    const float df = __half2float(dh);
+    sc = __half_as_ushort(dh);
+    const float inv = __fdiv_rn(1.0f, df);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float r = rintf(__fmul_rn(v[j], inv));
+      r = fminf(fmaxf(r, (float)(-half)), (float)(half - 1));
+      u[j] = df == 0.0f ? (uint32_t)half : (uint32_t)((int)r + half);
+    }
+  }
+  {
+    constexpr int per = 32 / LO;
+    uint32_t w[LO];
+#pragma unroll
+    for (int k = 0; k < LO; ++k) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int i = 0; i < per; ++i) x |= (u[k * per + i] & ((1u << LO) - 1u)) << (LO * i);
+      w[k] = x;
+    }
+    store_plane<LO>(codes, kplane, cb, t, 0, b, w);
+  }
+  if constexpr (HI > 0) {
+    constexpr int per = 32 / HI;
+    uint32_t w[HI];
+#pragma unroll
+    for (int k = 0; k < HI; ++k) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int i = 0; i < per; ++i) x |= ((u[k * per + i] >> LO) & ((1u << HI) - 1u)) << (HI * i);
+      w[k] = x;
+    }
+    store_plane<HI>(codes, kplane, cb, t, 4 * LO, b, w);
+  }
+  return sc;
+}
+
+// Write the quad's row (v: this lane's block; stored basis, or raw values for
+// F16) with `codec` to token row t: F16 as fp16 values, block codecs through
+// quantize_block_quad, the four scale words written by lane 0 of the quad.
+__device__ __forceinline__ void quantize_row_quad(int codec, const float v[32], uint8_t* codes, uint8_t* scales,
+                                                  int t, bool kplane, int cb, int sb) {
+  const int b = threadIdx.x & 3;
+  uint32_t sc = 0;
+  switch (codec) {
+    case KVQ_F16:
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __half2 hv = __floats2half2_rn(v[8 * c + 2 * k], v[8 * c + 2 * k + 1]);
+          w[k] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(row_word_ptr(codes, kplane, cb, t, 16 * b + 4 * c)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      return;
+    case KVQ_Q8_0: sc = quantize_block_quad<0, 8>(v, codes, t, kplane, cb); break;
+    case KVQ_Q6_0: sc = quantize_block_quad<0, 6>(v, codes, t, kplane, cb); break;
+    case KVQ_Q5_0: sc = quantize_block_quad<0, 5>(v, codes, t, kplane, cb); break;
+    case KVQ_Q4_0: sc = quantize_block_quad<0, 4>(v, codes, t, kplane, cb); break;
+    case KVQ_Q3_0: sc = quantize_block_quad<0, 3>(v, codes, t, kplane, cb); break;
+    case KVQ_Q2_0: sc = quantize_block_quad<0, 2>(v, codes, t, kplane, cb); break;
+    case KVQ_Q8_1: sc = quantize_block_quad<1, 8>(v, codes, t, kplane, cb); break;
+    case KVQ_Q6_1: sc = quantize_block_quad<1, 6>(v, codes, t, kplane, cb); break;
+    case KVQ_Q5_1: sc = quantize_block_quad<1, 5>(v, codes, t, kplane, cb); break;
+    case KVQ_Q4_1: sc = quantize_block_quad<1, 4>(v, codes, t, kplane, cb); break;
+    case KVQ_Q3_1: sc = quantize_block_quad<1, 3>(v, codes, t, kplane, cb); break;
+    case KVQ_Q2_1: sc = quantize_block_quad<1, 2>(v, codes, t, kplane, cb); break;
+    default: return;
+  }
+  const unsigned mask = quad_mask();
+  const uint32_t s1 = __shfl_down_sync(mask, sc, 1, 4);
+  const uint32_t s2 = __shfl_down_sync(mask, sc, 2, 4);
+  const uint32_t s3 = __shfl_down_sync(mask, sc, 3, 4);
+  if (b == 0) {
+    if (codec_is_asym(codec))
+      *reinterpret_cast<uint4*>(scales + t * sb) = make_uint4(sc, s1, s2, s3);
+    else
+      *reinterpret_cast<uint2*>(scales + t * sb) = make_uint2(sc | (s1 << 16), s2 | (s3 << 16));
+  }
+}
+
+// Exact dequantization of this lane's block b = q of token row t of a _0 (KIND 0)
+// or _1 (KIND 1) codec of BITS bits into the stored basis: _0 (u - 2^(b-1)) d,
+// _1 u d + m.
+template <int KIND, int BITS>
+__device__ __forceinline__ void dequantize_block_quad(const uint8_t* codes, const uint8_t* scales, int t, bool kplane,
+                                                      int cb, int sb, float v[32]) {
+  constexpr int LO = Planes<BITS>::LO, HI = Planes<BITS>::HI;
+  const int b = threadIdx.x & 3;
+  float d, off;
+  if constexpr (KIND == 1) {
+    const __half2 dm = *reinterpret_cast<const __half2*>(scales + t * sb + 4 * b);
+    d = __low2float(dm);
+    off = __high2float(dm);
+  } else {
+    d = __half2float(*reinterpret_cast<const __half*>(scales + t * sb + 2 * b));
+    off = -(float)(1 << (BITS - 1)) * d;
+  }
+  uint32_t w0[LO];
+  load_plane<LO>(codes, kplane, cb, t, 0, b, w0);
+  uint32_t w1[HI > 0 ? HI : 1];
+  if constexpr (HI > 0) load_plane<HI>(codes, kplane, cb, t, 4 * LO, b, w1);
+  constexpr int per0 = 32 / LO;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    uint32_t u = (w0[j / per0] >> (LO * (j % per0))) & ((1u << LO) - 1u);
+    if constexpr (HI > 0) {
+      constexpr int per1 = 32 / (HI > 0 ? HI : 1);
+      u |= ((w1[j / per1] >> (HI * (j % per1))) & ((1u << HI) - 1u)) << LO;
+    }
+    v[j] = fmaf((float)u, d, off);
+  }
+}
+
 }  // namespace kvq

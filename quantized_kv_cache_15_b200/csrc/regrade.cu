@@ -15,67 +15,72 @@
 
 namespace kvq {
 
+// Four threads per (row, kv head, K|V), one 32-value block each (quad layout:
+// quant.cuh); consecutive quads take consecutive rows, so both pools are read and
+// written in coalesced runs.
 __global__ void __launch_bounds__(256) regrade_kernel(const __grid_constant__ RegradeParams p) {
-  const int lane = threadIdx.x & 31;
-  const long gw = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const long row = gw / (p.Hkv * 2);
-  if (row >= p.total_rows) return;
-  const int rem = (int)(gw % (p.Hkv * 2));
-  const int head = rem >> 1, kv = rem & 1;
-  int si = 0;
-  for (int i = 1; i < p.n_seqs; ++i)
-    if (p.row0[i] <= row) si = i;
-  const long pos = row - p.row0[si];
-  const int pid = p.block_table[(size_t)p.seq[si] * p.max_pages_per_seq + pos / PAGE];
+  const long task = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 2;
+  const int q = threadIdx.x & 3;
+  if (task >= p.total_rows * p.Hkv * 2) return;  // whole quads leave together
+  const int hk = (int)(task / p.total_rows);
+  const long row = task - (long)hk * p.total_rows;
+  const int head = hk >> 1, kv = hk & 1;
+  int lo = 0, hi = p.n_seqs - 1;                 // the last sequence whose first row is <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.row0[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  const long pos = row - p.row0[lo];
+  const int pid = p.block_table[(size_t)p.seq[lo] * p.max_pages_per_seq + pos / PAGE];
   if (pid < 0) {
-    if (lane == 0) atomicOr(p.err, ERR_NO_PAGE);
+    if (q == 0) atomicOr(p.err, ERR_NO_PAGE);
     return;
   }
   const int t = (int)(pos % PAGE);
+  const bool kplane = kv == 0;
   const HeadInfo& hs = p.src[head];
   const HeadInfo& hd = p.dst[head];
-  const int cs = kv ? hs.vcodec : hs.kcodec, bs = kv ? hs.vbits : hs.kbits;
-  const int cd = kv ? hd.vcodec : hd.kcodec, bd = kv ? hd.vbits : hd.kbits;
+  const int cs = kv ? hs.vcodec : hs.kcodec;
+  const int cd = kv ? hd.vcodec : hd.kcodec;
   const int cbs = kv ? hs.cbV : hs.cbK, sbs = kv ? hs.sbV : hs.sbK;
   const uint8_t* region = p.src_pool + (size_t)pid * p.src_page_bytes + hs.off;
   const uint8_t* codes = kv ? region + PAGE * (hs.cbK + hs.sbK) : region;
   const uint8_t* scales = codes + PAGE * cbs;
-  float x[4];
-  if (cs == KVQ_F16) {
-    const uint8_t* src = codes + (kv == 0 ? kplane_off(cbs, t, 8 * lane) : t * cbs + 8 * lane);
-    const uint2 w = *reinterpret_cast<const uint2*>(src);
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-    transform_row(x, cd, p.rot, p.inv_s ? p.inv_s + ((size_t)head * 2 + kv) * D : nullptr);
-  } else {
-    // exact dequantization in the stored basis: _0 code * d, _1 u * d + m
-    uint32_t u[4];
-    lane_codes(codes, cbs, t, kv == 0, bs, D, lane, u);
-    const int b = (4 * lane) / 32;
-    float d, off;
-    if (codec_is_asym(cs)) {
-      const __half2 dm = *reinterpret_cast<const __half2*>(scales + t * sbs + 4 * b);
-      d = __low2float(dm);
-      off = __high2float(dm);
-    } else {
-      d = __half2float(*reinterpret_cast<const __half*>(scales + t * sbs + 2 * b));
-      off = -(float)(1 << (bs - 1)) * d;
-    }
+  float v[32];
+  switch (cs) {
+    case KVQ_F16: {
+      // raw rows: into the stored basis of the new codec
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = fmaf((float)u[i], d, off);
+      for (int c = 0; c < 4; ++c)
+        chunk_to_float(*reinterpret_cast<const uint4*>(row_word_ptr(codes, kplane, cbs, t, 16 * q + 4 * c)), v + 8 * c);
+      if (cd != KVQ_F16)
+        transform_row_quad(v, p.rot, p.inv_s ? p.inv_s + ((size_t)head * 2 + kv) * D : nullptr);
+    } break;
+    case KVQ_Q8_0: dequantize_block_quad<0, 8>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q6_0: dequantize_block_quad<0, 6>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q5_0: dequantize_block_quad<0, 5>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q4_0: dequantize_block_quad<0, 4>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q3_0: dequantize_block_quad<0, 3>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q2_0: dequantize_block_quad<0, 2>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q8_1: dequantize_block_quad<1, 8>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q6_1: dequantize_block_quad<1, 6>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q5_1: dequantize_block_quad<1, 5>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q4_1: dequantize_block_quad<1, 4>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q3_1: dequantize_block_quad<1, 3>(codes, scales, t, kplane, cbs, sbs, v); break;
+    case KVQ_Q2_1: dequantize_block_quad<1, 2>(codes, scales, t, kplane, cbs, sbs, v); break;
+    default: return;
   }
   uint8_t* dregion = p.dst_pool + (size_t)pid * p.dst_page_bytes + hd.off;
-  const int cbd = kv ? hd.cbV : hd.cbK;
+  const int cbd = kv ? hd.cbV : hd.cbK, sbd = kv ? hd.sbV : hd.sbK;
   uint8_t* dcodes = kv ? dregion + PAGE * (hd.cbK + hd.sbK) : dregion;
   uint8_t* dscales = dcodes + PAGE * cbd;
-  quantize_store_row(x, cd, D, bd, dcodes, dscales, t, kv == 0);
+  quantize_row_quad(cd, v, dcodes, dscales, t, kplane, cbd, sbd);
 }
 
 cudaError_t launch_regrade(const RegradeParams& p, cudaStream_t s) {
   if (p.total_rows <= 0) return cudaSuccess;
-  const long warps = p.total_rows * p.Hkv * 2;
-  regrade_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(p);
+  const long threads = 4L * p.total_rows * p.Hkv * 2;
+  regrade_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(p);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -18,6 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK, Q5_0, Q5_1 = range(14)
+ROWS_WARP, ROWS_QUAD = 0, 1          # kvq_row_layout
 ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION = range(4)
 HEAD_DIM = 128
 PAGE_TOKENS = 64
@@ -52,8 +53,8 @@ SIGNATURES = {
     "kvq_last_error": (ctypes.c_char_p, []),
     "kvq_launch_count": (_I, [ctypes.POINTER(ctypes.c_uint64)]),
     "kvq_cobra_allocate": (_I, [_I, _P, ctypes.c_double, _P, _IP, _IP, _IP]),
-    "kvq_debug_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
-    "kvq_debug_quantize_f32": (_I, [_I, _I, _I, _I, _P, _P, _P, _P]),
+    "kvq_debug_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P]),
+    "kvq_debug_quantize_f32": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P]),
 }
 
 
@@ -233,8 +234,10 @@ class Plan:
     def check_device_error(self, stream=None):
         _check(lib().kvq_check_device_error(self._h, _stream(stream)))
 
-    def debug_rotate(self, layer: int, head: int, kv: int, x: torch.Tensor, y: torch.Tensor, stream=None):
-        _check(lib().kvq_debug_rotate(self._h, layer, head, kv, x.shape[0], _ptr(x), _ptr(y), _stream(stream)))
+    def debug_rotate(self, layer: int, head: int, kv: int, x: torch.Tensor, y: torch.Tensor, layout: int = 0,
+                     stream=None):
+        _check(lib().kvq_debug_rotate(self._h, layer, head, kv, x.shape[0], _ptr(x), _ptr(y), layout,
+                                      _stream(stream)))
 
 
 def cobra_allocate(lambdas: np.ndarray, bpd: float, eps) -> tuple:
@@ -279,6 +282,6 @@ def calibrate_varnorm(x: torch.Tensor, n_channels: int, row_stride: int, inv_rms
 
 
 def debug_quantize_f32(codec: int, r: int, b: int, y: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
-                       stream=None):
-    _check(lib().kvq_debug_quantize_f32(codec, r, b, y.shape[0], _ptr(y), _ptr(codes), _ptr(scales),
+                       layout: int = 0, stream=None):
+    _check(lib().kvq_debug_quantize_f32(codec, r, b, y.shape[0], _ptr(y), _ptr(codes), _ptr(scales), layout,
                                         _stream(stream)))

@@ -53,3 +53,14 @@ def test_library_links_no_oracle_and_no_torch():
     assert "orc_" not in out and "torch" not in out and "c10" not in out
     deps = subprocess.run(["ldd", path], capture_output=True, text=True).stdout
     assert "liboracle" not in deps and "libtorch" not in deps
+
+
+def test_debug_quantize_rejects_bad_row_layouts_before_any_launch(libkvq):
+    """Argument checks run on the host: no device is touched."""
+    from quantized_kv_cache_15_b200 import kvq
+    f = libkvq.kvq_debug_quantize_f32
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.c_void_p]
+    fake = ctypes.c_void_p(16)
+    assert f(kvq.RANK, 64, 2, 1, fake, fake, fake, kvq.ROWS_QUAD, None) == 2       # KVQ_ERR_UNSUPPORTED
+    assert f(kvq.Q4_0, 128, 0, 1, fake, fake, fake, 7, None) == 1                  # KVQ_ERR_INVALID_ARG

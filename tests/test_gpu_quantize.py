@@ -33,23 +33,25 @@ def _rows(seed, n, width=128):
     return y.astype(np.float32)
 
 
-def _gpu_quantize(codec, y, r=128, b=0):
+def _gpu_quantize(codec, y, r=128, b=0, layout=kvq.ROWS_WARP):
     cb, sb = oracle.row_bytes(codec, r, b)
     yd = torch.from_numpy(y).cuda()
     codes = torch.zeros((y.shape[0], cb), dtype=torch.uint8, device="cuda")
     scales = torch.zeros((y.shape[0], max(sb, 2)), dtype=torch.uint8, device="cuda")
-    kvq.debug_quantize_f32(codec, r, b, yd, codes, scales)
+    kvq.debug_quantize_f32(codec, r, b, yd, codes, scales, layout)
     torch.cuda.synchronize()
     sc = scales.cpu().numpy()[:, :sb].copy().view(np.uint16) if sb else np.zeros((y.shape[0], 0), np.uint16)
     return codes.cpu().numpy(), sc
 
 
+@pytest.mark.parametrize("layout", [kvq.ROWS_WARP, kvq.ROWS_QUAD])
 @pytest.mark.parametrize("codec", CODECS)
-def test_block_quantizer_bit_exact(codec):
+def test_block_quantizer_bit_exact(codec, layout):
+    """Both row layouts (a warp per row; four threads per row) against the oracle."""
     y = _rows(codec, 3000)
     if codec == kvq.F16:
         y = y.astype(np.float16).astype(np.float32)
-    gc, gs = _gpu_quantize(codec, y)
+    gc, gs = _gpu_quantize(codec, y, layout=layout)
     oc, os_ = oracle.quantize_rows(codec, y)
     assert np.array_equal(gc, oc)
     assert np.array_equal(gs, os_)
@@ -65,8 +67,9 @@ def test_rank_quantizer_bit_exact(r, b):
     assert np.array_equal(gs, os_)
 
 
+@pytest.mark.parametrize("layout", [kvq.ROWS_WARP, kvq.ROWS_QUAD])
 @pytest.mark.parametrize("rot", [W.ROT_HADAMARD, W.ROT_VARNORM_HADAMARD])
-def test_rotation_bit_exact(rot):
+def test_rotation_bit_exact(rot, layout):
     w = W.make_workload(5 if rot == W.ROT_VARNORM_HADAMARD else 1, "small")
     w.rot = rot
     plan = H.make_plan(w)
@@ -74,7 +77,7 @@ def test_rotation_bit_exact(rot):
     inv = H.gpu_inv_rms(w)[0, 1, 0] if rot == W.ROT_VARNORM_HADAMARD else None
     for kv in (0, 1):
         y = torch.empty((700, 128), dtype=torch.float32, device="cuda")
-        plan.debug_rotate(0, 1, kv, x.cuda(), y)
+        plan.debug_rotate(0, 1, kv, x.cuda(), y, layout)
         torch.cuda.synchronize()
         invk = None
         if inv is not None:
