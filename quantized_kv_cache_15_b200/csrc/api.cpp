@@ -492,13 +492,24 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
     maxpages = std::max(maxpages, pages);
   }
   dp.stage_bytes = p->stage_bytes[layer];
+  // The consumer warps keep their weight tables in the K region of their current
+  // stage unless some head's (or the tail's) K rows are smaller than a table.
+  dp.wtab_smem = 0;
+  for (int h = 0; h < p->Hkv; ++h) {
+    const HeadInfo& hi = p->head(layer, h);
+    if ((uint32_t)PAGE * (uint32_t)(hi.cbK + hi.sbK) < wtab_bytes(p->G)) dp.wtab_smem = 1;
+  }
+  if (p->T > 0 && (uint32_t)TAIL_TOK * (uint32_t)(2 * D) < wtab_bytes(p->G)) dp.wtab_smem = 1;
   // Stage ring: one stage per consumer warp at least, deeper while the CTAs per SM
   // that the register allocation aims at still fit in shared memory.
   const int want_ctas = NCW <= 4 ? 3 : 2;
   dp.n_stages = NCW;
   for (int ns = 8; ns > NCW; --ns)
-    if (decode_smem_bytes(dp.stage_bytes, ns, p->G) + 1024 <= (228 * 1024) / want_ctas) { dp.n_stages = ns; break; }
-  const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G);
+    if (decode_smem_bytes(dp.stage_bytes, ns, p->G, dp.wtab_smem) + 1024 <= (228 * 1024) / want_ctas) {
+      dp.n_stages = ns;
+      break;
+    }
+  const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G, dp.wtab_smem);
   // Split size: the candidate with the smallest estimated makespan, counted in waves
   // of resident CTAs (registers and shared memory both counted) times the pages of
   // a split plus a fixed cost of about three pages (query preparation, publishing

@@ -217,7 +217,7 @@ __device__ __forceinline__ void v_lane(int vc, int vbits, int n, int cb, int sb,
 __host__ __device__ inline size_t post_bytes(int G) {
   return (size_t)NCW * G * (D + 4) * 4 + (size_t)2 * G * D * 4 + (size_t)2 * G * 4 + 16;
 }
-size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
+size_t decode_smem_bytes(int stage_bytes, int n_stages, int G, bool wtab_smem) {
   size_t ring = (size_t)stage_bytes * n_stages;
   // after the loop the ring's bytes hold the post region and at least one head's
   // staged partials (MAX_SPLITS of them) for the last CTA's merge
@@ -231,7 +231,7 @@ size_t decode_smem_bytes(int stage_bytes, int n_stages, int G) {
   a += (size_t)G * D * 2;            // qi16
   a += (size_t)2 * G * 64 * 4;       // pair tables
   a = (a + 15) & ~(size_t)15;
-  a += (size_t)NCW * 32 * (4 * G + 1) * 8;   // per-warp weight tables
+  if (wtab_smem) a += (size_t)NCW * wtab_bytes(G);   // per-warp weight tables
   a += (size_t)(2 * 8 + 2) * 8;      // mbarriers: ring full / empty, merge staging
   return a;
 }
@@ -334,7 +334,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   int16_t* qi16 = reinterpret_cast<int16_t*>(smem + off); off += (size_t)G * D * 2;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + off); off += (size_t)2 * G * 64 * 4;
   off = (off + 15) & ~(size_t)15;
-  uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off); off += (size_t)NCW * 32 * (4 * G + 1) * 8;
+  uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off);         // per-warp weight tables (p.wtab_smem)
+  if (p.wtab_smem) off += (size_t)NCW * wtab_bytes(G);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
   uint64_t* empty = full + 8;
   uint64_t* mmerge = full + 16;                                    // the merge's two staging buffers
@@ -486,8 +487,10 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     // This warp's weight table: (w, w) pairs per token on the fp32 path, int16 pairs
     // per token pair and block on the integer path (same bytes).
     constexpr int PWG = G + 1;                          // fp32 path row: G pairs + pad
-    uint64_t* pw = pw2 + (size_t)warp * 32 * (4 * G + 1);
-    uint32_t* wq = reinterpret_cast<uint32_t*>(pw);
+    // The weight table goes into the K region of the warp's own stage once the
+    // scores are taken (the stage is this warp's until it releases it), or into
+    // the warp's slot of the separate table area when the K rows are too small.
+    const bool wt_stage = (uint32_t)rows * (uint32_t)(cbK + sbK) >= wtab_bytes(G);
     for (int i = warp; i < n_tiles; i += NCW) {
       const int st = i % NS;
       if (!mbar_wait(&full[st], (i / NS) & 1)) atomicOr(p.err, ERR_TIMEOUT);
@@ -496,6 +499,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
       const uint8_t* ks = kp + rows * cbK;
       const uint8_t* vp = ks + rows * sbK;
       const uint8_t* vs = vp + rows * cbV;
+      uint64_t* pw = wt_stage ? reinterpret_cast<uint64_t*>(stages + (size_t)st * p.stage_bytes)
+                              : pw2 + (size_t)warp * (wtab_bytes(G) / 8);
+      uint32_t* wq = reinterpret_cast<uint32_t*>(pw);
       const int tok0 = (pg0 + i) * rows;
       const int nvalid = min(rows, seg_tokens - tok0);
       float s0[G], s1[G];
@@ -534,6 +540,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
         for (int b = 0; b < 4; ++b) off[g][b] *= alpha;
         m[g] = mnew;
       }
+      __syncwarp();                         // every lane's key reads are done: the K region may be reused
       switch (vclass) {
         case 8: value_tile_int<G, 8>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
         case 4: value_tile_int<G, 4>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
@@ -588,6 +595,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
             __syncwarp();
           }
       }
+      // the weight-table stores (generic proxy) must land before the stage's next
+      // bulk copy (async proxy) overwrites it
+      fence_proxy_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
@@ -777,7 +787,7 @@ int decode_max_smem() { return 227 * 1024; }
 
 template <int G>
 static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
-  const size_t smem = decode_smem_bytes(p.stage_bytes, p.n_stages, G);
+  const size_t smem = decode_smem_bytes(p.stage_bytes, p.n_stages, G, p.wtab_smem != 0);
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

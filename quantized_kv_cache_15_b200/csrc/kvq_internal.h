@@ -177,6 +177,7 @@ struct DecodeParams {
   int pps;                       // pages per split
   int stage_bytes;               // bytes of one pipeline stage
   int n_stages;                  // 4 or 8
+  int wtab_smem;                 // 1: the weight tables get their own shared memory (some head's K rows are too small)
   float* ws;                     // partials [n_seqs*Hkv][G][MAX_SPLITS][PARTIAL_FLOATS]
   float* qproj;                  // projected queries M_h q [n_seqs][Hq][128] (projection plans)
   int* tickets;                  // [n_seqs*Hkv]
@@ -224,7 +225,12 @@ cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float*
                                 float* y, bool quad, cudaStream_t s);
 cudaError_t launch_debug_quantize(int codec, int r, int b, int n, const float* y, uint8_t* codes, uint8_t* scales,
                                   bool quad, cudaStream_t s);
-size_t decode_smem_bytes(int stage_bytes, int n_stages, int G);
+size_t decode_smem_bytes(int stage_bytes, int n_stages, int G, bool wtab_smem);
+// Bytes of one consumer warp's softmax-weight table: 32 token-pair rows of
+// [4 blocks][G] int16 pairs plus a pad word per block (the fp32 path's (w, w)
+// pairs of 32 tokens take half of it).  It lives in the dead K-code region of the
+// warp's current stage whenever that region is large enough.
+__host__ __device__ constexpr uint32_t wtab_bytes(int G) { return 32u * (4u * (uint32_t)G + 4u) * 4u; }
 constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)16 << 20;   // = KVQ_NOALLOC_SCRATCH_BYTES
 cudaError_t noalloc_scratch(void** out);
 void note_launches(int n);   // counts kernel launches made by the library

@@ -35,13 +35,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Wait for the phase with the given parity to complete; gives up after ~2 s.
+// try_wait that may keep the thread suspended for up to `hint_ns` (it resumes as
+// soon as the phase completes), so a waiting warp takes no issue slots meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete; gives up after ~2 s.  Each
+// try suspends the thread for up to 20 us, so a long wait (a producer whose ring
+// is full, a consumer waiting for its first page) costs a handful of instructions.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < (1u << 26); ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u && globaltimer_ns() - t0 > 2000000000ull) break;
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    if (globaltimer_ns() - t0 > 2000000000ull) break;
   }
   return false;
 }
