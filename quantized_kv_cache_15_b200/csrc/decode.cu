@@ -491,6 +491,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     // scores are taken (the stage is this warp's until it releases it), or into
     // the warp's slot of the separate table area when the K rows are too small.
     const bool wt_stage = (uint32_t)rows * (uint32_t)(cbK + sbK) >= wtab_bytes(G);
+    // 0xF0F0F0F0 and 0x80808080 as run-time values (n_seqs >= 0, so rz == 0)
+    const uint32_t rz = (uint32_t)p.n_seqs >> 31;
+    const uint32_t kM = 0xF0F0F0F0u ^ rz, kC = 0x80808080u ^ rz;
     for (int i = warp; i < n_tiles; i += NCW) {
       const int st = i % NS;
       if (!mbar_wait(&full[st], (i / NS) & 1)) atomicOr(p.err, ERR_TIMEOUT);
@@ -542,33 +545,28 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
       }
       __syncwarp();                         // every lane's key reads are done: the K region may be reused
       switch (vclass) {
-        case 8: value_tile_int<G, 8>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
-        case 4: value_tile_int<G, 4>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
-        case 2: value_tile_int<G, 2>(vasym, vhalf, vp, vs, cbV, sbV, nvalid, lane, blane, wq, p0, p1, pm, O2, off); break;
-        case 42:
-          value_tile_planes<G, 4, 2>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
-                                          pm, O2, off);
+        case 8:
+          if (vasym) value_tile_int<G, 8, true>(vhalf, vp, vs, sbV, nvalid, lane, blane, wq, kM, kC, p0, p1, pm, O2, off);
+          else value_tile_int<G, 8, false>(vhalf, vp, vs, sbV, nvalid, lane, blane, wq, kM, kC, p0, p1, pm, O2, off);
           break;
-        case 41:
-          value_tile_planes<G, 4, 1>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
-                                          pm, O2, off);
+        case 4:
+          if (vasym) value_tile_int<G, 4, true>(vhalf, vp, vs, sbV, nvalid, lane, blane, wq, kM, kC, p0, p1, pm, O2, off);
+          else value_tile_int<G, 4, false>(vhalf, vp, vs, sbV, nvalid, lane, blane, wq, kM, kC, p0, p1, pm, O2, off);
           break;
-        case 21:
-          value_tile_planes<G, 2, 1>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
-                                          pm, O2, off);
+        case 2:
+          if (vasym) value_tile_int<G, 2, true>(vhalf, vp, vs, sbV, nvalid, lane, blane, wq, kM, kC, p0, p1, pm, O2, off);
+          else value_tile_int<G, 2, false>(vhalf, vp, vs, sbV, nvalid, lane, blane, wq, kM, kC, p0, p1, pm, O2, off);
           break;
-        case 40:
-          value_tile_planes<G, 4, 0>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
-                                          pm, O2, off);
-          break;
-        case 20:
-          value_tile_planes<G, 2, 0>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
-                                          pm, O2, off);
-          break;
-        case 10:
-          value_tile_planes<G, 1, 0>(nbV, blkV, vcl, vasym, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1,
-                                          pm, O2, off);
-          break;
+#define KVQ_PLANES(LO, HI, ASYM)                                                                                      \
+  value_tile_planes<G, LO, HI, ASYM>(nbV, blkV, vcl, vcen, voffB, vp, vs, cbV, sbV, nvalid, lane, wq, p0, p1, pm, O2, \
+                                     off)
+        case 42: if (vasym) KVQ_PLANES(4, 2, true); else KVQ_PLANES(4, 2, false); break;
+        case 41: if (vasym) KVQ_PLANES(4, 1, true); else KVQ_PLANES(4, 1, false); break;
+        case 21: if (vasym) KVQ_PLANES(2, 1, true); else KVQ_PLANES(2, 1, false); break;
+        case 40: KVQ_PLANES(4, 0, false); break;
+        case 20: KVQ_PLANES(2, 0, false); break;
+        case 10: KVQ_PLANES(1, 0, false); break;
+#undef KVQ_PLANES
         default:
           // fp32 path: dequantized values times the softmax numerator, packed FMAs
 #pragma unroll

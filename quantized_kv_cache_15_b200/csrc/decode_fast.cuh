@@ -450,23 +450,29 @@ __device__ __forceinline__ void load_wrow(const uint32_t* w, uint32_t out[G]) {
 // centred code times the class factor.
 // VB 8: slots = channels 0,1,2,3, factor 1.  VB 4: slots = channels 0, 2, 1, 3,
 // factor 16.  VB 2: slots = channels 0,1,2,3, factor 64.
+// The row stride of a V plane of VB-bit codes is 16 VB bytes (128 channels), a
+// compile-time constant.  kM / kC hold 0xF0F0F0F0 and 0x80808080 in registers (the
+// caller derives them from a run-time value), so that "(x & mask) ^ 0x80" takes one
+// three-input logic op rather than two with immediates.
 template <int G, int VB>
-__device__ __forceinline__ void value_dots(const uint8_t* vp, int cbV, int lane, const uint32_t* wr, int acc[G][4]) {
+__device__ __forceinline__ void value_dots(const uint8_t* vp, int lane, const uint32_t* wr, uint32_t kM, uint32_t kC,
+                                           int acc[G][4]) {
   constexpr int WRS = wq_row_words<G>();
-#pragma unroll 4
+  constexpr int cbV = 16 * VB;
+#pragma unroll 8
   for (int j = 0; j < 32; ++j) {
     uint32_t X, Y;
     if (VB == 8) {
       const uint32_t a = *reinterpret_cast<const uint32_t*>(vp + j * cbV + 4 * lane);
       const uint32_t b = *reinterpret_cast<const uint32_t*>(vp + (j + 32) * cbV + 4 * lane);
-      X = prmt(a, b, 0x5140u) ^ 0x80808080u;          // u - 128 as a signed byte
-      Y = prmt(a, b, 0x7362u) ^ 0x80808080u;
+      X = prmt(a, b, 0x5140u) ^ kC;                   // u - 128 as a signed byte
+      Y = prmt(a, b, 0x7362u) ^ kC;
     } else if (VB == 4) {
       const uint32_t a = *reinterpret_cast<const uint16_t*>(vp + j * cbV + 2 * lane);
       const uint32_t b = *reinterpret_cast<const uint16_t*>(vp + (j + 32) * cbV + 2 * lane);
       const uint32_t z = prmt(a, b, 0x5140u);
-      X = ((z << 4) & 0xF0F0F0F0u) ^ 0x80808080u;     // 16 (u - 8): low nibbles moved up
-      Y = (z & 0xF0F0F0F0u) ^ 0x80808080u;            // 16 (u - 8): high nibbles
+      X = ((z << 4) & kM) ^ kC;                       // 16 (u - 8): low nibbles moved up
+      Y = (z & kM) ^ kC;                              // 16 (u - 8): high nibbles
     } else {
       const uint32_t a = vp[j * cbV + lane];
       const uint32_t b = vp[(j + 32) * cbV + lane];
@@ -498,8 +504,8 @@ __device__ __forceinline__ void slot_channel(int k, int& ch, float& inv_factor) 
 // the warp's table ([4 blocks][G] words of (W_j, W_j+32)) and sigma_g is returned.
 // nb: blocks per row (absent blocks get weight 0).  For the _1 codecs
 // off[g][b] += p * (m + fcoef * d) per own token.
-template <int G>
-__device__ __forceinline__ void tile_weights(int nb, bool vasym, float fcoef, const uint8_t* vs, int sbV, int nvalid,
+template <int G, bool vasym>
+__device__ __forceinline__ void tile_weights(int nb, float fcoef, const uint8_t* vs, int sbV, int nvalid,
                                              int lane, uint32_t* wq, const float p0[G], const float p1[G],
                                              const float pm[G], float sg[G], float off[G][4]) {
   constexpr int WRS = wq_row_words<G>();
@@ -509,7 +515,7 @@ __device__ __forceinline__ void tile_weights(int nb, bool vasym, float fcoef, co
   for (int b = 0; b < 4; ++b) {
     d0[b] = 0.f; d1[b] = 0.f; f0[b] = 0.f; f1[b] = 0.f;
     if (b < nb && lane < nvalid) {
-      if (vasym) {
+      if constexpr (vasym) {
         const __half2 x = *reinterpret_cast<const __half2*>(vs + lane * sbV + 4 * b);
         d0[b] = __low2float(x); f0[b] = fmaf(fcoef, d0[b], __high2float(x));
       } else {
@@ -517,7 +523,7 @@ __device__ __forceinline__ void tile_weights(int nb, bool vasym, float fcoef, co
       }
     }
     if (b < nb && lane + 32 < nvalid) {
-      if (vasym) {
+      if constexpr (vasym) {
         const __half2 x = *reinterpret_cast<const __half2*>(vs + (lane + 32) * sbV + 4 * b);
         d1[b] = __low2float(x); f1[b] = fmaf(fcoef, d1[b], __high2float(x));
       } else {
@@ -539,7 +545,7 @@ __device__ __forceinline__ void tile_weights(int nb, bool vasym, float fcoef, co
     for (int b = 0; b < 4; ++b) {
       const float w0 = fmaf(q0, d0[b], RINT_MAGIC), w1 = fmaf(q1, d1[b], RINT_MAGIC);
       wv[b][g] = prmt(__float_as_uint(w0), __float_as_uint(w1), 0x5410u);
-      if (vasym) off[g][b] = fmaf(p0[g], f0[b], fmaf(p1[g], f1[b], off[g][b]));
+      if constexpr (vasym) off[g][b] = fmaf(p0[g], f0[b], fmaf(p1[g], f1[b], off[g][b]));
     }
   }
   uint32_t* row = wq + lane * WRS;
@@ -565,19 +571,19 @@ __device__ __forceinline__ void tile_weights(int nb, bool vasym, float fcoef, co
 // (lane, lane + 32); pm: the tile's largest numerator per head.  O2: packed fp32
 // accumulators of the lane's channels (already rescaled for this tile); off:
 // per-block offsets of the _1 codecs.
-template <int G, int VB>
-__device__ __forceinline__ void value_tile_int(bool vasym, float vhalf, const uint8_t* vp, const uint8_t* vs, int cbV,
-                                               int sbV, int nvalid, int lane, int blane, uint32_t* wq,
+template <int G, int VB, bool VASYM>
+__device__ __forceinline__ void value_tile_int(float vhalf, const uint8_t* vp, const uint8_t* vs, int sbV, int nvalid,
+                                               int lane, int blane, uint32_t* wq, uint32_t kM, uint32_t kC,
                                                const float p0[G], const float p1[G], const float pm[G],
                                                uint64_t O2[G][2], float off[G][4]) {
   float sg[G];
-  tile_weights<G>(4, vasym, vhalf, vs, sbV, nvalid, lane, wq, p0, p1, pm, sg, off);
+  tile_weights<G, VASYM>(4, vhalf, vs, sbV, nvalid, lane, wq, p0, p1, pm, sg, off);
   int acc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[g][k] = 0;
-  value_dots<G, VB>(vp, cbV, lane, wq + blane * G, acc);
+  value_dots<G, VB>(vp, lane, wq + blane * G, kM, kC, acc);
   __syncwarp();
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -639,14 +645,14 @@ __device__ __forceinline__ void plane_slot(int k, int& ch, double& inv_f) {
 // and 32/cl pairs side by side, summed over the lane groups at the end of the tile;
 // lane cg < cl then holds channels 4cg .. 4cg+3 (the other lanes hold copies for
 // channels that do not exist).
-template <int G, int LO, int HI>
-__device__ __forceinline__ void value_tile_planes(int nb, int blk, int cl, bool vasym, float cen, int offB,
+template <int G, int LO, int HI, bool VASYM>
+__device__ __forceinline__ void value_tile_planes(int nb, int blk, int cl, float cen, int offB,
                                                   const uint8_t* vp, const uint8_t* vs, int cbV, int sbV, int nvalid,
                                                   int lane, uint32_t* wq, const float p0[G], const float p1[G],
                                                   const float pm[G], uint64_t O2[G][2], float off[G][4]) {
   constexpr int WRS = wq_row_words<G>();
   float sg[G];
-  tile_weights<G>(nb, vasym, cen, vs, sbV, nvalid, lane, wq, p0, p1, pm, sg, off);
+  tile_weights<G, VASYM>(nb, cen, vs, sbV, nvalid, lane, wq, p0, p1, pm, sg, off);
   const int grp = lane / cl, cg = lane - grp * cl, ngrp = 32 / cl;
   const int blane = ((4 * cg) / blk) & 3;
   int accA[G][4], accB[G][4], sw[G];
