@@ -474,6 +474,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     if (vblock) vclass = (vbits == 8 || vbits == 4 || vbits == 2) ? vbits : (vbits == 6) ? 42 : (vbits == 5) ? 41 : 21;
     else if (vc == KVQ_RANK) vclass = (vbits == 4) ? 40 : (vbits == 3) ? 21 : (vbits == 2) ? 20 : 10;
     const bool vasym = codec_is_asym(vc);
+    const bool kasym = codec_is_asym(kc);
     const float vhalf = vblock ? (float)(1 << (vbits - 1)) : 0.f;
     // the codes' centre on the plane path, the byte offset of the high plane, the
     // blocks per row and the lanes per token pair
@@ -509,9 +510,11 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
       const int nvalid = min(rows, seg_tokens - tok0);
       float s0[G], s1[G];
       switch (kclass) {
-        case 8: score2_block_codec<G, 8>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
-        case 4: score2_block_codec<G, 4>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
-        case 2: score2_block_codec<G, 2>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
+#define KVQ_SCORE(KCL, ASYM) score2_block_codec<G, KCL, ASYM>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1)
+        case 8: if (kasym) KVQ_SCORE(8, true); else KVQ_SCORE(8, false); break;
+        case 4: if (kasym) KVQ_SCORE(4, true); else KVQ_SCORE(4, false); break;
+        case 2: if (kasym) KVQ_SCORE(2, true); else KVQ_SCORE(2, false); break;
+#undef KVQ_SCORE
         case 11: score2_rank<G, 1>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         case 12: score2_rank<G, 2>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         case 13: score2_rank<G, 3>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
@@ -603,10 +606,12 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     for (int g = 0; g < G; ++g) {
       l[g] = warp_sum(l[g]);
       float ob = 0.f;                     // the lane's block's offset sum, no dynamic register index
+      if (vasym) {                        // only the _1 codecs accumulate offsets
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const float sb = warp_sum(off[g][b]);
-        ob = (b == blane) ? sb : ob;
+        for (int b = 0; b < 4; ++b) {
+          const float sb = warp_sum(off[g][b]);
+          ob = (b == blane) ? sb : ob;
+        }
       }
       float a[4];
       unpack2(O2[g][0], a[0], a[1]);

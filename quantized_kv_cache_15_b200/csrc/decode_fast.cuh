@@ -118,12 +118,12 @@ __device__ __forceinline__ void tab_channels(int type, int w, int& c0, int& c1) 
 
 // Block epilogue of the integer score: s += (A - half*qsum) * d   (_0)
 //                                     s += A * d + qsum * m       (_1)
-template <int G>
-__device__ __forceinline__ void score_block_epilogue(const uint8_t* ks, int sb, bool asym, int half, int b, int t0,
+template <int G, bool asym>
+__device__ __forceinline__ void score_block_epilogue(const uint8_t* ks, int sb, int half, int b, int t0,
                                                      const int* qsi, const int a0[G], const int a1[G], float s0[G],
                                                      float s1[G]) {
   float d0, m0 = 0.f, d1, m1 = 0.f;
-  if (asym) {
+  if constexpr (asym) {
     const __half2 x0 = *reinterpret_cast<const __half2*>(ks + t0 * sb + 4 * b);
     const __half2 x1 = *reinterpret_cast<const __half2*>(ks + (t0 + 32) * sb + 4 * b);
     d0 = __low2float(x0); m0 = __high2float(x0);
@@ -135,7 +135,7 @@ __device__ __forceinline__ void score_block_epilogue(const uint8_t* ks, int sb, 
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const int qs = qsi[g * 4 + b];
-    if (asym) {
+    if constexpr (asym) {
       s0[g] = fmaf((float)a0[g], d0, fmaf((float)qs, m0, s0[g]));
       s1[g] = fmaf((float)a1[g], d1, fmaf((float)qs, m1, s1[g]));
     } else {
@@ -150,13 +150,12 @@ __device__ __forceinline__ void score_block_epilogue(const uint8_t* ks, int sb, 
 // KCLASS selects the code planes compiled in: 8 (q8), 4 (a nibble plane, plus a
 // 2-bit or 1-bit high plane for 6 / 5 bits), 2 (a 2-bit plane, plus a 1-bit high
 // plane for 3 bits).
-template <int G, int KCLASS>
+template <int G, int KCLASS, bool KASYM>
 __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, const uint8_t* ks, int sb, int t0,
                                                    const uint32_t* tab0, const uint32_t* tab1, const int* qsi,
                                                    float s0[G], float s1[G]) {
 #pragma unroll
   for (int g = 0; g < G; ++g) { s0[g] = 0.f; s1[g] = 0.f; }
-  const bool asym = codec_is_asym(kc);
   const int bits = codec_bits(kc);
   const int half = 1 << (bits - 1);
 #pragma unroll 1
@@ -279,7 +278,7 @@ __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, co
         for (int g = 0; g < G; ++g) { a0[g] += 4 * e0[g]; a1[g] += 4 * e1[g]; }
       }
     }
-    score_block_epilogue<G>(ks, sb, asym, half, b, t0, qsi, a0, a1, s0, s1);
+    score_block_epilogue<G, KASYM>(ks, sb, half, b, t0, qsi, a0, a1, s0, s1);
   }
 }
 
