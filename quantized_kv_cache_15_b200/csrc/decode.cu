@@ -46,10 +46,13 @@ __host__ __device__ inline int basis_of(int codec, int rot) {
   return BASIS_ROT;
 }
 
+// Warp-wide maximum of a float in one integer reduction: the map x -> key (the
+// bits, with the magnitude bits flipped for negative x) is monotone from floats to
+// int32, so the max of the keys is the key of the max (exact; no NaNs here).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
-  return v;
+  const int i = __float_as_int(v);
+  const int m = __reduce_max_sync(0xffffffffu, i >= 0 ? i : (i ^ 0x7FFFFFFF));
+  return __int_as_float(m >= 0 ? m : (m ^ 0x7FFFFFFF));
 }
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -542,8 +545,10 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
         const uint64_t a2 = pack2(alpha, alpha);
         O2[g][0] = mul2(O2[g][0], a2);
         O2[g][1] = mul2(O2[g][1], a2);
+        if (vasym) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) off[g][b] *= alpha;
+          for (int b = 0; b < 4; ++b) off[g][b] *= alpha;
+        }
         m[g] = mnew;
       }
       __syncwarp();                         // every lane's key reads are done: the K region may be reused

@@ -531,8 +531,8 @@ __device__ __forceinline__ void tile_weights(int nb, float fcoef, const uint8_t*
     }
     dm = fmaxf(dm, fmaxf(d0[b], d1[b]));
   }
-#pragma unroll
-  for (int m = 16; m > 0; m >>= 1) dm = fmaxf(dm, __shfl_xor_sync(0xffffffffu, dm, m));
+  // dm >= 0: its bits order like the values, so one unsigned reduction gives the max
+  dm = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(dm)));
   uint32_t wv[4][G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
