@@ -99,6 +99,15 @@ typedef enum {
   KVQ_ROT_NONE = 0, KVQ_ROT_HADAMARD = 1, KVQ_ROT_VARNORM_HADAMARD = 2, KVQ_ROT_PROJECTION = 3
 } kvq_rot;
 
+/* Dtype of the plan's raw 16-bit rows: the appended K/V rows (k_new, v_new), the
+ * decode queries q, the precision tail and the pages of the KVQ_F16 codec
+ * [BeeLlama v0.4.0 news, §KV cache 精度尾部: the newest tokens are kept in BF16 or
+ * F16].  KVQ_KV_BF16 plans take bf16 rows throughout (exactly widened to fp32 before
+ * the transform and the quantizer) and keep a bf16 tail; they support neither
+ * KVQ_ROT_PROJECTION nor KVQ_F16 pages (KVQ_ERR_UNSUPPORTED at plan creation or
+ * regrade).  kvq_calibrate_varnorm always reads fp16 rows. */
+typedef enum { KVQ_KV_F16 = 0, KVQ_KV_BF16 = 1 } kvq_kv_dtype;
+
 typedef struct kvq_plan kvq_plan;
 
 typedef struct {
@@ -121,6 +130,7 @@ typedef struct {
   const double* proj_basis;     /* host, PROJECTION only: for each (layer, head) in order, P_h as a
                                    row-major [128][r] matrix with orthonormal columns; concatenated */
   float softmax_scale;          /* 0 => 1/sqrt(128) */
+  int kv_dtype;                 /* kvq_kv_dtype of the raw 16-bit rows; 0 = KVQ_KV_F16 */
 } kvq_plan_desc;
 
 /* Create a plan on the current CUDA device: validates the descriptor, lays out
@@ -144,8 +154,8 @@ kvq_status kvq_cache_bind(kvq_plan* plan, void* dev_cache, size_t bytes);
 
 /* Append n_new[i] new tokens to sequence seq_ids[i] in one layer
  * [BeeLlama v0.4.0 news §KV cache 精度尾部 and §KVarN; KV-COBRA §The news].
- *  k_new, v_new: device fp16 [sum(n_new)][n_kv_heads][128], the sequences'
- *  rows concatenated in call order.
+ *  k_new, v_new: device fp16 (bf16 for KVQ_KV_BF16 plans)
+ *  [sum(n_new)][n_kv_heads][128], the sequences' rows concatenated in call order.
  * New rows enter the layer's F16 tail; rows pushed out of the tail (or every
  * row, when tail_tokens = 0) are transformed and quantized into the paged
  * cache.  seq_ids must be distinct.  Lengths advance at enqueue time (per
@@ -156,7 +166,7 @@ kvq_status kvq_append_quantize(kvq_plan* plan, int layer, int n_seqs, const int*
 
 /* Decode attention for one new query token per sequence
  * [forum thread on KV compression: dot, softmax, weighted average of values].
- *  q:   device fp16 [n_seqs][n_q_heads][128]
+ *  q:   device fp16 (bf16 for KVQ_KV_BF16 plans) [n_seqs][n_q_heads][128]
  *  out: device fp32 [n_seqs][n_q_heads][128]
  *  workspace: device, kvq_plan_workspace_bytes(plan, n_seqs), zeroed before first use;
  *    may be NULL when no sequence needs more than one split and the plan has no
@@ -299,7 +309,7 @@ enum kvq_row_layout { KVQ_ROWS_WARP = 0, KVQ_ROWS_QUAD = 1 };
  * before quantization: the staged Hadamard transform (after variance
  * normalisation) for rotated codecs, z = M_h x on the tensor cores for the
  * projection path, the raw values for F16.
- *  x: device fp16 [n][128];  y: device fp32 [n][128] (or [n][r]).
+ *  x: device raw rows in the plan's kv dtype [n][128];  y: device fp32 [n][128] (or [n][r]).
  *  layout: kvq_row_layout (ignored for the projection path). */
 kvq_status kvq_debug_rotate(const kvq_plan* plan, int layer, int head, int kv, int n, const void* x,
                             float* y, int layout, void* stream);

@@ -67,6 +67,8 @@ def _declare(L):
     L.orc_f16_rd.argtypes = [ctypes.c_float]
     L.orc_f16_to_f32.restype = ctypes.c_float
     L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+    L.orc_bf16_to_f32.restype = ctypes.c_float
+    L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
     for name in ("orc_f16_rn_array", "orc_f16_rd_array"):
         getattr(L, name).argtypes = [_P, _P, _I64]
     L.orc_f16_to_f32_array.argtypes = [_P, _P, _I64]
@@ -81,13 +83,14 @@ def _declare(L):
     L.orc_dequantize_rows.argtypes = [_I, _I, _I, _I64, _P, _P, _P]
     L.orc_varnorm_inv_rms.argtypes = [_I64, _I, _I64, _P, _P]
     L.orc_fuse_projection.argtypes = [_I, _P, _P]
-    L.orc_to_stored_basis.argtypes = [_I, _I, _I, _P, _P, _I64, _P, _P]
-    L.orc_encode_rows.argtypes = [_I, _I, _I, _I, _P, _P, _I64, _P, _P, _P]
+    L.orc_to_stored_basis_dt.argtypes = [_I, _I, _I, _I, _P, _P, _I64, _P, _P]
+    L.orc_encode_rows_dt.argtypes = [_I, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P]
     L.orc_decode_rows_original.argtypes = [_I, _I, _I, _I, _P, _P, _I64, _P, _P, _P]
     L.orc_attention.argtypes = [_I64, _P, _P, _P, ctypes.c_double, _P]
-    L.orc_decode_head.argtypes = [_I64, _I, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, ctypes.c_float, _P]
-    L.orc_decode_packed.argtypes = [_I64, _P, _P, _P, _P, _I64, _P, _P, _I, _P,
-                                    _I, _I, _I, _I, _I, _I, _P, _P, _P, ctypes.c_float, _P]
+    L.orc_decode_head_dt.argtypes = [_I, _I64, _I, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P,
+                                     ctypes.c_float, _P]
+    L.orc_decode_packed_dt.argtypes = [_I, _I64, _P, _P, _P, _P, _I64, _P, _P, _I, _P,
+                                       _I, _I, _I, _I, _I, _I, _P, _P, _P, ctypes.c_float, _P]
     L.orc_cobra_error.restype = ctypes.c_double
     L.orc_cobra_error.argtypes = [_P, _I, _I, _P]
     L.orc_cobra_best.argtypes = [_P, _I, _P, ctypes.POINTER(_I), ctypes.POINTER(_I)]
@@ -125,6 +128,12 @@ def f16_to_f32(h):
 
 
 # ----------------------------------------------------------------------------- rotation
+def bf16_to_f32(h):
+    """uint16 bf16 bit patterns -> float32 (exact widening), element by element."""
+    h = np.asarray(h, np.uint16)
+    return np.array([lib().orc_bf16_to_f32(int(x)) for x in h.reshape(-1)], np.float32).reshape(h.shape)
+
+
 def hadamard_matrix(n=D):
     H = np.empty((n, n), np.int8)
     lib().orc_hadamard_matrix(n, _ptr(H))
@@ -214,24 +223,27 @@ def fuse_projection(P):
 
 
 # ----------------------------------------------------------------------------- encode / decode
-def to_stored_basis(codec, rot, x_f16, inv_s=None, M=None, r=D):
+def to_stored_basis(codec, rot, x_f16, inv_s=None, M=None, r=D, bf16=False):
+    """x_f16: uint16 raw rows [n][128] (fp16 bits, or bf16 bits when bf16)."""
     x = _c(x_f16, np.uint16).reshape(-1, D)
     n_out = r if codec == RANK else D
     y = np.empty((x.shape[0], n_out), np.float32)
     inv_s = None if inv_s is None else _c(inv_s, np.float32)
     M = None if M is None else _c(M, np.float32)
-    lib().orc_to_stored_basis(codec, rot, r, _ptr(inv_s), _ptr(M), x.shape[0], _ptr(x), _ptr(y))
+    lib().orc_to_stored_basis_dt(int(bf16), codec, rot, r, _ptr(inv_s), _ptr(M), x.shape[0], _ptr(x), _ptr(y))
     return y
 
 
-def encode_rows(codec, rot, x_f16, inv_s=None, M=None, r=D, b=0):
+def encode_rows(codec, rot, x_f16, inv_s=None, M=None, r=D, b=0, bf16=False):
+    """x_f16: uint16 raw rows [n][128] (fp16 bits, or bf16 bits when bf16)."""
     x = _c(x_f16, np.uint16).reshape(-1, D)
     cb, sb = row_bytes(codec, r, b)
     codes = np.zeros((x.shape[0], cb), np.uint8)
     scales = np.zeros((x.shape[0], max(sb // 2, 1)), np.uint16)
     inv_s = None if inv_s is None else _c(inv_s, np.float32)
     M = None if M is None else _c(M, np.float32)
-    lib().orc_encode_rows(codec, rot, r, b, _ptr(inv_s), _ptr(M), x.shape[0], _ptr(x), _ptr(codes), _ptr(scales))
+    lib().orc_encode_rows_dt(int(bf16), codec, rot, r, b, _ptr(inv_s), _ptr(M), x.shape[0], _ptr(x), _ptr(codes),
+                             _ptr(scales))
     return codes, scales[:, : sb // 2]
 
 
@@ -272,9 +284,10 @@ def attention(q, K, V, scale):
 
 
 def decode_head(K_f16, V_f16, q_f16, k_codec, v_codec, rot, tail=0, r=D, kb=0, vb=0,
-                inv_s_k=None, inv_s_v=None, M=None, scale=None):
+                inv_s_k=None, inv_s_v=None, M=None, scale=None, bf16=False):
     """Decode attention for one (seq, layer, kv-head).  K_f16/V_f16: uint16 [len][128]
-    history; q_f16: uint16 [G][128].  Returns float32 [G][128]."""
+    history; q_f16: uint16 [G][128] (fp16 bits, or bf16 bits when bf16).  Returns
+    float32 [G][128]."""
     K = _c(K_f16, np.uint16).reshape(-1, D)
     V = _c(V_f16, np.uint16).reshape(-1, D)
     q = _c(q_f16, np.uint16).reshape(-1, D)
@@ -285,13 +298,13 @@ def decode_head(K_f16, V_f16, q_f16, k_codec, v_codec, rot, tail=0, r=D, kb=0, v
     inv_s_k = None if inv_s_k is None else _c(inv_s_k, np.float32)
     inv_s_v = None if inv_s_v is None else _c(inv_s_v, np.float32)
     M = None if M is None else _c(M, np.float32)
-    lib().orc_decode_head(K.shape[0], int(tail), G, _ptr(K), _ptr(V), _ptr(q), k_codec, v_codec, rot, r, kb, vb,
-                          _ptr(inv_s_k), _ptr(inv_s_v), _ptr(M), float(scale), _ptr(out))
+    lib().orc_decode_head_dt(int(bf16), K.shape[0], int(tail), G, _ptr(K), _ptr(V), _ptr(q), k_codec, v_codec, rot,
+                             r, kb, vb, _ptr(inv_s_k), _ptr(inv_s_v), _ptr(M), float(scale), _ptr(out))
     return out
 
 
 def decode_packed(ck, sk, cv, sv, Kt, Vt, q_f16, k_codec, v_codec, rot, r=D, kb=0, vb=0,
-                  inv_s_k=None, inv_s_v=None, M=None, scale=None):
+                  inv_s_k=None, inv_s_v=None, M=None, scale=None, bf16=False):
     """Decode attention from the oracle's own packed rows plus raw tail rows."""
     q = _c(q_f16, np.uint16).reshape(-1, D)
     G = q.shape[0]
@@ -305,8 +318,9 @@ def decode_packed(ck, sk, cv, sv, Kt, Vt, q_f16, k_codec, v_codec, rot, r=D, kb=
     inv_s_k = None if inv_s_k is None else _c(inv_s_k, np.float32)
     inv_s_v = None if inv_s_v is None else _c(inv_s_v, np.float32)
     M = None if M is None else _c(M, np.float32)
-    lib().orc_decode_packed(nq, *[_ptr(a) for a in args], Kt.shape[0], _ptr(Kt), _ptr(Vt), G, _ptr(q),
-                            k_codec, v_codec, rot, r, kb, vb, _ptr(inv_s_k), _ptr(inv_s_v), _ptr(M), float(scale), _ptr(out))
+    lib().orc_decode_packed_dt(int(bf16), nq, *[_ptr(a) for a in args], Kt.shape[0], _ptr(Kt), _ptr(Vt), G, _ptr(q),
+                               k_codec, v_codec, rot, r, kb, vb, _ptr(inv_s_k), _ptr(inv_s_v), _ptr(M), float(scale),
+                               _ptr(out))
     return out
 
 

@@ -106,6 +106,18 @@ float orc_f16_to_f32(uint16_t h) {
     return sign ? -mag : mag;
 }
 
+/* bf16 -> fp32: a bf16 value is the upper half of a binary32 (sign, 8-bit
+ * exponent, 7 fraction bits), so widening appends 16 zero bits.  Exact. */
+float orc_bf16_to_f32(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* A raw 16-bit row element (the plan's kv dtype: bf16 if nonzero, else fp16). */
+static float raw_to_f32(uint16_t h, int bf16) { return bf16 ? orc_bf16_to_f32(h) : orc_f16_to_f32(h); }
+
 void orc_f16_rn_array(const float* x, uint16_t* h, int64_t n) { for (int64_t i = 0; i < n; ++i) h[i] = orc_f16_rn(x[i]); }
 void orc_f16_rd_array(const float* x, uint16_t* h, int64_t n) { for (int64_t i = 0; i < n; ++i) h[i] = orc_f16_rd(x[i]); }
 void orc_f16_to_f32_array(const uint16_t* h, float* x, int64_t n) { for (int64_t i = 0; i < n; ++i) x[i] = orc_f16_to_f32(h[i]); }
@@ -471,12 +483,12 @@ enum { ROT_NONE = 0, ROT_HADAMARD = 1, ROT_VARNORM_HADAMARD = 2, ROT_PROJECTION 
  *  Hadamard:  spec FWHT of x;  varnorm: spec FWHT of (x * inv_s) (one fp32
  *  multiply per element, R10);
  *  projection: z = M x accumulated in double, rounded to fp32 (R12). */
-void orc_to_stored_basis(int codec, int rot, int r, const float* inv_s, const float* M,
-                         int64_t n_rows, const uint16_t* x, float* y) {
+void orc_to_stored_basis_dt(int bf16, int codec, int rot, int r, const float* inv_s, const float* M,
+                            int64_t n_rows, const uint16_t* x, float* y) {
     const int n_out = (codec == C_RANK) ? r : D;
     for (int64_t row = 0; row < n_rows; ++row) {
         float v[D];
-        for (int j = 0; j < D; ++j) v[j] = orc_f16_to_f32(x[row * D + j]);
+        for (int j = 0; j < D; ++j) v[j] = raw_to_f32(x[row * D + j], bf16);
         float* out = y + row * n_out;
         if (codec == C_F16 || rot == ROT_NONE) { memcpy(out, v, sizeof(float) * D); continue; }
         if (codec == C_RANK) {
@@ -493,14 +505,25 @@ void orc_to_stored_basis(int codec, int rot, int r, const float* inv_s, const fl
     }
 }
 
-/* Full encode of fp16 rows into canonical packed rows. */
-void orc_encode_rows(int codec, int rot, int r, int b, const float* inv_s, const float* M,
-                     int64_t n_rows, const uint16_t* x, uint8_t* codes, uint16_t* scales) {
+void orc_to_stored_basis(int codec, int rot, int r, const float* inv_s, const float* M,
+                         int64_t n_rows, const uint16_t* x, float* y) {
+    orc_to_stored_basis_dt(0, codec, rot, r, inv_s, M, n_rows, x, y);
+}
+
+/* Full encode of raw 16-bit rows (fp16, or bf16 if bf16 != 0) into canonical
+ * packed rows. */
+void orc_encode_rows_dt(int bf16, int codec, int rot, int r, int b, const float* inv_s, const float* M,
+                        int64_t n_rows, const uint16_t* x, uint8_t* codes, uint16_t* scales) {
     const int n_out = (codec == C_RANK) ? r : D;
     float* y = (float*)malloc(sizeof(float) * (size_t)(n_rows * n_out));
-    orc_to_stored_basis(codec, rot, r, inv_s, M, n_rows, x, y);
+    orc_to_stored_basis_dt(bf16, codec, rot, r, inv_s, M, n_rows, x, y);
     orc_quantize_rows(codec, r, b, n_rows, y, codes, scales);
     free(y);
+}
+
+void orc_encode_rows(int codec, int rot, int r, int b, const float* inv_s, const float* M,
+                     int64_t n_rows, const uint16_t* x, uint8_t* codes, uint16_t* scales) {
+    orc_encode_rows_dt(0, codec, rot, r, b, inv_s, M, n_rows, x, codes, scales);
 }
 
 /* Dequantize canonical rows and return them in the ORIGINAL basis, double:
@@ -566,9 +589,9 @@ void orc_attention(int64_t n, const double* q, const double* K, const double* V,
  * row is a tail row and the path is exactly the plain F16 attention below.
  * out: fp32 [G][128].  k_codec/v_codec: codec ids; kb/vb: bits for the rank
  * codec; r: rank. */
-void orc_decode_head(int64_t len, int T, int G, const uint16_t* Kx, const uint16_t* Vx, const uint16_t* q,
-                     int k_codec, int v_codec, int rot, int r, int kb, int vb,
-                     const float* inv_s_k, const float* inv_s_v, const float* M, float scale, float* out) {
+void orc_decode_head_dt(int bf16, int64_t len, int T, int G, const uint16_t* Kx, const uint16_t* Vx,
+                        const uint16_t* q, int k_codec, int v_codec, int rot, int r, int kb, int vb,
+                        const float* inv_s_k, const float* inv_s_v, const float* M, float scale, float* out) {
     int64_t nq = len > T ? len - T : 0;
     double* Kd = (double*)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * D));
     double* Vd = (double*)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * D));
@@ -580,32 +603,38 @@ void orc_decode_head(int64_t len, int T, int G, const uint16_t* Kx, const uint16
         uint16_t* sk = (uint16_t*)malloc((size_t)(nq * (sbk > 0 ? sbk : 2)));
         uint8_t* cv = (uint8_t*)malloc((size_t)(nq * cbv));
         uint16_t* sv = (uint16_t*)malloc((size_t)(nq * (sbv > 0 ? sbv : 2)));
-        orc_encode_rows(k_codec, rot, r, kb, inv_s_k, M, nq, Kx, ck, sk);
-        orc_encode_rows(v_codec, rot, r, vb, inv_s_v, M, nq, Vx, cv, sv);
+        orc_encode_rows_dt(bf16, k_codec, rot, r, kb, inv_s_k, M, nq, Kx, ck, sk);
+        orc_encode_rows_dt(bf16, v_codec, rot, r, vb, inv_s_v, M, nq, Vx, cv, sv);
         orc_decode_rows_original(k_codec, rot, r, kb, inv_s_k, M, nq, ck, sk, Kd);
         orc_decode_rows_original(v_codec, rot, r, vb, inv_s_v, M, nq, cv, sv, Vd);
         free(ck); free(sk); free(cv); free(sv);
     }
     for (int64_t i = nq; i < len; ++i)
         for (int j = 0; j < D; ++j) {
-            Kd[i * D + j] = (double)orc_f16_to_f32(Kx[i * D + j]);
-            Vd[i * D + j] = (double)orc_f16_to_f32(Vx[i * D + j]);
+            Kd[i * D + j] = (double)raw_to_f32(Kx[i * D + j], bf16);
+            Vd[i * D + j] = (double)raw_to_f32(Vx[i * D + j], bf16);
         }
     for (int g = 0; g < G; ++g) {
         double qd[D], o[D];
-        for (int j = 0; j < D; ++j) qd[j] = (double)orc_f16_to_f32(q[g * D + j]);
+        for (int j = 0; j < D; ++j) qd[j] = (double)raw_to_f32(q[g * D + j], bf16);
         orc_attention(len, qd, Kd, Vd, (double)scale, o);
         for (int j = 0; j < D; ++j) out[g * D + j] = (float)o[j];
     }
     free(Kd); free(Vd);
 }
 
+void orc_decode_head(int64_t len, int T, int G, const uint16_t* Kx, const uint16_t* Vx, const uint16_t* q,
+                     int k_codec, int v_codec, int rot, int r, int kb, int vb,
+                     const float* inv_s_k, const float* inv_s_v, const float* M, float scale, float* out) {
+    orc_decode_head_dt(0, len, T, G, Kx, Vx, q, k_codec, v_codec, rot, r, kb, vb, inv_s_k, inv_s_v, M, scale, out);
+}
+
 /* Decode attention from already packed canonical rows (the oracle's own), for
  * timing the decode step alone: nq quantized rows + nt raw fp16 tail rows. */
-void orc_decode_packed(int64_t nq, const uint8_t* ck, const uint16_t* sk, const uint8_t* cv, const uint16_t* sv,
-                       int64_t nt, const uint16_t* Kt, const uint16_t* Vt, int G, const uint16_t* q,
-                       int k_codec, int v_codec, int rot, int r, int kb, int vb,
-                       const float* inv_s_k, const float* inv_s_v, const float* M, float scale, float* out) {
+void orc_decode_packed_dt(int bf16, int64_t nq, const uint8_t* ck, const uint16_t* sk, const uint8_t* cv,
+                          const uint16_t* sv, int64_t nt, const uint16_t* Kt, const uint16_t* Vt, int G,
+                          const uint16_t* q, int k_codec, int v_codec, int rot, int r, int kb, int vb,
+                          const float* inv_s_k, const float* inv_s_v, const float* M, float scale, float* out) {
     int64_t len = nq + nt;
     double* Kd = (double*)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * D));
     double* Vd = (double*)malloc(sizeof(double) * (size_t)((len > 0 ? len : 1) * D));
@@ -615,16 +644,24 @@ void orc_decode_packed(int64_t nq, const uint8_t* ck, const uint16_t* sk, const 
     }
     for (int64_t i = 0; i < nt; ++i)
         for (int j = 0; j < D; ++j) {
-            Kd[(nq + i) * D + j] = (double)orc_f16_to_f32(Kt[i * D + j]);
-            Vd[(nq + i) * D + j] = (double)orc_f16_to_f32(Vt[i * D + j]);
+            Kd[(nq + i) * D + j] = (double)raw_to_f32(Kt[i * D + j], bf16);
+            Vd[(nq + i) * D + j] = (double)raw_to_f32(Vt[i * D + j], bf16);
         }
     for (int g = 0; g < G; ++g) {
         double qd[D], o[D];
-        for (int j = 0; j < D; ++j) qd[j] = (double)orc_f16_to_f32(q[g * D + j]);
+        for (int j = 0; j < D; ++j) qd[j] = (double)raw_to_f32(q[g * D + j], bf16);
         orc_attention(len, qd, Kd, Vd, (double)scale, o);
         for (int j = 0; j < D; ++j) out[g * D + j] = (float)o[j];
     }
     free(Kd); free(Vd);
+}
+
+void orc_decode_packed(int64_t nq, const uint8_t* ck, const uint16_t* sk, const uint8_t* cv, const uint16_t* sv,
+                       int64_t nt, const uint16_t* Kt, const uint16_t* Vt, int G, const uint16_t* q,
+                       int k_codec, int v_codec, int rot, int r, int kb, int vb,
+                       const float* inv_s_k, const float* inv_s_v, const float* M, float scale, float* out) {
+    orc_decode_packed_dt(0, nq, ck, sk, cv, sv, nt, Kt, Vt, G, q, k_codec, v_codec, rot, r, kb, vb, inv_s_k, inv_s_v,
+                         M, scale, out);
 }
 
 /* ------------------------------------------------------------------------- */

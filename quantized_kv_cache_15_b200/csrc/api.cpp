@@ -63,6 +63,7 @@ struct kvq_plan {
   int mpps = 0;            // max pages per sequence
   int64_t n_pages = 0;
   int rot = 0;
+  bool bf16 = false;             // raw rows are bf16
   float scale = 0.f;
   std::vector<HeadInfo> heads;        // [L][Hkv]
   std::vector<uint64_t> layer_off;    // [L]
@@ -110,6 +111,7 @@ struct kvq_plan {
     p.tail = cache + tail_off;
     p.T = T; p.L = L; p.layer = layer; p.Hkv = Hkv; p.Hq = Hq; p.G = G;
     p.rot = rot;
+    p.bf16 = bf16;
     p.s_k = (rot == KVQ_ROT_VARNORM_HADAMARD) ? d_sk + (size_t)layer * Hkv * D : nullptr;
     p.s_v = (rot == KVQ_ROT_VARNORM_HADAMARD) ? d_sv + (size_t)layer * Hkv * D : nullptr;
     p.M = d_M;
@@ -147,6 +149,9 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
   if (d->rot == KVQ_ROT_VARNORM_HADAMARD && !d->inv_rms) return fail(KVQ_ERR_INVALID_ARG, "VARNORM_HADAMARD needs inv_rms");
   if (d->rot == KVQ_ROT_PROJECTION && (!d->rank || !d->k_bits || !d->v_bits || !d->proj_basis))
     return fail(KVQ_ERR_INVALID_ARG, "PROJECTION needs rank, k_bits, v_bits and proj_basis");
+  if (d->kv_dtype != KVQ_KV_F16 && d->kv_dtype != KVQ_KV_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad kv_dtype %d", d->kv_dtype);
+  if (d->kv_dtype == KVQ_KV_BF16 && d->rot == KVQ_ROT_PROJECTION)
+    return fail(KVQ_ERR_UNSUPPORTED, "bf16 rows are not supported with the projection path");
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -159,6 +164,7 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
   p->mpps = (int)((p->max_tokens + PAGE - 1) / PAGE);
   p->n_pages = d->max_pages > 0 ? d->max_pages : (int64_t)p->max_seqs * p->mpps;
   p->rot = d->rot;
+  p->bf16 = d->kv_dtype == KVQ_KV_BF16;
   p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / std::sqrt((double)D));
 
   // per-head codec info and page layout
@@ -179,6 +185,10 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
       std::memset(&hi, 0, sizeof(hi));
       const int kc = d->k_codec[i], vc = d->v_codec[i];
       if (!valid_codec(kc) || !valid_codec(vc)) { delete p; return fail(KVQ_ERR_UNSUPPORTED, "bad codec at layer %d head %d", l, h); }
+      if (p->bf16 && (kc == KVQ_F16 || vc == KVQ_F16)) {
+        delete p;
+        return fail(KVQ_ERR_UNSUPPORTED, "bf16 plans keep raw rows in the tail only: no KVQ_F16 pages (layer %d head %d)", l, h);
+      }
       const bool rank = (kc == KVQ_RANK || vc == KVQ_RANK);
       if (rank != (d->rot == KVQ_ROT_PROJECTION) && !(d->rot == KVQ_ROT_PROJECTION && kc == KVQ_F16 && vc == KVQ_F16)) {
         delete p;
@@ -408,7 +418,7 @@ kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* se
     ap.block_table = p->d_bt;
     ap.max_pages_per_seq = p->mpps;
     ap.tail = p->cache + p->tail_off;
-    ap.T = T; ap.L = p->L; ap.layer = layer; ap.Hkv = p->Hkv; ap.rot = p->rot;
+    ap.T = T; ap.L = p->L; ap.layer = layer; ap.Hkv = p->Hkv; ap.rot = p->rot; ap.bf16 = p->bf16;
     ap.k_in = (const __half*)k_new;
     ap.v_in = (const __half*)v_new;
     ap.inv_s = p->d_inv ? p->d_inv + (size_t)layer * p->Hkv * 2 * D : nullptr;
@@ -629,6 +639,10 @@ kvq_status kvq_read_rows(const kvq_plan* p, int layer, int seq_id, int64_t t0, i
 // rank codec): head infos with region offsets, the page bytes and the stage bytes.
 static kvq_status regrade_layout(const kvq_plan* p, int layer, const int* kc, const int* vc,
                                  std::vector<HeadInfo>& heads, uint32_t& page_bytes, int& stage) {
+  if (p->bf16)
+    for (int h = 0; h < p->Hkv; ++h)
+      if (kc[h] == KVQ_F16 || vc[h] == KVQ_F16)
+        return fail(KVQ_ERR_UNSUPPORTED, "bf16 plans keep raw rows in the tail only: no KVQ_F16 pages");
   if (p->rot == KVQ_ROT_PROJECTION) return fail(KVQ_ERR_UNSUPPORTED, "regrade of projection plans is not supported");
   heads.assign(p->Hkv, HeadInfo{});
   uint32_t poff = 0;
@@ -700,6 +714,7 @@ kvq_status kvq_regrade_layer(kvq_plan* p, int layer, const int* k_codec, const i
   rp.max_pages_per_seq = p->mpps;
   rp.Hkv = p->Hkv;
   rp.rot = p->rot;
+  rp.bf16 = p->bf16;
   rp.inv_s = p->d_inv ? p->d_inv + (size_t)layer * p->Hkv * 2 * D : nullptr;
   rp.err = p->d_err;
   for (int h = 0; h < p->Hkv; ++h) { rp.src[h] = p->head(layer, h); rp.dst[h] = heads[h]; }
@@ -805,7 +820,7 @@ kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int 
     return KVQ_OK;
   }
   const float* inv = p->d_inv ? p->d_inv + (((size_t)layer * p->Hkv + head) * 2 + kv) * D : nullptr;
-  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, n, (const __half*)x, y, layout == KVQ_ROWS_QUAD,
+  cudaError_t e = launch_debug_rotate(h, p->rot, kv, inv, n, (const __half*)x, y, layout == KVQ_ROWS_QUAD, p->bf16,
                                       (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "debug_rotate launch");
   return KVQ_OK;

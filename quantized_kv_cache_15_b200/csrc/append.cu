@@ -123,16 +123,15 @@ __global__ void __launch_bounds__(256) append_warp_kernel(const __grid_constant_
     float x[4];
     if (w.ring_slot >= 0) {
       const uint2 r = *reinterpret_cast<const uint2*>(ring_chunk(w.ring, w.ring_slot, kv, lane >> 1) + 8 * (lane & 1));
-      const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
-      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+      const float2 fa = raw2_to_float2(r.x, p.bf16), fb = raw2_to_float2(r.y, p.bf16);
       x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
     } else {
-      load_row_f16(in + ((size_t)w.src_row * p.Hkv + w.head) * D, x);
+      load_row_raw(in + ((size_t)w.src_row * p.Hkv + w.head) * D, x, p.bf16);
     }
     transform_row(x, codec, p.rot, p.inv_s ? p.inv_s + ((size_t)w.head * 2 + kv) * D : nullptr);
     uint8_t *codes, *scales;
     if (!page_row(p, w, &codes, &scales, lane == 0)) return;
-    quantize_store_row(x, codec, h.r, kv ? h.vbits : h.kbits, codes, scales, w.pos % PAGE, kv == 0);
+    quantize_store_row(x, codec, h.r, kv ? h.vbits : h.kbits, codes, scales, w.pos % PAGE, kv == 0, p.bf16);
   }
   if (w.write_slot >= 0) {
     const uint2 r = *reinterpret_cast<const uint2*>(in + ((size_t)w.write_row * p.Hkv + w.head) * D + 4 * lane);
@@ -162,13 +161,13 @@ __global__ void __launch_bounds__(256) append_quad_kernel(const __grid_constant_
       const uint4 r = w.ring_slot >= 0
                           ? *reinterpret_cast<const uint4*>(ring_chunk(w.ring, w.ring_slot, kv, 4 * q + c))
                           : *reinterpret_cast<const uint4*>(in + ((size_t)w.src_row * p.Hkv + w.head) * D + 32 * q + 8 * c);
-      chunk_to_float(r, v + 8 * c);
+      chunk_to_float(r, v + 8 * c, p.bf16);
     }
     uint8_t *codes, *scales;
     if (!page_row(p, w, &codes, &scales, q == 0)) return;
     if (codec != KVQ_F16)
       transform_row_quad(v, p.rot, p.inv_s ? p.inv_s + ((size_t)w.head * 2 + kv) * D : nullptr);
-    quantize_row_quad(codec, v, codes, scales, w.pos % PAGE, kv == 0, kv ? h.cbV : h.cbK, kv ? h.sbV : h.sbK);
+    quantize_row_quad(codec, v, codes, scales, w.pos % PAGE, kv == 0, kv ? h.cbV : h.cbK, kv ? h.sbV : h.sbK, p.bf16);
   }
   if (w.write_slot >= 0) {
     const uint4* src = reinterpret_cast<const uint4*>(in + ((size_t)w.write_row * p.Hkv + w.head) * D + 32 * q);
@@ -254,37 +253,38 @@ cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __ha
 // ---------------------------------------------------------------- debug hooks
 // The row transform and the block quantizer alone, in either row layout.
 __global__ void debug_rotate_kernel(HeadInfo h, int rot, int kv, const float* inv_s, int n, const __half* x,
-                                    float* y) {
+                                    float* y, bool bf16) {
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int row = blockIdx.x * 8 + wib;
   if (row >= n) return;
   const int codec = kv ? h.vcodec : h.kcodec;
   float v[4];
-  load_row_f16(x + (size_t)row * D, v);
+  load_row_raw(x + (size_t)row * D, v, bf16);
   transform_row(v, codec, rot, inv_s);
 #pragma unroll
   for (int i = 0; i < 4; ++i) y[(size_t)row * D + 4 * lane + i] = v[i];
 }
 __global__ void debug_rotate_quad_kernel(HeadInfo h, int rot, int kv, const float* inv_s, int n, const __half* x,
-                                         float* y) {
+                                         float* y, bool bf16) {
   const int q = threadIdx.x & 3;
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 2;
   if (row >= n) return;                          // whole quads leave together
   const int codec = kv ? h.vcodec : h.kcodec;
   float v[32];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) chunk_to_float(*reinterpret_cast<const uint4*>(x + (size_t)row * D + 32 * q + 8 * c), v + 8 * c);
+  for (int c = 0; c < 4; ++c)
+    chunk_to_float(*reinterpret_cast<const uint4*>(x + (size_t)row * D + 32 * q + 8 * c), v + 8 * c, bf16);
   if (codec != KVQ_F16) transform_row_quad(v, rot, inv_s);
 #pragma unroll
   for (int i = 0; i < 32; ++i) y[(size_t)row * D + 32 * q + i] = v[i];
 }
 cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, int n, const __half* x,
-                                float* y, bool quad, cudaStream_t s) {
+                                float* y, bool quad, bool bf16, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   if (quad)
-    debug_rotate_quad_kernel<<<(n + 63) / 64, 256, 0, s>>>(h, rot, kv, inv_s, n, x, y);
+    debug_rotate_quad_kernel<<<(n + 63) / 64, 256, 0, s>>>(h, rot, kv, inv_s, n, x, y, bf16);
   else
-    debug_rotate_kernel<<<(n + 7) / 8, 256, 0, s>>>(h, rot, kv, inv_s, n, x, y);
+    debug_rotate_kernel<<<(n + 7) / 8, 256, 0, s>>>(h, rot, kv, inv_s, n, x, y, bf16);
   note_launches(1);
   return cudaGetLastError();
 }

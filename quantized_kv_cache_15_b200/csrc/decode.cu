@@ -97,21 +97,16 @@ __device__ __forceinline__ uint32_t kcode_generic(const uint8_t* kp, int cb, int
 template <int G>
 __device__ __forceinline__ void score_token(int kc, int kbits, int n, int cb, int sb, const uint8_t* kp,
                                             const uint8_t* ks, int t, const float* __restrict__ qv,
-                                            const float* __restrict__ qsum, float s[G], int rows) {
+                                            const float* __restrict__ qsum, float s[G], int rows, bool bf16) {
 #pragma unroll
   for (int g = 0; g < G; ++g) s[g] = 0.f;
   if (kc == KVQ_F16) {
     if (t >= rows) return;                 // past the end of a tail tile (TAIL_TOK rows)
 #pragma unroll 2
     for (int c = 0; c < 16; ++c) {
-      uint4 v = *reinterpret_cast<const uint4*>(kp + (c * rows + t) * 16);
-      const __half2* hv = reinterpret_cast<const __half2*>(&v);
+      const uint4 v = *reinterpret_cast<const uint4*>(kp + (c * rows + t) * 16);
       float x[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float2 f = __half22float2(hv[k]);
-        x[2 * k] = f.x; x[2 * k + 1] = f.y;
-      }
+      chunk_to_float(v, x, bf16);
 #pragma unroll
       for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -171,13 +166,12 @@ __device__ __forceinline__ void score_token(int kc, int kbits, int n, int cb, in
 
 // Dequantized values of the lane's 4 channels (4l..4l+3) of V row t (row-major plane).
 __device__ __forceinline__ void v_lane(int vc, int vbits, int n, int cb, int sb, const uint8_t* vp, const uint8_t* vs,
-                                       int t, int lane, float v[4]) {
+                                       int t, int lane, float v[4], bool bf16) {
   if (4 * lane >= n) { v[0] = v[1] = v[2] = v[3] = 0.f; return; }
   const uint8_t* row = vp + t * cb;
   if (vc == KVQ_F16) {
-    uint2 w = *reinterpret_cast<const uint2*>(row + 8 * lane);
-    float2 a = __half22float2(*reinterpret_cast<__half2*>(&w.x));
-    float2 b = __half22float2(*reinterpret_cast<__half2*>(&w.y));
+    const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * lane);
+    const float2 a = raw2_to_float2(w.x, bf16), b = raw2_to_float2(w.y, bf16);
     v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
     return;
   }
@@ -373,9 +367,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   if (warp < NCW) {
     for (int g = warp; g < G; g += NCW) {
       const __half* qsrc = p.q + ((size_t)si * p.Hq + (size_t)head * G + g) * D;
-      uint2 raw = *reinterpret_cast<const uint2*>(qsrc + 4 * lane);
-      float2 a = __half22float2(*reinterpret_cast<__half2*>(&raw.x));
-      float2 b = __half22float2(*reinterpret_cast<__half2*>(&raw.y));
+      const uint2 raw = *reinterpret_cast<const uint2*>(qsrc + 4 * lane);
+      const float2 a = raw2_to_float2(raw.x, p.bf16), b = raw2_to_float2(raw.y, p.bf16);
       float x[4] = {a.x, a.y, b.x, b.y};
       if (kbasis == BASIS_ROT) {
         if (p.s_k) {
@@ -523,8 +516,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
         case 13: score2_rank<G, 3>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         case 14: score2_rank<G, 4>(nK, kp, ks, cbK, sbK, lane, tab, tab + G * 64, qsi, s0, s1); break;
         default:
-          score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0, rows);
-          score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1, rows);
+          score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane, qv, qsum, s0, rows, p.bf16);
+          score_token<G>(kc, kbits, nK, cbK, sbK, kp, ks, lane + 32, qv, qsum, s1, rows, p.bf16);
       }
       if (kclass) {
 #pragma unroll
@@ -588,7 +581,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
             const int ntok = min(32, nvalid - 32 * half);
             for (int tt = 0; tt < ntok; ++tt) {
               float v[4];
-              v_lane(vc, vbits, nV, cbV, sbV, vp, vs, 32 * half + tt, lane, v);
+              v_lane(vc, vbits, nV, cbV, sbV, vp, vs, 32 * half + tt, lane, v, p.bf16);
               const uint64_t u01 = pack2(v[0], v[1]), u23 = pack2(v[2], v[3]);
               const uint64_t* wrow = pw + (size_t)tt * PWG;
 #pragma unroll

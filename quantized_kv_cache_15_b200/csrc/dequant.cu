@@ -35,9 +35,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
     const int r = slot % TAIL_TOK;
     const uint8_t* src = kv == 0 ? tp + ((lane >> 1) * TAIL_TOK + r) * 16 + (lane & 1) * 8
                                  : tp + TAIL_TOK * D * 2 + r * (D * 2) + 8 * lane;
-    uint2 w = *reinterpret_cast<const uint2*>(src);
-    float2 a = __half22float2(*reinterpret_cast<__half2*>(&w.x));
-    float2 b = __half22float2(*reinterpret_cast<__half2*>(&w.y));
+    const uint2 w = *reinterpret_cast<const uint2*>(src);
+    const float2 a = raw2_to_float2(w.x, p.bf16), b = raw2_to_float2(w.y, p.bf16);
     x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
   } else {
     const int codec = kv ? h.vcodec : h.kcodec;
@@ -53,9 +52,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const __grid_constant__ De
     if (codec == KVQ_F16) {
       const int o = 8 * lane;
       const uint8_t* src = codes + (kv == 0 ? kplane_off(cb, t, o) : t * cb + o);
-      uint2 w = *reinterpret_cast<const uint2*>(src);
-      float2 a = __half22float2(*reinterpret_cast<__half2*>(&w.x));
-      float2 b = __half22float2(*reinterpret_cast<__half2*>(&w.y));
+      const uint2 w = *reinterpret_cast<const uint2*>(src);
+      const float2 a = raw2_to_float2(w.x, p.bf16), b = raw2_to_float2(w.y, p.bf16);
       x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
     } else {
       uint32_t u[4];

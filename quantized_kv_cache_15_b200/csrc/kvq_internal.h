@@ -126,7 +126,8 @@ struct AppendParams {
   uint8_t* tail;                 // tail region base (all sequences and layers)
   int T, L, layer, Hkv;
   int rot;
-  const __half* k_in;
+  int bf16;                      // raw rows (input, ring, F16 pages) are bf16, else fp16
+  const __half* k_in;            // raw 16-bit rows (see bf16)
   const __half* v_in;
   const float* inv_s;            // [Hkv][2][128] of this layer, or null
   const float* M;                // projection table (floats), or null
@@ -168,7 +169,8 @@ struct DecodeParams {
   const uint8_t* tail;
   int T, L, layer, Hkv, Hq, G;
   int rot;
-  const __half* q;               // [n_seqs][Hq][128]
+  int bf16;                      // raw rows (q, tail, F16 pages) are bf16, else fp16
+  const __half* q;               // [n_seqs][Hq][128], raw 16-bit (see bf16)
   float* out;                    // [n_seqs][Hq][128]
   const float* s_k;              // [Hkv][128] per-channel K dequant multiplier (varnorm) or null
   const float* s_v;              // [Hkv][128] per-channel V multiplier or null
@@ -204,6 +206,7 @@ struct RegradeParams {
   const int* block_table;
   int max_pages_per_seq;
   int Hkv, rot;
+  int bf16;                      // F16-codec rows are bf16
   const float* inv_s;            // [Hkv][2][128] of this layer, or null
   int* err;
   int n_seqs;
@@ -222,7 +225,7 @@ cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t
 cudaError_t launch_project(const ProjParams& p, int n_tiles, int n_heads, cudaStream_t s);
 cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __half* x, float* inv, cudaStream_t s);
 cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, int n, const __half* x,
-                                float* y, bool quad, cudaStream_t s);
+                                float* y, bool quad, bool bf16, cudaStream_t s);
 cudaError_t launch_debug_quantize(int codec, int r, int b, int n, const float* y, uint8_t* codes, uint8_t* scales,
                                   bool quad, cudaStream_t s);
 size_t decode_smem_bytes(int stage_bytes, int n_stages, int G, bool wtab_smem);

@@ -27,11 +27,29 @@
 // (d_k, m_k).  F16: the fp16 values.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "kvq_internal.h"
 
 namespace kvq {
 
 __device__ __forceinline__ float hadamard_c() { return __uint_as_float(0x3db504f3u); }  // fp32(1/sqrt(128))
+
+// One word of two raw 16-bit values (bf16 or fp16) -> two floats (exact).
+__device__ __forceinline__ float2 raw2_to_float2(uint32_t w, bool bf16) {
+  if (bf16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+// Two floats -> one word of raw 16-bit values, rounded to nearest even (exact for
+// values that came from raw rows of the same dtype).
+__device__ __forceinline__ uint32_t float2_to_raw2(float a, float b, bool bf16) {
+  if (bf16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 // In-place staged Hadamard transform of the warp's row (4 values per lane),
 // followed by the multiplication by c.
@@ -200,17 +218,14 @@ __device__ __forceinline__ int kplane_off(int cb, int t, int i) {
 //   interleaved: K plane layout (true) or row-major (false).
 // For codec F16 the values are written as fp16 (they are fp16 values already).
 __device__ __forceinline__ void quantize_store_row(const float x[4], int codec, int r, int bits, uint8_t* codes,
-                                                   uint8_t* scales, int t, bool interleaved) {
+                                                   uint8_t* scales, int t, bool interleaved, bool bf16 = false) {
   const int lane = threadIdx.x & 31;
   const int n = (codec == KVQ_RANK) ? r : D;
   int cb, sb;
   row_bytes(codec, r, bits, &cb, &sb);
   const bool active = 4 * lane < n;
   if (codec == KVQ_F16) {
-    __half2 h01 = __floats2half2_rn(x[0], x[1]);
-    __half2 h23 = __floats2half2_rn(x[2], x[3]);
-    uint64_t v = (uint64_t)(*reinterpret_cast<uint32_t*>(&h01)) |
-                 ((uint64_t)(*reinterpret_cast<uint32_t*>(&h23)) << 32);
+    const uint64_t v = (uint64_t)float2_to_raw2(x[0], x[1], bf16) | ((uint64_t)float2_to_raw2(x[2], x[3], bf16) << 32);
     int off = 8 * lane;
     uint8_t* dst = codes + (interleaved ? kplane_off(cb, t, off) : t * cb + off);
     store_piece(dst, 8, v);
@@ -243,13 +258,11 @@ __device__ __forceinline__ void quantize_store_row(const float x[4], int codec, 
   }
 }
 
-// The warp's fp16 row (lane: 4 values) as fp32.
-__device__ __forceinline__ void load_row_f16(const __half* src, float x[4]) {
+// The warp's raw 16-bit row (lane: 4 values; bf16 or fp16) as fp32.
+__device__ __forceinline__ void load_row_raw(const __half* src, float x[4], bool bf16) {
   const int lane = threadIdx.x & 31;
-  uint2 v = *reinterpret_cast<const uint2*>(src + 4 * lane);
-  __half2 a = *reinterpret_cast<__half2*>(&v.x);
-  __half2 b = *reinterpret_cast<__half2*>(&v.y);
-  float2 fa = __half22float2(a), fb = __half22float2(b);
+  const uint2 v = *reinterpret_cast<const uint2*>(src + 4 * lane);
+  const float2 fa = raw2_to_float2(v.x, bf16), fb = raw2_to_float2(v.y, bf16);
   x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
 }
 
@@ -349,12 +362,12 @@ __device__ __forceinline__ void transform_row_quad(float v[32], int rot, const f
   fwht_quad(v);
 }
 
-// 16 bytes of raw fp16 values -> 8 floats.
-__device__ __forceinline__ void chunk_to_float(const uint4 w, float* x) {
+// 16 bytes of raw 16-bit values (bf16 or fp16) -> 8 floats.
+__device__ __forceinline__ void chunk_to_float(const uint4 w, float* x, bool bf16) {
   const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+    const float2 f = raw2_to_float2(u[k], bf16);
     x[2 * k] = f.x; x[2 * k + 1] = f.y;
   }
 }
@@ -489,7 +502,7 @@ __device__ __forceinline__ uint32_t quantize_block_quad(const float v[32], uint8
 // F16) with `codec` to token row t: F16 as fp16 values, block codecs through
 // quantize_block_quad, the four scale words written by lane 0 of the quad.
 __device__ __forceinline__ void quantize_row_quad(int codec, const float v[32], uint8_t* codes, uint8_t* scales,
-                                                  int t, bool kplane, int cb, int sb) {
+                                                  int t, bool kplane, int cb, int sb, bool bf16 = false) {
   const int b = threadIdx.x & 3;
   uint32_t sc = 0;
   switch (codec) {
@@ -498,10 +511,7 @@ __device__ __forceinline__ void quantize_row_quad(int codec, const float v[32], 
       for (int c = 0; c < 4; ++c) {
         uint32_t w[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const __half2 hv = __floats2half2_rn(v[8 * c + 2 * k], v[8 * c + 2 * k + 1]);
-          w[k] = *reinterpret_cast<const uint32_t*>(&hv);
-        }
+        for (int k = 0; k < 4; ++k) w[k] = float2_to_raw2(v[8 * c + 2 * k], v[8 * c + 2 * k + 1], bf16);
         *reinterpret_cast<uint4*>(row_word_ptr(codes, kplane, cb, t, 16 * b + 4 * c)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       return;

@@ -52,7 +52,8 @@ __global__ void __launch_bounds__(256) regrade_kernel(const __grid_constant__ Re
       // raw rows: into the stored basis of the new codec
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        chunk_to_float(*reinterpret_cast<const uint4*>(row_word_ptr(codes, kplane, cbs, t, 16 * q + 4 * c)), v + 8 * c);
+        chunk_to_float(*reinterpret_cast<const uint4*>(row_word_ptr(codes, kplane, cbs, t, 16 * q + 4 * c)), v + 8 * c,
+                       p.bf16);
       if (cd != KVQ_F16)
         transform_row_quad(v, p.rot, p.inv_s ? p.inv_s + ((size_t)head * 2 + kv) * D : nullptr);
     } break;
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(256) regrade_kernel(const __grid_constant__ Re
   const int cbd = kv ? hd.cbV : hd.cbK, sbd = kv ? hd.sbV : hd.sbK;
   uint8_t* dcodes = kv ? dregion + PAGE * (hd.cbK + hd.sbK) : dregion;
   uint8_t* dscales = dcodes + PAGE * cbd;
-  quantize_row_quad(cd, v, dcodes, dscales, t, kplane, cbd, sbd);
+  quantize_row_quad(cd, v, dcodes, dscales, t, kplane, cbd, sbd, p.bf16);
 }
 
 cudaError_t launch_regrade(const RegradeParams& p, cudaStream_t s) {

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 
 F16, Q8_0, Q6_0, Q4_0, Q3_0, Q2_0, Q8_1, Q6_1, Q4_1, Q3_1, Q2_1, RANK, Q5_0, Q5_1 = range(14)
 ROWS_WARP, ROWS_QUAD = 0, 1          # kvq_row_layout
+KV_F16, KV_BF16 = 0, 1                # kvq_kv_dtype
 ROT_NONE, ROT_HADAMARD, ROT_VARNORM_HADAMARD, ROT_PROJECTION = range(4)
 HEAD_DIM = 128
 PAGE_TOKENS = 64
@@ -69,7 +70,7 @@ class _Desc(ctypes.Structure):
                 ("max_seqs", _I), ("max_tokens_per_seq", _I64), ("max_pages", _I64), ("tail_tokens", _I),
                 ("k_codec", _IP), ("v_codec", _IP), ("rot", _I), ("inv_rms", ctypes.POINTER(ctypes.c_float)),
                 ("rank", _IP), ("k_bits", _IP), ("v_bits", _IP), ("proj_basis", ctypes.POINTER(ctypes.c_double)),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("kv_dtype", _I)]
 
 
 _lib = None
@@ -114,8 +115,10 @@ class Plan:
 
     def __init__(self, n_layers: int, n_q_heads: int, n_kv_heads: int, max_seqs: int, max_tokens_per_seq: int,
                  k_codec, v_codec, rot: int = ROT_HADAMARD, tail_tokens: int = 0, inv_rms=None, rank=None,
-                 k_bits=None, v_bits=None, proj_basis=None, softmax_scale: float = 0.0, max_pages: int = 0):
+                 k_bits=None, v_bits=None, proj_basis=None, softmax_scale: float = 0.0, max_pages: int = 0,
+                 kv_dtype: int = KV_F16):
         self.n_layers, self.n_q_heads, self.n_kv_heads = n_layers, n_q_heads, n_kv_heads
+        self.kv_dtype = kv_dtype
         self.tail_tokens = tail_tokens
         self.rot = rot
         n = n_layers * n_kv_heads
@@ -142,6 +145,7 @@ class Plan:
             keep.append(a)
             d.proj_basis = a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
         d.softmax_scale = softmax_scale
+        d.kv_dtype = kv_dtype
         h = ctypes.c_void_p()
         _check(lib().kvq_plan_create(ctypes.byref(d), ctypes.byref(h)))
         self._h = h
