@@ -145,7 +145,8 @@ kvq_status kvq_plan_cache_bytes(const kvq_plan* plan, size_t* bytes);
 
 /* Bytes of device workspace kvq_decode_attention needs for n_seqs sequences.
  * The workspace must be zero-filled once before its first use; every call
- * leaves its counters back at zero. */
+ * leaves its counters back at zero, and a workspace sized for n sequences serves
+ * every later call (decode or prefill) with at most n entries. */
 kvq_status kvq_plan_workspace_bytes(const kvq_plan* plan, int n_seqs, size_t* bytes);
 
 /* Attach caller-owned device memory of at least kvq_plan_cache_bytes(), 256-byte
@@ -178,6 +179,21 @@ kvq_status kvq_append_quantize(kvq_plan* plan, int layer, int n_seqs, const int*
 kvq_status kvq_decode_attention(kvq_plan* plan, int layer, int n_seqs, const int* seq_ids /*host*/,
                                 const void* q, float* out, void* workspace, size_t workspace_bytes,
                                 void* stream);
+
+/* Chunked-prefill attention over the quantized cache [forum thread on KV
+ * compression: dot, softmax, weighted average; BeeLlama v0.4.0 news §KV cache
+ * 精度尾部 for the tail]: the last n_q tokens of sequence seq_id in this layer,
+ * already appended, attend causally to the cache, so query i (position
+ * len - n_q + i) sees positions 0 .. len - n_q + i, quantized rows dequantized in
+ * registers and tail rows raw, with the same GQA grouping as decode.
+ *  q:   device raw dtype [n_q][n_q_heads][128];  out: device fp32 [n_q][n_q_heads][128]
+ *  workspace: kvq_plan_workspace_bytes(plan, min(n_q, KVQ_MAX_BATCH)), zeroed before
+ *    first use (the calls leave it ready for reuse).
+ * Each query runs the split-K decode kernel over its visible prefix, KVQ_MAX_BATCH
+ * queries per launch; keys and values are not shared between the queries of a
+ * launch (beyond what L2 keeps).  KVQ_ERR_INVALID_ARG if n_q exceeds the length. */
+kvq_status kvq_prefill_attention(kvq_plan* plan, int layer, int seq_id, int n_q, const void* q, float* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* Decode attention without any allocation, for callers that cannot allocate
  * device memory (no counterpart in the pages: this is a deployment variant of

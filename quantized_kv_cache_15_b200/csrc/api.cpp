@@ -329,8 +329,12 @@ static size_t partial_bytes(const kvq_plan* p, int n_seqs) {
 static size_t qproj_bytes(const kvq_plan* p, int n_seqs) {
   return p->rot == KVQ_ROT_PROJECTION ? (size_t)n_seqs * p->Hq * D * sizeof(float) : 0;
 }
+// Workspace layout: [merge tickets for KVQ_MAX_BATCH entries][partials][projected
+// queries].  The tickets sit at a fixed place whatever the call's entry count, so a
+// workspace zeroed once serves every later call with at most as many entries.
+static size_t ticket_bytes(const kvq_plan* p) { return ((size_t)MAX_BATCH * p->Hkv * sizeof(int) + 255) & ~(size_t)255; }
 static size_t workspace_bytes(const kvq_plan* p, int n_seqs) {
-  return partial_bytes(p, n_seqs) + qproj_bytes(p, n_seqs) + (size_t)n_seqs * p->Hkv * sizeof(int);
+  return ticket_bytes(p) + partial_bytes(p, n_seqs) + qproj_bytes(p, n_seqs);
 }
 
 kvq_status kvq_plan_workspace_bytes(const kvq_plan* p, int n_seqs, size_t* bytes) {
@@ -475,8 +479,13 @@ kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* se
   return KVQ_OK;
 }
 
-kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const void* q, float* out,
-                                void* workspace, size_t workspace_bytes_given, void* stream) {
+}  // extern "C"
+
+// One decode launch over n_seqs entries; entry i attends sequence seq_ids[i] over
+// its first lims[i] tokens (all of them when lims is null).
+static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* lims,
+                                const void* q, float* out, void* workspace, size_t workspace_bytes_given,
+                                void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
@@ -496,7 +505,10 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
     const int64_t len = p->len[(size_t)s * p->L + layer];
     dp.seq[i] = s;
     dp.len[i] = (int)len;
-    const SplitCounts c = split_counts((int)len, (int)p->T, 1);
+    dp.lim[i] = lims ? lims[i] : (int)len;
+    if (dp.lim[i] < 0 || dp.lim[i] > len) return fail(KVQ_ERR_INVALID_ARG, "visible length %d outside [0, %lld]",
+                                                       dp.lim[i], (long long)len);
+    const SplitCounts c = split_counts((int)len, (int)p->T, 1, dp.lim[i]);
     const int pages = c.nqp + c.ntp;
     work += (int64_t)pages * p->Hkv;
     maxpages = std::max(maxpages, pages);
@@ -531,7 +543,7 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   auto makespan = [&](int pp) {
     int64_t ctas = 0;
     for (int i = 0; i < n_seqs; ++i) {
-      const SplitCounts c = split_counts(dp.len[i], (int)p->T, pp);
+      const SplitCounts c = split_counts(dp.len[i], (int)p->T, pp, dp.lim[i]);
       ctas += (int64_t)(c.qsplits + c.tsplits) * p->Hkv;
     }
     return ((ctas + target - 1) / target) * (int64_t)(pp + 3);
@@ -550,7 +562,7 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   dp.pps = pps;
   int grid_x = 1;
   for (int i = 0; i < n_seqs; ++i) {
-    const SplitCounts c = split_counts(dp.len[i], (int)p->T, pps);
+    const SplitCounts c = split_counts(dp.len[i], (int)p->T, pps, dp.lim[i]);
     grid_x = std::max(grid_x, c.qsplits + c.tsplits);
   }
   const bool proj = p->rot == KVQ_ROT_PROJECTION;
@@ -559,9 +571,9 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
     if (!workspace || workspace_bytes_given < need)
       return fail(KVQ_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes_given);
     if ((uintptr_t)workspace % 16) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-    dp.ws = (float*)workspace;
-    dp.qproj = (float*)((char*)workspace + partial_bytes(p, n_seqs));
-    dp.tickets = (int*)((char*)workspace + partial_bytes(p, n_seqs) + qproj_bytes(p, n_seqs));
+    dp.tickets = (int*)workspace;
+    dp.ws = (float*)((char*)workspace + ticket_bytes(p));
+    dp.qproj = (float*)((char*)workspace + ticket_bytes(p) + partial_bytes(p, n_seqs));
   }
   if (proj) {
     cudaError_t e = launch_project_query(dp, (cudaStream_t)stream);
@@ -569,6 +581,37 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   }
   cudaError_t e = launch_decode(dp, grid_x, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KVQ_OK;
+}
+
+extern "C" {
+
+kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const void* q, float* out,
+                                void* workspace, size_t workspace_bytes_given, void* stream) {
+  return decode_launch(p, layer, n_seqs, seq_ids, nullptr, q, out, workspace, workspace_bytes_given, stream);
+}
+
+kvq_status kvq_prefill_attention(kvq_plan* p, int layer, int seq_id, int n_q, const void* q, float* out,
+                                 void* workspace, size_t workspace_bytes_given, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
+  if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d out of range", seq_id);
+  const int64_t len = p->len[(size_t)seq_id * p->L + layer];
+  if (n_q < 0 || n_q > len) return fail(KVQ_ERR_INVALID_ARG, "n_q %d outside [0, %lld]", n_q, (long long)len);
+  if (n_q == 0) return KVQ_OK;
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "null q or out");
+  int ids[MAX_BATCH], lims[MAX_BATCH];
+  for (int c0 = 0; c0 < n_q; c0 += MAX_BATCH) {
+    const int n = std::min(MAX_BATCH, n_q - c0);
+    for (int i = 0; i < n; ++i) {
+      ids[i] = seq_id;
+      lims[i] = (int)(len - n_q + c0 + i + 1);          // query c0 + i sits at position len - n_q + c0 + i
+    }
+    const kvq_status st = decode_launch(p, layer, n, ids, lims, (const char*)q + (size_t)c0 * p->Hq * D * 2,
+                                        out + (size_t)c0 * p->Hq * D, workspace, workspace_bytes_given, stream);
+    if (st != KVQ_OK) return st;
+  }
   return KVQ_OK;
 }
 
@@ -586,7 +629,7 @@ kvq_status kvq_decode_attention_noalloc(kvq_plan* p, int layer, int n_seqs, cons
   // merge counters must start at zero (partials are written before they are read)
   const size_t tickets = (size_t)n_seqs * p->Hkv * sizeof(int);
   if (tickets) {
-    e = cudaMemsetAsync((char*)scratch + (need - tickets), 0, tickets, (cudaStream_t)stream);
+    e = cudaMemsetAsync(scratch, 0, tickets, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "scratch counter reset");
   }
   return kvq_decode_attention(p, layer, n_seqs, seq_ids, q, out, scratch, NOALLOC_SCRATCH_BYTES, stream);

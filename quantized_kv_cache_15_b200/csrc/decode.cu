@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
   const int seq = p.seq[si], len = p.len[si];
   const int T = p.T;
-  const SplitCounts sc = split_counts(len, T, p.pps);
+  const SplitCounts sc = split_counts(len, T, p.pps, p.lim[si]);
   const int nq = sc.nq, nt = sc.nt, NQP = sc.nqp, NTP = sc.ntp, qsplits = sc.qsplits;
   const int S = sc.qsplits + sc.tsplits;
   float* out_base = p.out + ((size_t)si * p.Hq + (size_t)head * G) * D;
@@ -504,6 +504,14 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
       uint32_t* wq = reinterpret_cast<uint32_t*>(pw);
       const int tok0 = (pg0 + i) * rows;
       const int nvalid = min(rows, seg_tokens - tok0);
+      // the lane's first token (the second one, lane + 32, lies past a 16-row tail
+      // tile): inside the segment, and for a tail slot also visible to the query
+      const bool vis0 = lane < nvalid && (!is_tail || tail_visible(sc, T, tok0 + lane));
+      if (is_tail && !__any_sync(0xffffffffu, vis0)) {   // no visible token in this tile
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+        continue;
+      }
       float s0[G], s1[G];
       switch (kclass) {
 #define KVQ_SCORE(KCL, ASYM) score2_block_codec<G, KCL, ASYM>(kc, kp, ks, sbK, lane, tab, tab + G * 64, qsi, s0, s1)
@@ -526,7 +534,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
       float p0[G], p1[G], pm[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        if (lane >= nvalid) s0[g] = -INFINITY;
+        if (!vis0) s0[g] = -INFINITY;
         if (lane + 32 >= nvalid) s1[g] = -INFINITY;
         const float tmax = warp_max(fmaxf(s0[g], s1[g]));
         const float mnew = fmaxf(m[g], tmax);

@@ -50,16 +50,30 @@ constexpr int DECODE_THREADS = 32 * (NCW + 1);
 // Split-K layout of one sequence of `len` tokens, shared by the host (grid size)
 // and the decode kernel: the quantized segment in 64-token pages, the tail
 // segment in TAIL_TOK-token tail pages, each cut into splits of `pps` pages.
-struct SplitCounts { int nq, nt, nqp, ntp, qsplits, tsplits; };
-__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps) {
+// Splits of one (sequence, kv head) of length len whose query sees the first lim
+// tokens (lim = len for decode; lim < len for the earlier queries of a prefill
+// chunk).  nq: visible quantized tokens (pages in position order); nt: tail slots
+// to visit.  While len <= T the tail holds positions 0 .. len-1 in slots 0 .. len-1,
+// so the visible ones are the first lim slots.  Past that every slot is occupied
+// and the visible positions nq_all .. lim-1 sit in a cyclic run of slots starting
+// at nq_all mod T: all T slots are visited and the others are masked (tail_visible).
+struct SplitCounts { int nq, nt, nqp, ntp, qsplits, tsplits, nq_all, nt_vis; };
+__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps, int lim) {
   SplitCounts c;
-  c.nq = len > T ? len - T : 0;
-  c.nt = len < T ? len : T;
+  c.nq_all = len > T ? len - T : 0;
+  c.nq = c.nq_all < lim ? c.nq_all : lim;
+  c.nt_vis = lim > c.nq_all ? lim - c.nq_all : 0;
+  c.nt = len <= T ? c.nt_vis : (c.nt_vis > 0 ? T : 0);
   c.nqp = (c.nq + PAGE - 1) / PAGE;
   c.ntp = (c.nt + TAIL_TOK - 1) / TAIL_TOK;
   c.qsplits = (c.nqp + pps - 1) / pps;
   c.tsplits = (c.ntp + pps - 1) / pps;
   return c;
+}
+__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps) { return split_counts(len, T, pps, len); }
+// Whether tail slot s holds a visible position (see split_counts).
+__host__ __device__ inline bool tail_visible(const SplitCounts& c, int T, int s) {
+  return ((s - c.nq_all % T) % T + T) % T < c.nt_vis;
 }
 
 // Device error word bits.
@@ -188,6 +202,7 @@ struct DecodeParams {
   HeadInfo heads[MAX_HKV];
   int seq[MAX_BATCH];
   int len[MAX_BATCH];
+  int lim[MAX_BATCH];            // tokens the entry's query sees (len, or fewer for prefill queries)
 };
 
 // ---------------------------------------------------------------- launchers (host)

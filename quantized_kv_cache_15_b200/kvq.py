@@ -39,6 +39,7 @@ SIGNATURES = {
     "kvq_cache_bind": (_I, [_P, _P, _SZ]),
     "kvq_append_quantize": (_I, [_P, _I, _I, _IP, _IP, _P, _P, _P]),
     "kvq_decode_attention": (_I, [_P, _I, _I, _IP, _P, _P, _P, _SZ, _P]),
+    "kvq_prefill_attention": (_I, [_P, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "kvq_decode_attention_noalloc": (_I, [_P, _I, _I, _IP, _P, _P, _P]),
     "kvq_plan_regrade_bytes": (_I, [_P, _I, _IP, _IP, ctypes.POINTER(ctypes.c_size_t)]),
     "kvq_regrade_layer": (_I, [_P, _I, _IP, _IP, _P, ctypes.c_size_t, _P]),
@@ -237,6 +238,11 @@ class Plan:
 
     def check_device_error(self, stream=None):
         _check(lib().kvq_check_device_error(self._h, _stream(stream)))
+
+    def prefill(self, layer: int, seq: int, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, stream=None):
+        """Causal attention of the last q.shape[0] tokens of `seq` (already appended)."""
+        _check(lib().kvq_prefill_attention(self._h, layer, seq, q.shape[0], _ptr(q), _ptr(out), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream)))
 
     def debug_rotate(self, layer: int, head: int, kv: int, x: torch.Tensor, y: torch.Tensor, layout: int = 0,
                      stream=None):

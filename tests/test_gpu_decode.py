@@ -128,3 +128,22 @@ def test_every_codec_as_key_and_value(kc):
     plan = H.make_plan(w)
     H.fill(plan, w, chunk=250)
     _check(plan, w)
+
+
+def test_one_workspace_serves_calls_of_any_smaller_size():
+    """The merge counters sit at a fixed place in the workspace, so one zeroed
+    workspace serves a mix of batch sizes (here 6, 2, 5, 6 sequences)."""
+    w = W.make_workload(5, "small")
+    plan = H.make_plan(w)
+    H.fill(plan, w, chunk=640)
+    ws = plan.new_workspace(w.batch)
+    for seqs in (list(range(w.batch)), [4, 1], [0, 2, 3, 4, 5], list(range(w.batch))):
+        q = torch.stack([w.queries(0, s, 0, "cuda") for s in seqs])
+        out = torch.empty((len(seqs), w.n_q_heads, 128), dtype=torch.float32, device="cuda")
+        plan.decode(0, seqs, q, out, ws)
+        torch.cuda.synchronize()
+        out = out.cpu().numpy()
+        for i, s in enumerate(seqs):
+            for h in range(w.n_kv_heads):
+                ref = H.oracle_decode(w, 0, s, h, H.f16_bits(q[i, h * w.G:(h + 1) * w.G]))
+                assert H.rel_err_rows(out[i, h * w.G:(h + 1) * w.G], ref).max() <= H.TOL, (seqs, s, h)
