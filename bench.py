@@ -484,6 +484,30 @@ def run_kvq(args, world, rank, local):
 
     app_step_bytes = sum(n_app * n_app_seqs * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, l, Hkv)) for l in range(L))
     step_bytes = sum(dec_bytes_all) + app_step_bytes
+    # ---- chunked-prefill attention: the newest (up to) 2048 tokens of the longest
+    # sequence in layer 0 attend causally to the cache (one kvq_prefill_attention call)
+    ps = max(seqs, key=lambda s: plan.seq_length(s, 0))
+    p_len = plan.seq_length(ps, 0)
+    n_pq = min(2048, p_len)
+    pq = torch.stack([w.queries(0, ps, i, dev) for i in range(n_pq)]).contiguous()
+    pout = torch.empty((n_pq, Hq, 128), dtype=torch.float32, device=dev)
+    pws = plan.new_workspace(min(n_pq, 256))
+    pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        plan.prefill(0, ps, pq, pout, pws, stream)                      # warm-up
+        pa.record(stream)
+        for _ in range(2):
+            plan.prefill(0, ps, pq, pout, pws, stream)
+        pb.record(stream)
+    stream.synchronize()
+    plan.check_device_error(stream)
+    p_ms = pa.elapsed_time(pb) / 2
+    prefill = {"layer": 0, "seq": int(ps), "queries": n_pq, "context": int(p_len), "ms": p_ms,
+               "tokens_per_s": n_pq / (p_ms / 1e3),
+               "note": "causal: query i sees the first len - n_q + i + 1 tokens; each query runs the split-K "
+                       "decode kernel over its prefix (256 queries per launch)"}
+    del pws, pq, pout
+
     # ---- VBR regrade of one layer (last, since it changes that layer's codecs):
     # K to q4_0 and V to q2_0 where that does not grow the pages
     regrade = None
@@ -538,6 +562,7 @@ def run_kvq(args, world, rank, local):
         "append_note": f"2048-token chunk appended to all {L} layers (K and V quantized): {app_ms:.3f} ms, "
                        f"{app_bytes / (app_ms / 1e3) / 1e9:.0f} GB/s algorithmic",
         "regrade": regrade,
+        "prefill": prefill,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "kernel": f"decode_kernel<{w.G}>",
                      "bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
