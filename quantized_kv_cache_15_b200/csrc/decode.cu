@@ -690,13 +690,14 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   if (!flag[0]) return;
   // ---- last CTA: merge every split in a fixed order (deterministic).  Each head's
   // S partials are pulled into shared memory with one bulk copy (double-buffered
-  // over the heads when room allows); one warp reduces the split maxima and sums,
-  // then one thread per channel sums the rescaled partials.
+  // over the heads when room allows); meanwhile every head's split maxima, factors
+  // and sums are taken straight from L2, and then one thread per channel sums the
+  // rescaled partials of a head as it lands.
   const uint32_t per_g = (uint32_t)S * PARTIAL_FLOATS * 4;
   const size_t stage_off = (post_bytes(G) + 127) & ~(size_t)127;
   const size_t stage_room = (size_t)(reinterpret_cast<uint8_t*>(full) - smem) - stage_off;   // all dead after the loop
   const int nbuf = min(min(G, 2), (int)(stage_room / per_g));      // >= 1: see decode_smem_bytes
-  float* fsc = mg;                                                  // [MAX_SPLITS] factors of the current head
+  float* fsc = mg;                                                  // [G][MAX_SPLITS] split factors
   if (threadIdx.x == 0) {
     fence_proxy_async_global();          // the acquired partials, read through the bulk-copy path
     fence_proxy_async_shared();          // the staging area was last used by ordinary loads and stores
@@ -706,37 +707,51 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
                &mmerge[b]);
     }
   }
+  // every head's split maxima, factors and sums, read from L2 while the copies land
+  // (the partials were published with release and acquired by the ticket above)
+  for (int g = warp; g < G; g += blockDim.x / 32) {
+    float ms[2], ls[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s2 = lane + 32 * k;
+      const float* src = pbase + ((size_t)g * MAX_SPLITS + s2) * PARTIAL_FLOATS;
+      ms[k] = s2 < S ? __ldcg(src) : -INFINITY;
+      ls[k] = s2 < S ? __ldcg(src + 1) : 0.f;
+    }
+    const float M = warp_max(fmaxf(ms[0], ms[1]));
+    float part = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s2 = lane + 32 * k;
+      const float f = (ms[k] == -INFINITY) ? 0.f : exp2f(ms[k] - M);
+      if (s2 < S) fsc[g * MAX_SPLITS + s2] = f;
+      part += f * ls[k];
+    }
+    const float L = warp_sum(part);
+    if (lane == 0) { fm[g] = M; fl[g] = L; }
+  }
+  __syncthreads();
   for (int g = 0; g < G; ++g) {
     const int b = g % nbuf;
     if (!mbar_wait(&mmerge[b], (g / nbuf) & 1)) atomicOr(p.err, ERR_TIMEOUT);
     const float* pg = reinterpret_cast<const float*>(smem + stage_off + (size_t)b * per_g);
-    if (warp == 0) {
-      float ms[2], ls[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int s = lane + 32 * k;
-        ms[k] = s < S ? pg[(size_t)s * PARTIAL_FLOATS] : -INFINITY;
-        ls[k] = s < S ? pg[(size_t)s * PARTIAL_FLOATS + 1] : 0.f;
-      }
-      const float M = warp_max(fmaxf(ms[0], ms[1]));
-      float part = 0.f;
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int s = lane + 32 * k;
-        const float f = (ms[k] == -INFINITY) ? 0.f : exp2f(ms[k] - M);
-        if (s < S) fsc[s] = f;
-        part += f * ls[k];
-      }
-      const float L = warp_sum(part);
-      if (lane == 0) { fm[g] = M; fl[g] = L; }
-    }
-    __syncthreads();
+    const float* fg = fsc + g * MAX_SPLITS;
+    // two chains per sum (even and odd splits), added in that order: a fixed order
     for (int c = threadIdx.x; c < D; c += blockDim.x) {
-      float A = 0.f, B = 0.f;
-      for (int s2 = 0; s2 < qsplits; ++s2) A = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fsc[s2], A);
-      for (int s2 = qsplits; s2 < S; ++s2) B = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fsc[s2], B);
-      aq[g * D + c] = A;
-      at[g * D + c] = B;
+      float A0 = 0.f, A1 = 0.f, B0 = 0.f, B1 = 0.f;
+      int s2 = 0;
+      for (; s2 + 1 < qsplits; s2 += 2) {
+        A0 = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fg[s2], A0);
+        A1 = fmaf(pg[(size_t)(s2 + 1) * PARTIAL_FLOATS + 4 + c], fg[s2 + 1], A1);
+      }
+      if (s2 < qsplits) { A0 = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fg[s2], A0); ++s2; }
+      for (; s2 + 1 < S; s2 += 2) {
+        B0 = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fg[s2], B0);
+        B1 = fmaf(pg[(size_t)(s2 + 1) * PARTIAL_FLOATS + 4 + c], fg[s2 + 1], B1);
+      }
+      if (s2 < S) B0 = fmaf(pg[(size_t)s2 * PARTIAL_FLOATS + 4 + c], fg[s2], B0);
+      aq[g * D + c] = A0 + A1;
+      at[g * D + c] = B0 + B1;
     }
     __syncthreads();
     if (threadIdx.x == 0 && g + nbuf < G) {
