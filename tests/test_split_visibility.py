@@ -1,0 +1,69 @@
+"""Host-side check of the split and causal-visibility arithmetic that decode and
+chunked prefill share (split_counts / tail_visible in the library's internal
+header), compiled with the host compiler and run on the CPU.
+
+For every (len, tail T, visible length lim) the tiles the kernel visits and the
+slots it keeps must cover exactly positions 0 .. lim-1: the quantized pages in
+position order, then the tail ring, where position p lives in slot p % T.
+"""
+import os
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "quantized_kv_cache_15_b200", "csrc")
+CUDA_INC = "/usr/local/cuda/include"
+
+PROGRAM = r'''
+#include <cstdio>
+#include <vector>
+#include "kvq_internal.h"
+using namespace kvq;
+int main() {
+  long checked = 0;
+  const int tails[] = {0, 16, 64, 256, 1024};
+  for (int T : tails)
+    for (int len = 0; len <= 1300; len += (len < 200 ? 1 : 37))
+      for (int lim = 0; lim <= len; lim += (len < 200 ? 1 : 13)) {
+        for (int pps : {1, 3, 8}) {
+          const SplitCounts c = split_counts(len, T, pps, lim);
+          const int nq_all = len > T ? len - T : 0;
+          std::vector<int> seen(len > 0 ? len : 1, 0);
+          // quantized pages: splits of pps pages, 64 rows each, first nq tokens
+          if (c.qsplits * pps < c.nqp || (c.qsplits - 1) * pps >= c.nqp + (c.nqp == 0)) { printf("bad qsplits\n"); return 1; }
+          for (int t = 0; t < c.nq; ++t) seen[t]++;
+          // tail: ntp tiles of TAIL_TOK slots, slots < nt visited, then masked
+          if (c.tsplits * pps < c.ntp) { printf("bad tsplits\n"); return 1; }
+          for (int s = 0; s < c.ntp * TAIL_TOK; ++s) {
+            if (s >= c.nt) continue;
+            if (!tail_visible(c, T, s)) continue;
+            const int p = len <= T ? s : nq_all + ((s - nq_all) % T + T) % T;
+            if (p < nq_all || p >= len) { printf("slot %d maps outside the tail\n", s); return 1; }
+            seen[p]++;
+          }
+          for (int p = 0; p < len; ++p)
+            if (seen[p] != (p < lim ? 1 : 0)) {
+              printf("len %d T %d lim %d pps %d: position %d seen %d times\n", len, T, lim, pps, p, seen[p]);
+              return 1;
+            }
+          ++checked;
+        }
+      }
+  printf("ok %ld\n", checked);
+  return 0;
+}
+'''
+
+
+def test_visited_tiles_cover_exactly_the_visible_prefix(tmp_path):
+    if not os.path.isdir(CUDA_INC):
+        pytest.skip("CUDA headers not installed")
+    src = tmp_path / "vis.cpp"
+    src.write_text(PROGRAM)
+    exe = tmp_path / "vis"
+    r = subprocess.run(["g++", "-O1", "-std=c++17", "-I", CSRC, "-I", CUDA_INC, str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout[-500:]
