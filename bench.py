@@ -247,6 +247,20 @@ def cpu_oracle_decode_us_per_token(w, seconds, log, max_pairs=None, threads=None
 
 
 # ----------------------------------------------------------------------------- reference arm
+def workload_config(w, layers, world, l2):
+    """The `config` object of both arms' JSON lines for workload w."""
+    B = w.batch
+    n_app = w.append_tokens if w.append_tokens else 1
+    n_app_seqs = w.append_seqs if w.append_seqs else B
+    codecs = sorted({W_NAMES[c] for row in w.k_codec for c in row}) + sorted({W_NAMES[c] for row in w.v_codec for c in row})
+    return {"workload": w.name, "layers": layers, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads, "head_dim": 128,
+            "batch": B, "context": w.ctx[0] if B == 1 else f"{min(w.ctx)}..{max(w.ctx)} (mean {sum(w.ctx) / B:.0f})",
+            "tail": w.tail, "codecs_k_v": codecs,
+            "rotation": ["none", "hadamard-128", "varnorm+hadamard-128", "per-head projection"][w.rot],
+            "step": f"per layer: append {n_app} token(s) x {n_app_seqs} seq(s) + decode attention for {B} seq(s)",
+            "parallelism": f"replicas x{world}", "l2": l2}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -263,8 +277,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us/token", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "layers": w.n_layers, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
-                       "context": w.ctx[0], "batch": 1},
+            "config": workload_config(w, w.n_layers, world, "n/a: the oracle runs on the host cores"),
             "cpu_baseline": {"value": v, "unit": "us/token", "cores": threads, "kind": "oracle",
                              "sample": f"each step: oracle decode of {threads} (layer, kv head) pairs of sequence 0 "
                                        f"over its full context on {threads} host threads at once, scaled to every "
@@ -543,18 +556,12 @@ def run_kvq(args, world, rank, local):
     traffic = traffic_from_profile(os.path.join(ROOT, "quantized_kv_cache_15_b200", "csrc", "decode.cu"))
     hbm_gbs = step_bytes / (step_ms / 1e3) / 1e9
     us_per_token = step_ms * 1e3 / (B * world)
-    codecs = sorted({W_NAMES[c] for row in w.k_codec for c in row}) + sorted({W_NAMES[c] for row in w.v_codec for c in row})
     line = {
         "metric": METRIC, "value": us_per_token, "unit": "us/token", "n_gpus": world, "steps": K, "warmup": Wm,
         "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": {"workload": w.name, "layers": L, "q_heads": Hq, "kv_heads": Hkv, "head_dim": 128,
-                   "batch": B, "context": w.ctx[0] if B == 1 else f"{min(w.ctx)}..{max(w.ctx)} (mean {sum(w.ctx) / B:.0f})",
-                   "tail": w.tail, "codecs_k_v": codecs, "rotation": ["none", "hadamard-128", "varnorm+hadamard-128",
-                                                                       "per-head projection"][w.rot],
-                   "step": f"per layer: append {n_app} token(s) x {n_app_seqs} seq(s) + decode attention for {B} seq(s)",
-                   "parallelism": f"replicas x{world}",
-                   "l2": "no flush: packed cache read per step (%.2f GB) >> L2 (126 MB)" % (sum(dec_bytes_all) / 1e9)},
+        "config": workload_config(w, L, world, "no flush: packed cache read per step (%.2f GB) >> L2 (126 MB)"
+                                  % (sum(dec_bytes_all) / 1e9)),
         "us_per_step": step_ms * 1e3,
         "hbm_gbs": hbm_gbs, "hbm_frac_of_8tbs": hbm_gbs / NOMINAL_HBM_GBS,
         "hbm_frac_of_measured": hbm_gbs / peak,
