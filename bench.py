@@ -113,9 +113,10 @@ def kernel_source_sha256():
     return h.hexdigest()
 
 
-def traffic_from_profile(kernel_file=None):
-    """dram bytes per launch recorded in profiles/decode_attention_llama8b.md, if the
-    kernel source still matches the one profiled (else None)."""
+def traffic_from_profile(workload):
+    """dram bytes per decode launch recorded in profiles/decode_attention_llama8b.md,
+    if that capture is of this workload and the kernel source still matches the one
+    profiled (else None)."""
     path = os.path.join(ROOT, "profiles", "decode_attention_llama8b.md")
     try:
         text = open(path).read()
@@ -123,7 +124,8 @@ def traffic_from_profile(kernel_file=None):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
-    if not m or not h:
+    wl = re.search(r"profiled_workload:\s*(\S+)", text)
+    if not m or not h or not wl or wl.group(1) != workload:
         return None
     if kernel_source_sha256() != h.group(1):
         return None
@@ -553,7 +555,7 @@ def run_kvq(args, world, rank, local):
     peaks = measured_peaks()
     peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
-    traffic = traffic_from_profile(os.path.join(ROOT, "quantized_kv_cache_15_b200", "csrc", "decode.cu"))
+    traffic = traffic_from_profile(w.name)
     hbm_gbs = step_bytes / (step_ms / 1e3) / 1e9
     us_per_token = step_ms * 1e3 / (B * world)
     line = {
