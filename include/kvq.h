@@ -2,8 +2,9 @@
  * kvq.h -- C ABI of the B200 quantized KV cache: append-quantize and decode
  * attention over packed q8/q6/q4/q3/q2 (_0 and _1), F16 and per-head rank/bit
  * codecs, with a Hadamard rotation (optionally variance-normalised, or fused
- * into a per-head projection), an F16 precision tail for the newest tokens, a
- * per-layer / per-head codec map and grouped-query decode attention.
+ * into a per-head projection), an F16 (or BF16) precision tail for the newest
+ * tokens, a per-layer / per-head codec map, grouped-query decode attention and
+ * chunked-prefill attention over the cache.
  *
  * Sources (web pages, cited by title and section):
  *  - "BeeLlama.cpp v0.4.0 发布：聚焦 KV cache 量化，新增 KVarN 与精度尾部机制":
@@ -78,10 +79,16 @@ typedef enum {
  *     min(32, r) coordinates is quantized mid-rise with all 2^b levels
  *     (levels (k + 1/2) d, d = max|z| / (2^(b-1) - 1/2)); r and b per head.
  *  KVQ_F16: raw fp16 rows (unrotated).
- * Codes are stored offset-binary (u = code + 2^(b-1) for _0).  Bit planes:
- * 6 bits = 4-bit plane + 2-bit plane, 5 bits = 4-bit plane + 1-bit plane,
- * 3 bits = 2-bit plane + 1-bit plane.  Byte layouts are given in the
- * repository's design document. */
+ * Codes are stored offset-binary (u = code + 2^(b-1) for _0).  A canonical
+ * packed row (what kvq_read_rows returns) is the code planes, then the block
+ * scales.  Planes hold b-bit fields, lowest field in the lowest bits of each
+ * byte, in value order; 6 bits = 4-bit plane then 2-bit plane, 5 bits = 4-bit
+ * plane then 1-bit plane, 3 bits = 2-bit plane then 1-bit plane (a value's low
+ * bits in the first plane).  Scales: fp16 d per block (_0, KVQ_RANK), or fp16
+ * (d, m) pairs per block (_1).  Row bytes for 128 values: 16 b of codes plus 8
+ * (_0) or 16 (_1) of scales; F16 rows are the 256 bytes of raw values.  In the
+ * cache, a page's K code rows are interleaved in 16-byte chunks across its 64
+ * token rows and every other plane is row-major. */
 typedef enum {
   KVQ_F16 = 0, KVQ_Q8_0 = 1, KVQ_Q6_0 = 2, KVQ_Q4_0 = 3, KVQ_Q3_0 = 4, KVQ_Q2_0 = 5,
   KVQ_Q8_1 = 6, KVQ_Q6_1 = 7, KVQ_Q4_1 = 8, KVQ_Q3_1 = 9, KVQ_Q2_1 = 10, KVQ_RANK = 11,
@@ -119,7 +126,8 @@ typedef struct {
   int64_t max_tokens_per_seq;   /* capacity of one sequence (every layer) */
   int64_t max_pages;            /* pages in the pool (each page: 64 tokens x all kv heads of a layer, in
                                    every layer); 0 = max_seqs * ceil(max_tokens_per_seq / 64) */
-  int tail_tokens;              /* F16 precision tail length per (seq, layer, kv-head); 0 or a multiple of 64 */
+  int tail_tokens;              /* precision tail length per (seq, layer, kv-head), raw rows in kv_dtype;
+                                   0 or a multiple of 64 */
   const int* k_codec;           /* host [n_layers][n_kv_heads] kvq_codec of K */
   const int* v_codec;           /* host [n_layers][n_kv_heads] kvq_codec of V */
   int rot;                      /* kvq_rot */

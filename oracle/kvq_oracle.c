@@ -18,8 +18,9 @@
  *  [VBR]     "Introducing a new KV format: VBR (Variable Bit Rate)" (thread)
  *  [FORUM]   forum thread explaining decode attention and the memory-bandwidth
  *             bound (swe-vps threads?id=maurelius2)
- * Readings where the pages are silent are numbered R1..R18 and listed in the
- * repository's design document; each function below names the ones it uses.
+ * Where the pages are silent this file takes a reading, stated at the code that
+ * uses it and tagged R1, R2, ... so that one choice keeps one name wherever it
+ * recurs (the GPU side carries the same tags).
  *
  * Every function here is pinned by CPU tests against something other than
  * itself (closed forms, exhaustive comparisons with numpy's float16, worked
