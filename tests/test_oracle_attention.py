@@ -191,3 +191,21 @@ def test_quality_orderings_synthetic_analogue():
                                  inv_s_v=np.ones(128, np.float32))
     e_kvarn = np.linalg.norm(o_kvarn - exact) / np.linalg.norm(exact)
     assert e_kvarn < err(Q4_0, Q4_0, ROT_NONE)
+
+
+def test_packed_decode_equals_history_decode():
+    """decode_packed over the oracle's own encoding of the rows older than the tail,
+    plus the raw tail rows, is decode_head over the history (the composition the
+    prefill parity test uses for every causal prefix)."""
+    K, V, q = _hist(6, 300)
+    T = 64
+    out = oracle.decode_head(K, V, q, Q6_0, Q2_1, ROT_HADAMARD, tail=T)
+    ck, sk = oracle.encode_rows(Q6_0, ROT_HADAMARD, K[:-T])
+    cv, sv = oracle.encode_rows(Q2_1, ROT_HADAMARD, V[:-T])
+    got = oracle.decode_packed(ck, sk, cv, sv, K[-T:], V[-T:], q, Q6_0, Q2_1, ROT_HADAMARD)
+    assert np.array_equal(out, got)
+    # a causal prefix ending inside the tail: quantized rows + the first raw rows
+    lim = 300 - T + 10
+    pre = oracle.decode_packed(ck, sk, cv, sv, K[-T:lim], V[-T:lim], q, Q6_0, Q2_1, ROT_HADAMARD)
+    ref = oracle.decode_head(K[:lim], V[:lim], q, Q6_0, Q2_1, ROT_HADAMARD, tail=10)
+    assert np.array_equal(pre, ref)
