@@ -64,3 +64,21 @@ def test_debug_quantize_rejects_bad_row_layouts_before_any_launch(libkvq):
     fake = ctypes.c_void_p(16)
     assert f(kvq.RANK, 64, 2, 1, fake, fake, fake, kvq.ROWS_QUAD, None) == 2       # KVQ_ERR_UNSUPPORTED
     assert f(kvq.Q4_0, 128, 0, 1, fake, fake, fake, 7, None) == 1                  # KVQ_ERR_INVALID_ARG
+
+
+def _prototypes():
+    """name -> number of parameters, from the header's function prototypes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(kvq_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", text):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    from quantized_kv_cache_15_b200 import kvq
+    protos = _prototypes()
+    assert set(protos) == set(kvq.SIGNATURES)
+    bad = {n: (protos[n], len(kvq.SIGNATURES[n][1])) for n in protos if protos[n] != len(kvq.SIGNATURES[n][1])}
+    assert not bad, bad
