@@ -82,3 +82,23 @@ def test_binding_argument_counts_match_the_header():
     assert set(protos) == set(kvq.SIGNATURES)
     bad = {n: (protos[n], len(kvq.SIGNATURES[n][1])) for n in protos if protos[n] != len(kvq.SIGNATURES[n][1])}
     assert not bad, bad
+
+
+def test_host_argument_checks_run_before_any_device_call(libkvq):
+    """Descriptor and pointer checks return their status without touching a GPU."""
+    from quantized_kv_cache_15_b200 import kvq
+    import numpy as np
+    with pytest.raises(kvq.KVQError) as e:       # kv_dtype outside kvq_kv_dtype
+        kvq.Plan(1, 8, 2, max_seqs=1, max_tokens_per_seq=64, k_codec=[kvq.Q4_0] * 2, v_codec=[kvq.Q4_0] * 2,
+                 kv_dtype=5)
+    assert e.value.status == 1
+    with pytest.raises(kvq.KVQError) as e:       # tail not a multiple of 64
+        kvq.Plan(1, 8, 2, max_seqs=1, max_tokens_per_seq=64, k_codec=[kvq.Q4_0] * 2, v_codec=[kvq.Q4_0] * 2,
+                 tail_tokens=10)
+    assert e.value.status == 1
+    f = libkvq.kvq_prefill_attention
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert f(None, 0, 0, 1, None, None, None, 0, None) == 1           # null plan
+    assert np.int32(kvq.KV_BF16) == 1
