@@ -1,23 +1,34 @@
 #!/usr/bin/env python
 """Benchmark: decode attention + append-quantize over a quantized KV cache on B200.
 
-Workload (default): Llama-3.1-8B-shaped decode over an asymmetric cache -- 32
-layers, 32 query / 8 kv heads, head_dim 128, batch 1, context 32768, K q8_0 and
-V q4_0 after the Hadamard rotation; every step appends one token per layer and
-then runs decode attention for that layer.  Synthetic seeded data.
+Headline workload (default, --workload 5): batched serving under KVarN-style
+normalisation -- 64 sequences with ragged contexts of 1k..32k tokens, 32 layers,
+32 query / 8 kv heads, head_dim 128, variance normalisation + Hadamard-128 + q4_0
+for K and V, a 256-token F16 tail per sequence.  Every step appends a 2048-token
+chunk to 8 of the sequences (taken in rotation) and runs one decode query per
+sequence, layer by layer.  It is the largest of the five workloads that fits one
+GPU (about 41 GB of packed cache).  Synthetic seeded data.
 
-One step = for each layer: kvq_append_quantize (1 token) + kvq_decode_attention.
-  value : device time of one step, inputs resident in HBM (a CUDA graph of the
-          step's library launches, replayed; the packed cache read per step,
-          1.74 GB, is far larger than L2, so no flush is needed).
+One step = for each layer: kvq_append_quantize + kvq_decode_attention.
+  value : device time of one step per sequence (us/token), inputs resident in
+          HBM (a CUDA graph of the step's library launches, replayed; the packed
+          cache read per step is far larger than L2, so no flush is needed).
   e2e   : the same step through the public API, with the step's new K/V rows and
           queries copied from pinned host memory and the outputs copied back,
           inside the timed region.
+  roofline : the decode launch (the dominant kernel) against the measured HBM
+          copy rate; append_roofline: the chunk append likewise.
+  per_workload : the other four workloads (tiny; Llama-8B-shaped 32k; VBR mix with
+          a 1024-token tail; per-head rank/bits 128k), each with its step time,
+          decode roofline and chunk-append roofline, measured the same way (the
+          tiny workload's cache fits in L2, so L2 is flushed before each timed
+          call there).
 Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle instead.
 """
 from __future__ import annotations
 
 import argparse
+import glob
 import hashlib
 import json
 import os
@@ -39,6 +50,8 @@ W_NAMES = {0: "f16", 1: "q8_0", 2: "q6_0", 3: "q4_0", 4: "q3_0", 5: "q2_0", 6: "
            9: "q3_1", 10: "q2_1", 11: "rank", 12: "q5_0", 13: "q5_1"}
 METRIC = "decode-attn µs/token & HBM GB/s (% of 8 TB/s); append-quantize tokens/s, 1 B200"
 NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+HEADLINE = 5
 
 
 def parse():
@@ -50,8 +63,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs only)")
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5],
-                    help="which workload (default 2: the Llama-3.1-8B-shaped 32k decode)")
+    ap.add_argument("--workload", type=int, default=HEADLINE, choices=[1, 2, 3, 4, 5],
+                    help="headline workload (default 5: batch 64, KVarN q4_0, 256-token tail)")
+    ap.add_argument("--only", action="store_true", help="measure the headline workload only (no per_workload)")
     return ap.parse_args()
 
 
@@ -86,20 +100,68 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------- accounting
-def bytes_per_token_head(plan, layer, n_kv):
+def row_bytes(codec, r=128, b=0):
+    """Bytes of one packed row (codes + scales) in the documented format of
+    include/kvq.h: 16 b code bytes and 8 (_0) or 16 (_1) scale bytes per 128 values,
+    256 for F16, r b / 8 + 2 ceil(r / 32) for the rank codec."""
+    if codec == W.F16:
+        return 256
+    if codec == W.RANK:
+        return r * b // 8 + 2 * ((r + 31) // 32)
+    bits = {W.Q8_0: 8, W.Q8_1: 8, W.Q6_0: 6, W.Q6_1: 6, W.Q5_0: 5, W.Q5_1: 5, W.Q4_0: 4, W.Q4_1: 4,
+            W.Q3_0: 3, W.Q3_1: 3, W.Q2_0: 2, W.Q2_1: 2}[codec]
+    asym = codec in (W.Q8_1, W.Q6_1, W.Q5_1, W.Q4_1, W.Q3_1, W.Q2_1)
+    return 16 * bits + (16 if asym else 8)
+
+
+def token_head_bytes(w, layer):
+    """Packed bytes of one cached token of one layer, over all kv heads, K and V."""
     tot = 0
-    for h in range(n_kv):
-        for kv in (0, 1):
-            cb, sb = plan.row_bytes(layer, h, kv)
-            tot += cb + sb
+    for h in range(w.n_kv_heads):
+        r = w.rank[layer][h] if w.rank else 128
+        kb = w.k_bits[layer][h] if w.k_bits else 0
+        vb = w.v_bits[layer][h] if w.v_bits else 0
+        tot += row_bytes(w.k_codec[layer][h], r, kb) + row_bytes(w.v_codec[layer][h], r, vb)
     return tot
 
 
-def decode_algorithmic_bytes(plan, w, layer, length):
-    """Bytes one decode launch must move: the packed cache (codes + scales of every
-    cached token of every kv head), the fp16 queries and the fp32 outputs."""
-    cache = bytes_per_token_head(plan, layer, w.n_kv_heads) * length
-    return cache + w.n_q_heads * 128 * 2 + w.n_q_heads * 128 * 4
+def decode_bytes(w, layer, lengths):
+    """Algorithmic bytes of one decode launch: every cached token's packed rows (raw
+    rows for the tail), the fp16 queries and the fp32 outputs."""
+    tot = 0
+    bpt = token_head_bytes(w, layer)
+    for n in lengths:
+        nq = max(0, n - w.tail)
+        tot += nq * bpt + (n - nq) * w.n_kv_heads * 2 * 128 * 2
+    return tot + len(lengths) * w.n_q_heads * 128 * (2 + 4)
+
+
+def append_bytes(w, layer, len_old, n):
+    """Algorithmic bytes of appending n tokens to a sequence of len_old tokens in one
+    layer: raw input rows read; rows leaving the tail read from the ring; quantized
+    rows written; rows entering the tail written (K and V, every kv head)."""
+    raw = w.n_kv_heads * 2 * 128 * 2
+    T = w.tail
+    if T == 0:
+        return n * raw + n * token_head_bytes(w, layer)
+    e0, e1 = max(0, len_old - T), min(len_old, len_old + n - T)
+    nE = max(0, e1 - e0)
+    nP = max(0, len_old + n - T - len_old) if n > T else 0
+    nF = min(n, T)
+    return n * raw + nE * raw + (nE + nP) * token_head_bytes(w, layer) + nF * raw
+
+
+def step_cache_bytes(w):
+    return sum(decode_bytes(w, l, w.ctx) for l in range(w.n_layers))
+
+
+def l2_note(w):
+    """How the timed steps avoid L2 hits, from the workload alone (same text in both arms)."""
+    b = step_cache_bytes(w)
+    if b < 4 * L2_BYTES:
+        return (f"L2 flushed before every timed call (a 512 MB write): the step reads only {b / 1e6:.2f} MB "
+                f"of packed cache")
+    return f"no flush: the step reads {b / 1e9:.2f} GB of packed cache, far more than L2 (126 MB)"
 
 
 DECODE_SOURCES = ("decode.cu", "decode_fast.cuh", "kvq_internal.h", "ptx.cuh", "quant.cuh")
@@ -114,22 +176,20 @@ def kernel_source_sha256():
 
 
 def traffic_from_profile(workload):
-    """dram bytes per decode launch recorded in profiles/decode_attention_llama8b.md,
-    if that capture is of this workload and the kernel source still matches the one
-    profiled (else None)."""
-    path = os.path.join(ROOT, "profiles", "decode_attention_llama8b.md")
-    try:
+    """DRAM bytes per decode launch recorded under profiles/ for this workload (a
+    block "profiled_workload / traffic_bytes_per_launch / kernel_source_sha256"),
+    only while the decode kernel's source still matches the one profiled; else None."""
+    sha = None
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         text = open(path).read()
-    except OSError:
-        return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
-    wl = re.search(r"profiled_workload:\s*(\S+)", text)
-    if not m or not h or not wl or wl.group(1) != workload:
-        return None
-    if kernel_source_sha256() != h.group(1):
-        return None
-    return float(m.group(1))
+        for m in re.finditer(r"profiled_workload:\s*(\S+)\s*\ntraffic_bytes_per_launch:\s*([0-9.eE+]+)\s*\n"
+                             r"kernel_source_sha256:\s*([0-9a-f]{64})", text):
+            if m.group(1) != workload:
+                continue
+            sha = sha or kernel_source_sha256()
+            if m.group(3) == sha:
+                return float(m.group(2))
+    return None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -249,7 +309,7 @@ def cpu_oracle_decode_us_per_token(w, seconds, log, max_pairs=None, threads=None
 
 
 # ----------------------------------------------------------------------------- reference arm
-def workload_config(w, layers, world, l2):
+def workload_config(w, layers, world):
     """The `config` object of both arms' JSON lines for workload w."""
     B = w.batch
     n_app = w.append_tokens if w.append_tokens else 1
@@ -260,7 +320,7 @@ def workload_config(w, layers, world, l2):
             "tail": w.tail, "codecs_k_v": codecs,
             "rotation": ["none", "hadamard-128", "varnorm+hadamard-128", "per-head projection"][w.rot],
             "step": f"per layer: append {n_app} token(s) x {n_app_seqs} seq(s) + decode attention for {B} seq(s)",
-            "parallelism": f"replicas x{world}", "l2": l2}
+            "parallelism": f"replicas x{world}", "l2": l2_note(w)}
 
 
 def run_reference(args, world, rank):
@@ -277,9 +337,9 @@ def run_reference(args, world, rank):
             vals.append(cb["value"])
     v = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "us/token", "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1000.0, "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, w.n_layers, world, "n/a: the oracle runs on the host cores"),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * w.batch / 1000.0,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, w.n_layers, world),
             "cpu_baseline": {"value": v, "unit": "us/token", "cores": threads, "kind": "oracle",
                              "sample": f"each step: oracle decode of {threads} (layer, kv head) pairs of sequence 0 "
                                        f"over its full context on {threads} host threads at once, scaled to every "
@@ -310,25 +370,52 @@ def make_plan(kvq, w, extra, dev):
                     k_codec=w.k_codec, v_codec=w.v_codec, rot=w.rot, tail_tokens=w.tail, max_pages=pages, **kw)
 
 
-def run_kvq(args, world, rank, local):
-    from quantized_kv_cache_15_b200 import kvq
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    log = (lambda m: print(m, file=sys.stderr, flush=True)) if rank == 0 else (lambda m: None)
-    w = W.make_workload(args.workload, "full")
-    if args.layers:
-        w.n_layers = args.layers
-        for f in ("k_codec", "v_codec", "rank", "k_bits", "v_bits"):
-            if getattr(w, f) is not None:
-                setattr(w, f, getattr(w, f)[:args.layers])
-    L, Hq, Hkv, B = w.n_layers, w.n_q_heads, w.n_kv_heads, w.batch
-    K, Wm = args.steps, args.warmup
-    # appends per step: one token per layer for every sequence, or (serving workload)
-    # a chunk for `append_seqs` sequences taken in rotation
+class L2Flush:
+    """Writes a buffer larger than L2 on `stream` (for workloads whose cache fits in L2)."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.v = 0
+
+    def __call__(self):
+        self.v = (self.v + 1) & 0xFF
+        self.buf.fill_(self.v)
+
+
+def timed_replays(graph, stream, reps, flush=None):
+    """Mean ms of one replay of `graph`, timed with events on `stream` (the graph's
+    launches run there).  With `flush`, L2 is flushed before each replay and only the
+    replay is timed."""
+    with torch.cuda.stream(stream):
+        if flush is None:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            b.record(stream)
+            stream.synchronize()
+            return a.elapsed_time(b) / reps
+        tot = 0.0
+        for _ in range(reps):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+            stream.synchronize()
+            tot += a.elapsed_time(b)
+        return tot / reps
+
+
+def measure_workload(kvq, w, dev, K, Wm, world, log, headline):
+    """Fill w's cache and measure its step, decode launch and chunk append; the
+    headline workload also gets the e2e step, the clocks, a prefill call and a VBR
+    regrade.  Frees its device memory before returning."""
+    L, Hq, B = w.n_layers, w.n_q_heads, w.batch
     n_app = w.append_tokens if w.append_tokens else 1
     n_app_seqs = w.append_seqs if w.append_seqs else B
     n_groups = max(1, B // n_app_seqs)
-    host_steps = Wm + 1 + K                              # warm-up, captured, e2e steps advance host lengths
+    host_steps = Wm + 1 + (K if headline else 0)     # warm-up, captured and e2e steps advance host lengths
     growth = ((host_steps + n_groups - 1) // n_groups) * n_app + 2 * 2048 + 64
     plan = make_plan(kvq, w, growth, dev)
     plan.allocate_cache(dev)
@@ -341,12 +428,13 @@ def run_kvq(args, world, rank, local):
                 plan.append(l, [s], [b - a], w.rows("K", l, s, a, b, dev), w.rows("V", l, s, a, b, dev))
     torch.cuda.synchronize()
     plan.check_device_error()
-    log(f"filled {L} layers x {sum(w.ctx)} tokens in {time.time() - t0:.1f} s; cache {plan.cache_bytes() / 1e9:.2f} GB")
+    log(f"[{w.name}] filled {L} layers x {sum(w.ctx)} tokens in {time.time() - t0:.1f} s; "
+        f"cache {plan.cache_bytes() / 1e9:.2f} GB")
+    flush = L2Flush(dev) if step_cache_bytes(w) < 4 * L2_BYTES else None
 
     stream = torch.cuda.Stream(dev)
     ws = plan.new_workspace(B, dev)
     seqs = list(range(B))
-    # new rows of one step (same values every step; positions advance) and queries
     knew = torch.stack([torch.cat([w.rows("K", l, s, w.ctx[s], w.ctx[s] + n_app, dev) for s in range(n_app_seqs)])
                         for l in range(L)])
     vnew = torch.stack([torch.cat([w.rows("V", l, s, w.ctx[s], w.ctx[s] + n_app, dev) for s in range(n_app_seqs)])
@@ -377,6 +465,7 @@ def run_kvq(args, world, rank, local):
     # capture one step (fixed positions; every replay does the full step's work)
     lengths = [[plan.seq_length(s, l) for s in seqs] for l in range(L)]
     grp = app_group()
+    old_len = [[lengths[l][s] for s in seqs] for l in range(L)]
     for l in range(L):
         for s in grp:
             lengths[l][s] += n_app
@@ -385,8 +474,6 @@ def run_kvq(args, world, rank, local):
     with torch.cuda.graph(g, stream=stream):
         step()
     launches_per_step = kvq.launch_count() - n0
-    # CUDAGraph.replay() launches on the current stream: replay on `stream`, where the
-    # timing events are recorded
     with torch.cuda.stream(stream):
         for _ in range(Wm):
             g.replay()
@@ -394,68 +481,70 @@ def run_kvq(args, world, rank, local):
 
     # ---- timed region: device time of K steps
     barrier = (lambda: torch.distributed.barrier()) if world > 1 else (lambda: None)
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = None
+    if headline:
+        clocks = ClockSampler(dev.index or 0)
+        clocks.start()
+        time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(K):
-            g.replay()
-        e1.record(stream)
+    step_ms = timed_replays(g, stream, K, flush)
     torch.cuda.synchronize()
     barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    clk = clocks.stop()
-    step_ms = ms / K
+    step_ms = max_over_ranks(step_ms, world, dev)
+    clk = clocks.stop() if clocks else None
     plan.check_device_error(stream)
 
     # ---- per-launch decode durations: a CUDA graph of the step's L decode calls
-    # (back to back, every layer's cache read once: far more than L2), replayed
-    # between two events on the launching stream; duration = elapsed / L
+    # (back to back; every layer's cache read once), replayed between two events on
+    # the launching stream; duration = elapsed / L
     gd = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gd, stream=stream):
         for l in range(L):
             plan.decode(l, seqs, qall[l], out[l], ws, stream)
-    dec_reps = max(3, K // 4)
     with torch.cuda.stream(stream):
         for _ in range(2):
             gd.replay()
     stream.synchronize()
-    da, db = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        da.record(stream)
-        for _ in range(dec_reps):
-            gd.replay()
-        db.record(stream)
-    stream.synchronize()
-    dec_ms = max_over_ranks(da.elapsed_time(db) / (dec_reps * L), world, dev)
+    dec_ms = max_over_ranks(timed_replays(gd, stream, max(3, K // 4), flush) / L, world, dev)
     plan.check_device_error(stream)
+    dec_bytes_all = [decode_bytes(w, l, lengths[l]) for l in range(L)]
+    dec_bytes = statistics.mean(dec_bytes_all)
+
+    res = {"workload": w.name, "ms_per_step": step_ms, "us_per_token": step_ms * 1e3 / B,
+           "gpu_launches_per_step": launches_per_step, "l2": l2_note(w)}
 
     # ---- e2e through the public API: host buffers in, host buffers out
-    kh, vh, qh = knew.cpu().pin_memory(), vnew.cpu().pin_memory(), qall.cpu().pin_memory()
-    oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    kd, vd, qd = torch.empty_like(knew), torch.empty_like(vnew), torch.empty_like(qall)
-    h2d = (kd.numel() + vd.numel() + qd.numel()) * 2
-    d2h = oh.numel() * 4
-    e2e_ms = []
-    for s in range(K):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        a.record(stream)
-        with torch.cuda.stream(stream):
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            qd.copy_(qh, non_blocking=True)
-            step(kd, vd, qd)
-            oh.copy_(out, non_blocking=True)
-        b.record(stream)
-        stream.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    e2e_step = max_over_ranks(statistics.mean(e2e_ms), world, dev)
-    plan.check_device_error(stream)
+    if headline:
+        kh, vh, qh = knew.cpu().pin_memory(), vnew.cpu().pin_memory(), qall.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        kd, vd, qd = torch.empty_like(knew), torch.empty_like(vnew), torch.empty_like(qall)
+        h2d = (kd.numel() + vd.numel() + qd.numel()) * 2
+        d2h = oh.numel() * 4
+        e2e_ms = []
+        for _ in range(K):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            a.record(stream)
+            with torch.cuda.stream(stream):
+                kd.copy_(kh, non_blocking=True)
+                vd.copy_(vh, non_blocking=True)
+                qd.copy_(qh, non_blocking=True)
+                step(kd, vd, qd)
+                oh.copy_(out, non_blocking=True)
+            b.record(stream)
+            stream.synchronize()
+            e2e_ms.append(a.elapsed_time(b))
+        e2e_step = max_over_ranks(statistics.mean(e2e_ms), world, dev)
+        plan.check_device_error(stream)
+        res["e2e"] = {"value": e2e_step * 1e3 / (B * world), "unit": "us/token", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h}
+        del kd, vd, qd, kh, vh, qh, oh
+
+    # ---- step accounting
+    app_step_bytes = sum(append_bytes(w, l, old_len[l][s], n_app) for l in range(L) for s in grp)
+    step_bytes = sum(dec_bytes_all) + app_step_bytes
+    res["step_gb_s"] = step_bytes / (step_ms / 1e3) / 1e9
 
     # ---- append-quantize throughput: a 2048-token chunk into every layer of sequence 0
     ck = torch.stack([w.rows("K", l, 0, 0, 2048, dev) for l in range(L)])
@@ -464,130 +553,153 @@ def run_kvq(args, world, rank, local):
         for l in range(L):
             plan.append(l, [0], [2048], ck[l], cv[l], stream)   # warm: allocates the chunk's pages
     stream.synchronize()
+    len0 = [plan.seq_length(0, l) for l in range(L)]
     ga = torch.cuda.CUDAGraph()
     with torch.cuda.graph(ga, stream=stream):
         for l in range(L):
             plan.append(l, [0], [2048], ck[l], cv[l], stream)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 10
     with torch.cuda.stream(stream):
         for _ in range(3):
             ga.replay()
-        a.record(stream)
-        for _ in range(reps):
-            ga.replay()
-        b.record(stream)
     stream.synchronize()
-    app_ms = a.elapsed_time(b) / reps
-    append_tps = 2048 / (app_ms / 1e3)
-    app_bytes = sum(2048 * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, l, Hkv)) for l in range(L))
+    app_ms = timed_replays(ga, stream, 10)
     plan.check_device_error(stream)
+    app_b = sum(append_bytes(w, l, len0[l], 2048) for l in range(L))
+    res["append_tokens_per_s"] = 2048 / (app_ms / 1e3)
+    res["append_roofline"] = {"bound": "hbm", "kernel": "kvq_append_quantize (2048 tokens, one layer)",
+                              "bytes_per_launch": app_b / L, "launch_ms": app_ms / L,
+                              "achieved": app_b / (app_ms / 1e3) / 1e9, "unit": "GB/s",
+                              "note": "raw rows read (input and ring) + packed rows and ring rows written"}
+    res["decode"] = {"bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
+                     "achieved": dec_bytes / (dec_ms / 1e3) / 1e9, "kernel": f"decode_kernel<{w.G}>",
+                     "traffic": traffic_from_profile(w.name)}
+    del ck, cv, ga
 
-    # ---- accounting (algorithmic bytes of the captured step's decode launches)
-    def layer_decode_bytes(l):
-        tot = 0
-        bpt = bytes_per_token_head(plan, l, Hkv)
-        for s in seqs:
-            n = lengths[l][s]
-            nq = max(0, n - w.tail)
-            nt = n - nq
-            tot += nq * bpt + nt * Hkv * 2 * 128 * 2
-        return tot + B * Hq * 128 * (2 + 4)
+    if headline:
+        res["clocks"] = clk
+        # ---- chunked-prefill attention: the newest (up to) 2048 tokens of the longest
+        # sequence in layer 0 attend causally to the cache (one kvq_prefill_attention call)
+        ps = max(seqs, key=lambda s: plan.seq_length(s, 0))
+        p_len = plan.seq_length(ps, 0)
+        n_pq = min(2048, p_len)
+        pq = torch.stack([w.queries(0, ps, i, dev) for i in range(n_pq)]).contiguous()
+        pout = torch.empty((n_pq, Hq, 128), dtype=torch.float32, device=dev)
+        pws = plan.new_workspace(min(n_pq, 256))
+        pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            plan.prefill(0, ps, pq, pout, pws, stream)                      # warm-up
+            pa.record(stream)
+            for _ in range(2):
+                plan.prefill(0, ps, pq, pout, pws, stream)
+            pb.record(stream)
+        stream.synchronize()
+        plan.check_device_error(stream)
+        p_ms = pa.elapsed_time(pb) / 2
+        res["prefill"] = {"layer": 0, "seq": int(ps), "queries": n_pq, "context": int(p_len), "ms": p_ms,
+                          "tokens_per_s": n_pq / (p_ms / 1e3),
+                          "note": "causal: query i sees the first len - n_q + i + 1 tokens"}
+        del pws, pq, pout
+        # ---- VBR regrade of one layer (last, since it changes that layer's codecs)
+        res["regrade"] = None
+        if w.rot != W.ROT_PROJECTION:
+            rl = L // 2
+            Hkv = w.n_kv_heads
+            nk, nv = [W.Q4_0] * Hkv, [W.Q2_0] * Hkv
+            try:
+                rbytes = plan.regrade_bytes(rl, nk, nv)
+            except kvq.KVQError:
+                rbytes = None
+            if rbytes:
+                rows = sum(max(0, plan.seq_length(s, rl) - w.tail) for s in seqs)
+                old_b = rows * token_head_bytes(w, rl)
+                scratch = torch.empty(rbytes, dtype=torch.uint8, device=dev)
+                ra, rb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    ra.record(stream)
+                    plan.regrade(rl, nk, nv, scratch, stream)
+                    rb.record(stream)
+                stream.synchronize()
+                plan.check_device_error(stream)
+                new_b = rows * Hkv * (row_bytes(W.Q4_0) + row_bytes(W.Q2_0))
+                r_ms = ra.elapsed_time(rb)
+                res["regrade"] = {"layer": rl, "ms": r_ms, "rows": rows * Hkv, "to": ["q4_0", "q2_0"],
+                                  "gb_s": (old_b + new_b) / (r_ms / 1e3) / 1e9,
+                                  "note": "bytes = old rows read + new rows written"}
+                del scratch
+    del g, gd
+    del plan, ws, knew, vnew, qall, out
+    if flush is not None:
+        del flush
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
-    dec_bytes_all = [layer_decode_bytes(l) for l in range(L)]
-    dec_bytes = statistics.mean(dec_bytes_all)
 
-    app_step_bytes = sum(n_app * n_app_seqs * (Hkv * 2 * 128 * 2 + bytes_per_token_head(plan, l, Hkv)) for l in range(L))
-    step_bytes = sum(dec_bytes_all) + app_step_bytes
-    # ---- chunked-prefill attention: the newest (up to) 2048 tokens of the longest
-    # sequence in layer 0 attend causally to the cache (one kvq_prefill_attention call)
-    ps = max(seqs, key=lambda s: plan.seq_length(s, 0))
-    p_len = plan.seq_length(ps, 0)
-    n_pq = min(2048, p_len)
-    pq = torch.stack([w.queries(0, ps, i, dev) for i in range(n_pq)]).contiguous()
-    pout = torch.empty((n_pq, Hq, 128), dtype=torch.float32, device=dev)
-    pws = plan.new_workspace(min(n_pq, 256))
-    pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        plan.prefill(0, ps, pq, pout, pws, stream)                      # warm-up
-        pa.record(stream)
-        for _ in range(2):
-            plan.prefill(0, ps, pq, pout, pws, stream)
-        pb.record(stream)
-    stream.synchronize()
-    plan.check_device_error(stream)
-    p_ms = pa.elapsed_time(pb) / 2
-    prefill = {"layer": 0, "seq": int(ps), "queries": n_pq, "context": int(p_len), "ms": p_ms,
-               "tokens_per_s": n_pq / (p_ms / 1e3),
-               "note": "causal: query i sees the first len - n_q + i + 1 tokens; each query runs the split-K "
-                       "decode kernel over its prefix (256 queries per launch)"}
-    del pws, pq, pout
+def roofline(d, peak, peaks):
+    return {"bound": "hbm", "achieved": d["achieved"], "peak": peak, "unit": "GB/s", "frac": d["achieved"] / peak,
+            "traffic": d.get("traffic"), "kernel": d.get("kernel"), "bytes_per_launch": d["bytes_per_launch"],
+            "launch_ms": d["launch_ms"],
+            "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, burst), of measured" if peaks
+            else "fallback 6650 GB/s"}
 
-    # ---- VBR regrade of one layer (last, since it changes that layer's codecs):
-    # K to q4_0 and V to q2_0 where that does not grow the pages
-    regrade = None
-    if w.rot != W.ROT_PROJECTION:
-        rl = L // 2
-        nk, nv = [W.Q4_0] * Hkv, [W.Q2_0] * Hkv
-        try:
-            rbytes = plan.regrade_bytes(rl, nk, nv)
-        except kvq.KVQError:
-            rbytes = None
-        if rbytes:
-            rows = sum(max(0, lengths[rl][s] - w.tail) for s in seqs) * Hkv
-            old_b = rows * bytes_per_token_head(plan, rl, Hkv) / Hkv
-            scratch = torch.empty(rbytes, dtype=torch.uint8, device=dev)
-            ra, rb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            with torch.cuda.stream(stream):
-                ra.record(stream)
-                plan.regrade(rl, nk, nv, scratch, stream)
-                rb.record(stream)
-            stream.synchronize()
-            plan.check_device_error(stream)
-            new_b = rows * bytes_per_token_head(plan, rl, Hkv) / Hkv
-            r_ms = ra.elapsed_time(rb)
-            moved = old_b + new_b + 2 * rbytes                 # read old rows, write scratch, copy back
-            regrade = {"layer": rl, "ms": r_ms, "rows": rows, "to": ["q4_0", "q2_0"],
-                       "gb_s": moved / (r_ms / 1e3) / 1e9,
-                       "note": "kernel + copy-back of the whole layer pool; bytes = old rows read + new rows "
-                               "written + scratch copied back"}
+
+def run_kvq(args, world, rank, local):
+    from quantized_kv_cache_15_b200 import kvq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    log = (lambda m: print(m, file=sys.stderr, flush=True)) if rank == 0 else (lambda m: None)
+
+    def load(cfg):
+        w = W.make_workload(cfg, "full")
+        if args.layers:
+            w.n_layers = args.layers
+            for f in ("k_codec", "v_codec", "rank", "k_bits", "v_bits"):
+                if getattr(w, f) is not None:
+                    setattr(w, f, getattr(w, f)[:args.layers])
+        return w
 
     peaks = measured_peaks()
     peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
-    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
-    traffic = traffic_from_profile(w.name)
-    hbm_gbs = step_bytes / (step_ms / 1e3) / 1e9
-    us_per_token = step_ms * 1e3 / (B * world)
+    w = load(args.workload)
+    K, Wm = args.steps, args.warmup
+    h = measure_workload(kvq, w, dev, K, Wm, world, log, headline=True)
+    step_ms = h["ms_per_step"]
     line = {
-        "metric": METRIC, "value": us_per_token, "unit": "us/token", "n_gpus": world, "steps": K, "warmup": Wm,
-        "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, L, world, "no flush: packed cache read per step (%.2f GB) >> L2 (126 MB)"
-                                  % (sum(dec_bytes_all) / 1e9)),
+        "metric": METRIC, "value": step_ms * 1e3 / (w.batch * world), "unit": "us/token", "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": step_ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, w.n_layers, world),
         "us_per_step": step_ms * 1e3,
-        "hbm_gbs": hbm_gbs, "hbm_frac_of_8tbs": hbm_gbs / NOMINAL_HBM_GBS,
-        "hbm_frac_of_measured": hbm_gbs / peak,
-        "append_tokens_per_s": append_tps,
-        "append_note": f"2048-token chunk appended to all {L} layers (K and V quantized): {app_ms:.3f} ms, "
-                       f"{app_bytes / (app_ms / 1e3) / 1e9:.0f} GB/s algorithmic",
-        "regrade": regrade,
-        "prefill": prefill,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": f"decode_kernel<{w.G}>",
-                     "bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
-                     "peak_source": "MEASURED_PEAKS.json hbm_gbs (copy, burst), of measured" if peaks
-                     else "fallback 6650 GB/s"},
-        "e2e": {"value": e2e_step * 1e3 / (B * world), "unit": "us/token", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * K,
-        "clocks": clk,
+        "hbm_gbs": h["step_gb_s"], "hbm_frac_of_8tbs": h["step_gb_s"] / NOMINAL_HBM_GBS,
+        "hbm_frac_of_measured": h["step_gb_s"] / peak,
+        "append_tokens_per_s": h["append_tokens_per_s"],
+        "append_roofline": dict(h["append_roofline"], peak=peak, frac=h["append_roofline"]["achieved"] / peak),
+        "regrade": h.get("regrade"),
+        "prefill": h.get("prefill"),
+        "roofline": roofline(h["decode"], peak, peaks),
+        "e2e": h["e2e"],
+        "gpu_launches": h["gpu_launches_per_step"] * K,
+        "clocks": h["clocks"],
     }
+    if not args.only:
+        per = {}
+        for cfg in (1, 2, 3, 4, 5):
+            if cfg == args.workload:
+                continue
+            wc = load(cfg)
+            r = measure_workload(kvq, wc, dev, min(K, 10), max(3, min(Wm, 3)), world, log, headline=False)
+            per[str(cfg)] = {"workload": r["workload"], "ms_per_step": r["ms_per_step"],
+                             "us_per_token": r["us_per_token"], "step_gb_s": r["step_gb_s"], "l2": r["l2"],
+                             "roofline": roofline(r["decode"], peak, peaks),
+                             "append_tokens_per_s": r["append_tokens_per_s"],
+                             "append_roofline": dict(r["append_roofline"], peak=peak,
+                                                     frac=r["append_roofline"]["achieved"] / peak)}
+        line["per_workload"] = per
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ncpu = os.cpu_count() or 1
         line["cpu_baseline"] = cpu_oracle_decode_us_per_token(w, args.cpu_seconds, log, max_pairs=ncpu, threads=ncpu)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g, ga
     return 0
 
 

@@ -347,6 +347,24 @@ kvq_status kvq_debug_rotate(const kvq_plan* plan, int layer, int head, int kv, i
 kvq_status kvq_debug_quantize_f32(int codec, int r, int b, int n_rows, const float* y, void* codes,
                                   void* scales, int layout, void* stream);
 
+/* Fixed split-K size for this plan's decode and prefill calls (test-only; no
+ * counterpart in the pages): pages_per_split > 0 cuts every sequence into splits of
+ * that many pages (at least as many as the split limit needs); 0 restores the
+ * automatic choice.  The merge order is fixed either way, so results differ only
+ * by the rounding of the merge.  KVQ_ERR_INVALID_ARG for a negative count. */
+kvq_status kvq_debug_set_decode_split(kvq_plan* plan, int pages_per_split);
+
+/* Failure injection for the failure-path tests (test-only; no counterpart in the
+ * pages).  wait_limit_ns: every bounded wait inside this plan's decode kernels
+ * gives up after this long (default 2e9; accepted range [1e3, 2e9]) and latches
+ * KVQ_ERR_TIMEOUT in the plan's error word.  drop_last_tile = 1 makes every decode
+ * CTA's producer skip loading its last tile, so the consumer waiting for it runs
+ * out its wait, finishes the launch on stale shared memory (the output of that
+ * call is garbage) and the next kvq_check_device_error() returns KVQ_ERR_TIMEOUT;
+ * the context stays usable.  No bulk copy is left in flight: the skipped tile is
+ * the last use of its stage.  (2e9, 0) restores normal operation. */
+kvq_status kvq_debug_fault_injection(kvq_plan* plan, int64_t wait_limit_ns, int drop_last_tile);
+
 #ifdef __cplusplus
 }
 #endif

@@ -82,6 +82,10 @@ struct kvq_plan {
   std::vector<int> bt;                // host mirror of the block table
   std::vector<int> npages;            // pages held per sequence
   std::vector<int> free_pages;        // stack of free page ids
+  // test-only settings (kvq_debug_set_decode_split, kvq_debug_fault_injection)
+  int debug_pps = 0;                          // fixed pages per split, 0 = chosen per call
+  unsigned long long wait_ns = 2000000000ull; // give-up time of the kernels' bounded waits
+  int drop_last_tile = 0;                     // decode producers skip their last tile
 
   ~kvq_plan() {
     int prev = 0;
@@ -117,6 +121,8 @@ struct kvq_plan {
     p.M = d_M;
     p.qscale = scale * 1.4426950408889634f;
     p.err = d_err;
+    p.wait_ns = wait_ns;
+    p.drop_last_tile = drop_last_tile;
     for (int h = 0; h < Hkv; ++h) p.heads[h] = head(layer, h);
     return p;
   }
@@ -481,19 +487,28 @@ kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* se
 
 }  // extern "C"
 
-// One decode launch over n_seqs entries; entry i attends sequence seq_ids[i] over
-// its first lims[i] tokens (all of them when lims is null).
-static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* lims,
-                                const void* q, float* out, void* workspace, size_t workspace_bytes_given,
-                                void* stream) {
+// A validated decode launch: parameters, grid and whether it uses the workspace.
+struct DecodeLaunch {
+  DecodeParams dp;
+  int grid_x = 1;
+  bool uses_ws = false;     // split-K partials / merge counters / projected queries live in the workspace
+  bool proj = false;        // the projected-query kernel runs first
+};
+
+// Validate one decode launch over n_seqs entries (entry i attends sequence
+// seq_ids[i] over its first lims[i] tokens, all of them when lims is null) and
+// size it.  Nothing is enqueued; on failure the plan is unchanged.
+static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* lims,
+                                 const void* q, float* out, void* workspace, size_t workspace_bytes_given,
+                                 DecodeLaunch& L) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
-  if (n_seqs == 0) return KVQ_OK;
-  if (!seq_ids || !q || !out) return fail(KVQ_ERR_INVALID_ARG, "null seq_ids, q or out");
+  if (n_seqs > 0 && (!seq_ids || !q || !out)) return fail(KVQ_ERR_INVALID_ARG, "null seq_ids, q or out");
   if (((uintptr_t)q % 16) || ((uintptr_t)out % 16)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
-  DecodeParams dp = p->base_params(layer);
+  DecodeParams& dp = L.dp;
+  dp = p->base_params(layer);
   dp.q = (const __half*)q;
   dp.out = out;
   dp.n_seqs = n_seqs;
@@ -513,6 +528,10 @@ static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* s
     work += (int64_t)pages * p->Hkv;
     maxpages = std::max(maxpages, pages);
   }
+  L.grid_x = 1;
+  L.uses_ws = false;
+  L.proj = p->rot == KVQ_ROT_PROJECTION;
+  if (n_seqs == 0) return KVQ_OK;
   dp.stage_bytes = p->stage_bytes[layer];
   // The consumer warps keep their weight tables in the K region of their current
   // stage unless some head's (or the tail's) K rows are smaller than a table.
@@ -555,18 +574,13 @@ static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* s
     const int64_t m = makespan(cand);
     if (m < best) { best = m; pps = cand; }
   }
-  if (const char* env = std::getenv("KVQ_DECODE_PAGES_PER_SPLIT")) {   // fixed split size (tests, tuning)
-    const int v = std::atoi(env);
-    if (v > 0) pps = std::max(v, min_pps);
-  }
+  if (p->debug_pps > 0) pps = std::max(p->debug_pps, min_pps);   // fixed split size (tests)
   dp.pps = pps;
-  int grid_x = 1;
   for (int i = 0; i < n_seqs; ++i) {
     const SplitCounts c = split_counts(dp.len[i], (int)p->T, pps, dp.lim[i]);
-    grid_x = std::max(grid_x, c.qsplits + c.tsplits);
+    L.grid_x = std::max(L.grid_x, c.qsplits + c.tsplits);
   }
-  const bool proj = p->rot == KVQ_ROT_PROJECTION;
-  if (grid_x > 1 || proj) {
+  if (L.grid_x > 1 || L.proj) {
     const size_t need = workspace_bytes(p, n_seqs);
     if (!workspace || workspace_bytes_given < need)
       return fail(KVQ_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes_given);
@@ -574,14 +588,29 @@ static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* s
     dp.tickets = (int*)workspace;
     dp.ws = (float*)((char*)workspace + ticket_bytes(p));
     dp.qproj = (float*)((char*)workspace + ticket_bytes(p) + partial_bytes(p, n_seqs));
+    L.uses_ws = true;
   }
-  if (proj) {
-    cudaError_t e = launch_project_query(dp, (cudaStream_t)stream);
+  return KVQ_OK;
+}
+
+static kvq_status decode_enqueue(const DecodeLaunch& L, void* stream) {
+  if (L.dp.n_seqs == 0) return KVQ_OK;
+  if (L.proj) {
+    cudaError_t e = launch_project_query(L.dp, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "query projection launch");
   }
-  cudaError_t e = launch_decode(dp, grid_x, (cudaStream_t)stream);
+  cudaError_t e = launch_decode(L.dp, L.grid_x, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return KVQ_OK;
+}
+
+static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* lims,
+                                const void* q, float* out, void* workspace, size_t workspace_bytes_given,
+                                void* stream) {
+  DecodeLaunch L;
+  const kvq_status st = decode_prepare(p, layer, n_seqs, seq_ids, lims, q, out, workspace, workspace_bytes_given, L);
+  if (st != KVQ_OK) return st;
+  return decode_enqueue(L, stream);
 }
 
 extern "C" {
@@ -619,20 +648,30 @@ kvq_status kvq_decode_attention_noalloc(kvq_plan* p, int layer, int n_seqs, cons
                                         float* out, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
   if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
+  // the scratch array is looked up on the current device: it must be the plan's
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != p->device)
+    return fail(KVQ_ERR_STATE, "current device %d is not the plan's device %d", dev, p->device);
   const size_t need = workspace_bytes(p, n_seqs);
   if (need > NOALLOC_SCRATCH_BYTES)
     return fail(KVQ_ERR_CAPACITY, "decode of %d sequences needs %zu bytes of scratch; the built-in array holds %zu "
                 "(use kvq_decode_attention with a workspace)", n_seqs, need, NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
-  cudaError_t e = noalloc_scratch(&scratch);
+  e = noalloc_scratch(p->device, &scratch);
   if (e != cudaSuccess) return cuda_fail(e, "scratch address lookup");
+  // every argument is checked before anything is enqueued
+  DecodeLaunch L;
+  const kvq_status st = decode_prepare(p, layer, n_seqs, seq_ids, nullptr, q, out, scratch, NOALLOC_SCRATCH_BYTES, L);
+  if (st != KVQ_OK) return st;
   // merge counters must start at zero (partials are written before they are read)
   const size_t tickets = (size_t)n_seqs * p->Hkv * sizeof(int);
-  if (tickets) {
+  if (L.uses_ws && tickets) {
     e = cudaMemsetAsync(scratch, 0, tickets, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "scratch counter reset");
   }
-  return kvq_decode_attention(p, layer, n_seqs, seq_ids, q, out, scratch, NOALLOC_SCRATCH_BYTES, stream);
+  return decode_enqueue(L, stream);
 }
 
 kvq_status kvq_dequantize(const kvq_plan* p, int layer, int seq_id, int64_t t0, int64_t t1, float* k_out,
@@ -841,6 +880,23 @@ kvq_status kvq_check_device_error(kvq_plan* p, void* stream) {
   cudaMemset(p->d_err, 0, sizeof(int));
   if (v & ERR_TIMEOUT) return fail(KVQ_ERR_TIMEOUT, "a bounded wait inside a kernel ran out (error word 0x%x)", v);
   return fail(KVQ_ERR_DEVICE, "a kernel latched device error word 0x%x (1 = missing page)", v);
+}
+
+kvq_status kvq_debug_set_decode_split(kvq_plan* p, int pages_per_split) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (pages_per_split < 0) return fail(KVQ_ERR_INVALID_ARG, "pages_per_split must be >= 0");
+  p->debug_pps = pages_per_split;
+  return KVQ_OK;
+}
+
+kvq_status kvq_debug_fault_injection(kvq_plan* p, int64_t wait_limit_ns, int drop_last_tile) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (wait_limit_ns < 1000 || wait_limit_ns > 2000000000ll)
+    return fail(KVQ_ERR_INVALID_ARG, "wait_limit_ns must be in [1e3, 2e9]");
+  if (drop_last_tile != 0 && drop_last_tile != 1) return fail(KVQ_ERR_INVALID_ARG, "drop_last_tile must be 0 or 1");
+  p->wait_ns = (unsigned long long)wait_limit_ns;
+  p->drop_last_tile = drop_last_tile;
+  return KVQ_OK;
 }
 
 kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int n, const void* x, float* y,

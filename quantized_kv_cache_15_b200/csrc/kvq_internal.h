@@ -198,6 +198,8 @@ struct DecodeParams {
   float* qproj;                  // projected queries M_h q [n_seqs][Hq][128] (projection plans)
   int* tickets;                  // [n_seqs*Hkv]
   int* err;
+  unsigned long long wait_ns;    // bounded waits give up after this long (latching ERR_TIMEOUT)
+  int drop_last_tile;            // test-only fault injection: producers skip their last tile
   int n_seqs;
   HeadInfo heads[MAX_HKV];
   int seq[MAX_BATCH];
@@ -250,7 +252,7 @@ size_t decode_smem_bytes(int stage_bytes, int n_stages, int G, bool wtab_smem);
 // warp's current stage whenever that region is large enough.
 __host__ __device__ constexpr uint32_t wtab_bytes(int G) { return 32u * (4u * (uint32_t)G + 4u) * 4u; }
 constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)16 << 20;   // = KVQ_NOALLOC_SCRATCH_BYTES
-cudaError_t noalloc_scratch(void** out);
+cudaError_t noalloc_scratch(int device, void** out);
 void note_launches(int n);   // counts kernel launches made by the library
 int decode_max_smem();
 

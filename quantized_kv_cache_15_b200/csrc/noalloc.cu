@@ -25,13 +25,14 @@ std::mutex g_mu;
 void* g_ptr[64] = {};
 }  // namespace
 
-// Device address of the scratch array on the current device (looked up on the
-// first call per device).  Returns the CUDA error of the lookup, if any.
-cudaError_t noalloc_scratch(void** out) {
+// Device address of the scratch array on `device`, which must be the current
+// device (looked up on the first call per device).  Returns the CUDA error of the
+// lookup, if any, or cudaErrorInvalidDevice when another device is current.
+cudaError_t noalloc_scratch(int device, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (dev != device || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_ptr[dev]) {
     void* p = nullptr;

@@ -57,6 +57,8 @@ SIGNATURES = {
     "kvq_cobra_allocate": (_I, [_I, _P, ctypes.c_double, _P, _IP, _IP, _IP]),
     "kvq_debug_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "kvq_debug_quantize_f32": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P]),
+    "kvq_debug_set_decode_split": (_I, [_P, _I]),
+    "kvq_debug_fault_injection": (_I, [_P, _I64, _I]),
 }
 
 
@@ -243,6 +245,14 @@ class Plan:
         """Causal attention of the last q.shape[0] tokens of `seq` (already appended)."""
         _check(lib().kvq_prefill_attention(self._h, layer, seq, q.shape[0], _ptr(q), _ptr(out), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), _stream(stream)))
+
+    def debug_set_decode_split(self, pages_per_split: int):
+        """Test-only: fixed pages per split-K piece (0 = automatic)."""
+        _check(lib().kvq_debug_set_decode_split(self._h, pages_per_split))
+
+    def debug_fault_injection(self, wait_limit_ns: int = 2_000_000_000, drop_last_tile: bool = False):
+        """Test-only: bounded-wait limit of the decode kernels and dropped last tiles."""
+        _check(lib().kvq_debug_fault_injection(self._h, int(wait_limit_ns), int(bool(drop_last_tile))))
 
     def debug_rotate(self, layer: int, head: int, kv: int, x: torch.Tensor, y: torch.Tensor, layout: int = 0,
                      stream=None):

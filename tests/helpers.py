@@ -153,57 +153,3 @@ def projection_ambiguous_rows(x_f16: np.ndarray, M: np.ndarray, r: int, b: int) 
     near &= (df > 0)[..., None]
     amb |= near.any(axis=-1)
     return amb.any(axis=-1)
-
-
-def make_projection_unambiguous(w: W.Workload, cells) -> None:
-    """Swap, in w's K and V rows, every row of the given (layer, seq, kv head) cells
-    that projection_ambiguous_rows flags for a fresh draw of the same distribution
-    (the row at the same position of another sequence stream) that it does not
-    flag, so that the cache has exactly one valid encoding and the decode output one
-    expected value.  Replacements come from the leading rows of other sequence
-    streams (1000 k + seq, k = 1, 2, ...).  Installs the substitution into w.rows
-    for the GPU fill and the oracle alike."""
-    base = w.rows
-    reps = {}
-    memo = {}
-
-    def draw(kind, l, s, n):
-        key = (kind, l, s, n)
-        if key not in memo:
-            memo[key] = f16_bits(base(kind, l, s, 0, n))
-        return memo[key]
-
-    for (l, s, h) in cells:
-        r = w.rank[l][h]
-        M = oracle.fuse_projection(w.proj_basis(l, h))
-        for kind in "KV":
-            b = w.k_bits[l][h] if kind == "K" else w.v_bits[l][h]
-            n = w.ctx[s]
-            x = draw(kind, l, s, n)[:, h, :]
-            todo = np.nonzero(projection_ambiguous_rows(x, M, r, b))[0]
-            idx, new = [], []
-            k = 1
-            while len(todo):
-                assert k < 64, "no unambiguous replacement found"
-                cand = draw(kind, l, s + 1000 * k, len(todo))[:, h, :]
-                bad = projection_ambiguous_rows(cand, M, r, b)
-                idx.append(todo[~bad])
-                new.append(cand[~bad])
-                todo = todo[bad]
-                k += 1
-            if idx:
-                reps[(kind, l, s, h)] = (np.concatenate(idx), np.concatenate(new))
-
-    def rows(kind, layer, seq, t0, t1, device="cpu"):
-        out = base(kind, layer, seq, t0, t1, "cpu")
-        for h in range(w.n_kv_heads):
-            rep = reps.get((kind, layer, seq, h))
-            if rep is None:
-                continue
-            i, v = rep
-            sel = (i >= t0) & (i < t1)
-            if sel.any():
-                out[torch.from_numpy(i[sel] - t0), h, :] = torch.from_numpy(v[sel].view(np.int16)).view(torch.float16)
-        return out.to(device)
-
-    w.rows = rows

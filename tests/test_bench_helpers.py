@@ -1,6 +1,6 @@
-"""Host-side helpers of bench.py: the shared config object, the profiled-traffic
-lookup (only for the captured workload and the captured kernel source) and the
-oracle baseline's scaling to the step."""
+"""Host-side helpers of bench.py: the shared config object (identical in both
+arms), the byte accounting, the profiled-traffic lookup (only for the captured
+workload and the captured kernel source)."""
 import os
 import sys
 
@@ -14,19 +14,40 @@ from quantized_kv_cache_15_b200 import workloads as W  # noqa: E402
 
 def test_both_arms_describe_the_workload_alike():
     w = W.make_workload(5, "full")
-    c = bench.workload_config(w, w.n_layers, 1, "x")
+    c = bench.workload_config(w, w.n_layers, 1)
+    assert c == bench.workload_config(W.make_workload(5, "full"), w.n_layers, 1)
     assert c["workload"] == w.name and c["batch"] == w.batch and c["layers"] == w.n_layers
     assert c["tail"] == w.tail and c["rotation"] == "varnorm+hadamard-128"
     assert c["step"].startswith("per layer: append 2048 token(s) x 8 seq(s)")
+    assert c["l2"].startswith("no flush")
+
+
+def test_tiny_workload_is_timed_with_l2_flushes():
+    assert "flushed" in bench.l2_note(W.make_workload(1, "full"))
+    for cfg in (2, 3, 4, 5):
+        assert bench.l2_note(W.make_workload(cfg, "full")).startswith("no flush")
+
+
+def test_byte_accounting_matches_the_documented_row_sizes():
+    w = W.make_workload(2, "full")
+    assert bench.token_head_bytes(w, 0) == 8 * (136 + 72)
+    # one decode launch of the Llama-shaped layer: 32768 tokens x 8 heads x 208 B + q + out
+    assert bench.decode_bytes(w, 0, [32768]) == 32768 * 8 * 208 + 32 * 128 * 6
+    w5 = W.make_workload(5, "full")
+    raw = 8 * 2 * 256
+    # a 2048-token chunk into a sequence longer than its 256-token tail: 2048 input rows
+    # read, 256 ring rows read and requantized, 1792 pass straight through, 256 enter the ring
+    assert bench.append_bytes(w5, 0, 5000, 2048) == 2048 * raw + 256 * raw + 2048 * 8 * 144 + 256 * raw
+    w4 = W.make_workload(4, "full")
+    r, b = w4.rank[0][0], w4.k_bits[0][0]
+    assert bench.row_bytes(W.RANK, r, b) == r * b // 8 + 2 * ((r + 31) // 32)
 
 
 def test_profiled_traffic_is_reported_only_for_its_workload():
-    w2 = W.make_workload(2, "full").name
-    t = bench.traffic_from_profile(w2)
-    # the committed capture covers the llama8b workload; a stale kernel hash gives None
-    assert t is None or t > 54_000_000
-    for cfg in (1, 3, 4, 5):
-        assert bench.traffic_from_profile(W.make_workload(cfg, "full").name) is None
+    # only a capture of the workload, with the current decode source, is used
+    for cfg in (1, 2, 3, 4, 5):
+        t = bench.traffic_from_profile(W.make_workload(cfg, "full").name)
+        assert t is None or t > 0
 
 
 def test_kernel_source_hash_covers_the_decode_sources():
