@@ -40,16 +40,6 @@ kvq_status cuda_fail(cudaError_t e, const char* what) {
 bool valid_codec(int c) { return c >= KVQ_F16 && c <= KVQ_Q5_1; }
 bool valid_rank(int r) { return r == 16 || r == 32 || r == 64 || r == 96 || r == 128; }
 
-// In-place Sylvester Walsh-Hadamard transform of length n (power of two), double.
-void wht_inplace(double* v, int n) {
-  for (int h = 1; h < n; h <<= 1)
-    for (int i = 0; i < n; ++i)
-      if ((i & h) == 0) {
-        double a = v[i], b = v[i + h];
-        v[i] = a + b;
-        v[i + h] = a - b;
-      }
-}
 
 }  // namespace
 
@@ -74,8 +64,8 @@ struct kvq_plan {
   float* d_inv = nullptr;   // [L][Hkv][2][128] inverse RMS (append)
   float* d_sk = nullptr;    // [L][Hkv][128] 1/inv_rms of K (decode, dequantize)
   float* d_sv = nullptr;    // [L][Hkv][128] 1/inv_rms of V
-  float* d_M = nullptr;     // fused projections
-  uint8_t* d_Mimg = nullptr;  // fp16 hi/lo tensor-core images of the projections
+  float* d_M = nullptr;     // fused projections M_h, fp32 [r][128] per head
+  double* d_MT = nullptr;   // their transposes, widened to double [128][r] per head (append projection)
   int* d_bt = nullptr;      // block table [max_seqs][mpps]
   int* d_err = nullptr;
   std::vector<int64_t> len;           // [max_seqs][L]
@@ -91,7 +81,7 @@ struct kvq_plan {
     int prev = 0;
     cudaGetDevice(&prev);
     cudaSetDevice(device);
-    cudaFree(d_inv); cudaFree(d_sk); cudaFree(d_sv); cudaFree(d_M); cudaFree(d_Mimg); cudaFree(d_bt); cudaFree(d_err);
+    cudaFree(d_inv); cudaFree(d_sk); cudaFree(d_sv); cudaFree(d_M); cudaFree(d_MT); cudaFree(d_bt); cudaFree(d_err);
     cudaSetDevice(prev);
   }
 
@@ -175,7 +165,7 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
 
   // per-head codec info and page layout
   std::vector<float> Mhost;
-  std::vector<uint16_t> Mimg;    // per head: hi image then lo image, r x 128 fp16 each
+  std::vector<double> MT;        // per head: M_h^T widened to double, [128][r]
   const double* pb = d->proj_basis;
   p->heads.resize((size_t)p->L * p->Hkv);
   p->layer_off.resize(p->L);
@@ -220,33 +210,30 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
       poff += hi.bytes;
       stage = std::max(stage, (int)hi.bytes);
       if (d->rot == KVQ_ROT_PROJECTION) {
-        // M_h = R_r P_h^T (R_r: Sylvester Hadamard / sqrt(r), block-diagonal H_32 for r = 96)
+        // M_h = R_r P_h^T with R_r = H_r / sqrt(r) (Sylvester H; block-diagonal H_32 for
+        // r = 96): entry (i, c) is the sum over k of H[i][k] P[c][k] within the block of
+        // row i, taken in k order in double (every product is exact: H is +-1), times
+        // 1/sqrt(block), rounded once to fp32.
         hi.m_off = (uint32_t)Mhost.size();
         const int blk = (r == 96) ? 32 : r;
-        std::vector<double> col(r);
+        const double s = 1.0 / std::sqrt((double)blk);
         std::vector<float> M((size_t)r * D);
-        for (int c = 0; c < D; ++c) {
-          for (int k = 0; k < r; ++k) col[k] = pb[(size_t)c * r + k];
-          for (int b0 = 0; b0 < r; b0 += blk) wht_inplace(col.data() + b0, blk);
-          const double s = 1.0 / std::sqrt((double)blk);
-          for (int k = 0; k < r; ++k) M[(size_t)k * D + c] = (float)(col[k] * s);
+        for (int row = 0; row < r; ++row) {
+          const int b0 = (row / blk) * blk, ii = row % blk;
+          for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int k = 0; k < blk; ++k) {
+              const double h = (__builtin_popcount((unsigned)(ii & k)) & 1) ? -1.0 : 1.0;
+              acc += h * pb[(size_t)c * r + b0 + k];
+            }
+            M[(size_t)row * D + c] = (float)(acc * s);
+          }
         }
         Mhost.insert(Mhost.end(), M.begin(), M.end());
         while (Mhost.size() % 4) Mhost.push_back(0.f);
-        // tensor-core images: canonical K-major core-matrix layout, element (n, k) at
-        // ((n / 8) * 16 + k / 8) * 64 + (n % 8) * 8 + k % 8  (in fp16 elements)
-        hi.mimg_off = (uint32_t)(Mimg.size() * 2);
-        std::vector<uint16_t> img((size_t)2 * r * D);
-        for (int n = 0; n < r; ++n)
-          for (int k = 0; k < D; ++k) {
-            const float v = M[(size_t)n * D + k];
-            const __half hh = __float2half_rn(v);
-            const __half hl = __float2half_rn(v - __half2float(hh));
-            const size_t e = ((size_t)(n / 8) * 16 + k / 8) * 64 + (n % 8) * 8 + k % 8;
-            img[e] = __half_as_ushort(hh);
-            img[(size_t)r * D + e] = __half_as_ushort(hl);
-          }
-        Mimg.insert(Mimg.end(), img.begin(), img.end());
+        hi.mt_off = (uint32_t)MT.size();
+        for (int c = 0; c < D; ++c)
+          for (int row = 0; row < r; ++row) MT.push_back((double)M[(size_t)row * D + c]);
         pb += (size_t)D * r;
       }
       p->heads[i] = hi;
@@ -303,11 +290,11 @@ kvq_status kvq_plan_create(const kvq_plan_desc* d, kvq_plan** out) {
       return fail(KVQ_ERR_OOM, "device allocation for the projections failed");
     }
     cudaMemcpy(p->d_M, Mhost.data(), Mhost.size() * 4, cudaMemcpyHostToDevice);
-    if (!dmalloc((void**)&p->d_Mimg, Mimg.size() * 2)) {
+    if (!dmalloc((void**)&p->d_MT, MT.size() * sizeof(double))) {
       delete p;
-      return fail(KVQ_ERR_OOM, "device allocation for the projection images failed");
+      return fail(KVQ_ERR_OOM, "device allocation for the projection transposes failed");
     }
-    cudaMemcpy(p->d_Mimg, Mimg.data(), Mimg.size() * 2, cudaMemcpyHostToDevice);
+    cudaMemcpy(p->d_MT, MT.data(), MT.size() * sizeof(double), cudaMemcpyHostToDevice);
   }
   p->len.assign((size_t)p->max_seqs * p->L, 0);
   p->bt.assign((size_t)p->max_seqs * p->mpps, -1);
@@ -463,19 +450,19 @@ kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* se
     ap.n_seqs = cn;
     ap.total_items = items;
     if (p->rot == KVQ_ROT_PROJECTION && qitems > 0) {
-      // tensor-core projection + quantization of the rows leaving (or bypassing) the
-      // tail; it reads evicted rows from the ring, so it runs before the ring writes
+      // projection + quantization of the rows leaving (or bypassing) the tail; it
+      // reads evicted rows from the ring, so it runs before the ring writes
       ProjParams pp;
       std::memset(&pp, 0, sizeof(pp));
       pp.pool = ap.pool; pp.page_bytes = ap.page_bytes; pp.block_table = ap.block_table;
       pp.max_pages_per_seq = ap.max_pages_per_seq; pp.tail = ap.tail;
       pp.T = T; pp.L = p->L; pp.layer = layer; pp.Hkv = p->Hkv;
       pp.k_in = ap.k_in; pp.v_in = ap.v_in; pp.in_stride = p->Hkv * D;
-      pp.mimg = p->d_Mimg; pp.err = p->d_err;
+      pp.mt = p->d_MT; pp.err = p->d_err;
       pp.n_seqs = cn; pp.total_q = qitems;
       std::memcpy(pp.heads, ap.heads, sizeof(pp.heads));
       std::memcpy(pp.seqs, ap.seqs, sizeof(pp.seqs));
-      cudaError_t e = launch_project(pp, (qitems + 127) / 128, p->Hkv, st);
+      cudaError_t e = launch_project(pp, qitems, p->Hkv, st);
       if (e != cudaSuccess) return cuda_fail(e, "projection launch");
     }
     cudaError_t e = launch_append(ap, st);
@@ -512,8 +499,7 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
   dp.q = (const __half*)q;
   dp.out = out;
   dp.n_seqs = n_seqs;
-  int64_t work = 0;
-  int maxpages = 1;
+  int maxq = 0, maxt = 0;         // most quantized / tail pages of one entry
   for (int i = 0; i < n_seqs; ++i) {
     const int s = seq_ids[i];
     if (s < 0 || s >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d out of range", s);
@@ -523,10 +509,9 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
     dp.lim[i] = lims ? lims[i] : (int)len;
     if (dp.lim[i] < 0 || dp.lim[i] > len) return fail(KVQ_ERR_INVALID_ARG, "visible length %d outside [0, %lld]",
                                                        dp.lim[i], (long long)len);
-    const SplitCounts c = split_counts((int)len, (int)p->T, 1, dp.lim[i]);
-    const int pages = c.nqp + c.ntp;
-    work += (int64_t)pages * p->Hkv;
-    maxpages = std::max(maxpages, pages);
+    const SplitCounts c = split_counts((int)len, (int)p->T, 1, 1, dp.lim[i]);
+    maxq = std::max(maxq, c.nqp);
+    maxt = std::max(maxt, c.ntp);
   }
   L.grid_x = 1;
   L.uses_ws = false;
@@ -551,35 +536,90 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
       break;
     }
   const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G, dp.wtab_smem);
-  // Split size: the candidate with the smallest estimated makespan, counted in waves
-  // of resident CTAs (registers and shared memory both counted) times the pages of
-  // a split plus a fixed cost of about three pages (query preparation, publishing
-  // the partial).  One full wave of equal shares suits one long sequence; a batch of
-  // ragged sequences does better with short splits over many waves.
+  // Split sizes.  A tile's work is taken as its attention multiply-adds: a 64-token
+  // page of head h costs 64 (r_K + r_V) G (r = 128 for the block codecs, the head's
+  // rank for the projection codec), a 16-row tail tile 32 x 256 x G (only half the
+  // lanes score a 16-row tile).  Every head gets pps_q[h] pages per split such that
+  // its splits cost about the same (P unit pages, the unit being the cheapest head's
+  // page), and the tail its own pps_t.  P is the candidate with the smallest
+  // estimated makespan: the largest of (the costliest split) and (the average split
+  // cost x the waves of resident CTAs, registers and shared memory both counted),
+  // where a split of n tiles costs ceil(n / consumer warps) rounds of its tiles plus
+  // a fixed cost of three unit pages (query preparation, publishing the partial).
   const int per_sm = std::max(1, decode_blocks_per_sm(p->G, smem));
   const int64_t target = (int64_t)p->num_sms * per_sm;
-  const int min_pps = (maxpages + MAX_SPLITS - 3) / (MAX_SPLITS - 2);
-  auto makespan = [&](int pp) {
-    int64_t ctas = 0;
-    for (int i = 0; i < n_seqs; ++i) {
-      const SplitCounts c = split_counts(dp.len[i], (int)p->T, pp, dp.lim[i]);
-      ctas += (int64_t)(c.qsplits + c.tsplits) * p->Hkv;
+  std::vector<double> cq(p->Hkv);
+  double cmin = 1e300;
+  for (int h = 0; h < p->Hkv; ++h) {
+    const HeadInfo& hi = p->head(layer, h);
+    const int rk = hi.kcodec == KVQ_RANK ? hi.r : D, rv = hi.vcodec == KVQ_RANK ? hi.r : D;
+    cq[h] = 64.0 * (rk + rv) * p->G;
+    cmin = std::min(cmin, cq[h]);
+  }
+  const double ct = 32.0 * 2 * D * p->G;
+  const int min_q = std::max(1, (maxq + MAX_SPLITS - 3) / (MAX_SPLITS - 2));
+  const int min_t = std::max(1, (maxt + 1) / 2);
+  auto sizes = [&](int P, std::vector<int>& ppq, int& ppt) {
+    ppq.resize(p->Hkv);
+    for (int h = 0; h < p->Hkv; ++h)
+      ppq[h] = std::max(min_q, (int)std::lround((double)P * cmin / cq[h]));
+    ppt = std::max(min_t, (int)std::lround((double)P * cmin / ct));
+    if (p->debug_pps > 0) {                                   // fixed split size (tests)
+      for (int h = 0; h < p->Hkv; ++h) ppq[h] = std::max(min_q, p->debug_pps);
+      ppt = std::max(min_t, p->debug_pps);
     }
-    return ((ctas + target - 1) / target) * (int64_t)(pp + 3);
   };
-  int pps = std::max<int>(min_pps, (int)std::max<int64_t>(1, (work + target - 1) / target));
-  int64_t best = makespan(pps);
-  for (int cand : {8, 16, 32, 64}) {
-    if (cand < min_pps || cand >= pps) continue;
-    const int64_t m = makespan(cand);
-    if (m < best) { best = m; pps = cand; }
-  }
-  if (p->debug_pps > 0) pps = std::max(p->debug_pps, min_pps);   // fixed split size (tests)
-  dp.pps = pps;
+  auto makespan = [&](int P) {
+    std::vector<int> ppq;
+    int ppt;
+    sizes(P, ppq, ppt);
+    int64_t ctas = 0;
+    double total = 0.0, worst = 0.0;
+    // splits of n pages of size pp, each costing rounds of tiles of cost c
+    auto add = [&](int n, int pp, double c) {
+      if (n <= 0) return;
+      const int full = n / pp, rest = n - full * pp;
+      const double cf = (double)((pp + NCW - 1) / NCW) * NCW * c + 3.0 * cmin;
+      total += full * cf;
+      ctas += full;
+      if (full) worst = std::max(worst, cf);
+      if (rest) {
+        const double cr = (double)((rest + NCW - 1) / NCW) * NCW * c + 3.0 * cmin;
+        total += cr;
+        ++ctas;
+        worst = std::max(worst, cr);
+      }
+    };
+    for (int i = 0; i < n_seqs; ++i) {
+      const SplitCounts c = split_counts(dp.len[i], (int)p->T, 1, 1, dp.lim[i]);
+      for (int h = 0; h < p->Hkv; ++h) {
+        add(c.nqp, ppq[h], cq[h]);
+        add(c.ntp, ppt, ct);
+      }
+    }
+    const int64_t waves = (ctas + target - 1) / target;
+    return std::max(worst, (double)waves * total / (double)std::max<int64_t>(ctas, 1));
+  };
+  int64_t unit_pages = 0;
   for (int i = 0; i < n_seqs; ++i) {
-    const SplitCounts c = split_counts(dp.len[i], (int)p->T, pps, dp.lim[i]);
-    L.grid_x = std::max(L.grid_x, c.qsplits + c.tsplits);
+    const SplitCounts c = split_counts(dp.len[i], (int)p->T, 1, 1, dp.lim[i]);
+    for (int h = 0; h < p->Hkv; ++h) unit_pages += (int64_t)std::lround(c.nqp * cq[h] / cmin + c.ntp * ct / cmin);
   }
+  int best_P = std::max<int>(1, (int)((unit_pages + target - 1) / target));
+  double best = makespan(best_P);
+  for (int cand : {4, 6, 8, 10, 12, 16, 24, 32, 48, 64, 96, 128}) {
+    if (cand >= best_P) break;
+    const double m = makespan(cand);
+    if (m < best * 0.999) { best = m; best_P = cand; }
+  }
+  std::vector<int> ppq;
+  sizes(best_P, ppq, dp.pps_t);
+  for (int h = 0; h < p->Hkv; ++h) dp.pps_q[h] = (uint16_t)std::min(ppq[h], 65535);
+  for (int i = 0; i < n_seqs; ++i)
+    for (int h = 0; h < p->Hkv; ++h) {
+      const SplitCounts c = split_counts(dp.len[i], (int)p->T, dp.pps_q[h], dp.pps_t, dp.lim[i]);
+      L.grid_x = std::max(L.grid_x, c.qsplits + c.tsplits);
+    }
   if (L.grid_x > 1 || L.proj) {
     const size_t need = workspace_bytes(p, n_seqs);
     if (!workspace || workspace_bytes_given < need)
@@ -910,11 +950,11 @@ kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int 
     ProjParams pp;
     std::memset(&pp, 0, sizeof(pp));
     pp.k_in = (const __half*)x; pp.in_stride = D;
-    pp.mimg = p->d_Mimg; pp.err = p->d_err;
+    pp.mt = p->d_MT; pp.err = p->d_err;
     pp.z_out = y; pp.head_override = head; pp.kv_override = kv;
     pp.total_q = n; pp.Hkv = p->Hkv;
     for (int hh = 0; hh < p->Hkv; ++hh) pp.heads[hh] = p->head(layer, hh);
-    cudaError_t e = launch_project(pp, (n + 127) / 128, 1, (cudaStream_t)stream);
+    cudaError_t e = launch_project(pp, n, 1, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "projection launch");
     return KVQ_OK;
   }

@@ -9,8 +9,9 @@
 // BeeLlama v0.4.0 news, §KV cache 精度尾部: the tail segment is F16.
 //
 // Work split (split-K): grid (split, kv head, sequence).  A sequence's pages are
-// cut into splits of `pps` pages: first the quantized pages, then the tail
-// pages (never mixed in one split).  Each CTA:
+// cut into splits: first the quantized pages, pps_q[kv head] per split (heads
+// with more work per page -- higher rank, more bits -- get shorter splits), then
+// the tail pages, pps_t per split (never mixed in one split).  Each CTA:
 //   * warp 4 (producer) streams one page-head region per tile into a ring of
 //     shared-memory stages with cp.async.bulk (completion on mbarriers);
 //   * warps 0-3 (consumers) take tiles round-robin, each keeping its own online
@@ -285,7 +286,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
   const int seq = p.seq[si], len = p.len[si];
   const int T = p.T;
-  const SplitCounts sc = split_counts(len, T, p.pps, p.lim[si]);
+  const int pps_q = p.pps_q[head];
+  const SplitCounts sc = split_counts(len, T, pps_q, p.pps_t, p.lim[si]);
   const int nq = sc.nq, nt = sc.nt, NQP = sc.nqp, NTP = sc.ntp, qsplits = sc.qsplits;
   const int S = sc.qsplits + sc.tsplits;
   float* out_base = p.out + ((size_t)si * p.Hq + (size_t)head * G) * D;
@@ -296,8 +298,9 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   }
   if (split >= S) return;
   const bool is_tail = split >= qsplits;
-  const int pg0 = (is_tail ? split - qsplits : split) * p.pps;
-  const int pg1 = min(pg0 + p.pps, is_tail ? NTP : NQP);
+  const int pps = is_tail ? p.pps_t : pps_q;
+  const int pg0 = (is_tail ? split - qsplits : split) * pps;
+  const int pg1 = min(pg0 + pps, is_tail ? NTP : NQP);
   const int n_tiles = pg1 - pg0;
   const int seg_tokens = is_tail ? nt : nq;
   const HeadInfo h = p.heads[head];

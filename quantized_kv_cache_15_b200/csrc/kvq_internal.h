@@ -48,8 +48,9 @@ constexpr int DECODE_THREADS = 32 * (NCW + 1);
 #define DECODE_MIN_CTAS(G) ((NCW <= 4) ? ((G) <= 4 ? 3 : 2) : ((G) <= 4 ? 2 : 1))
 
 // Split-K layout of one sequence of `len` tokens, shared by the host (grid size)
-// and the decode kernel: the quantized segment in 64-token pages, the tail
-// segment in TAIL_TOK-token tail pages, each cut into splits of `pps` pages.
+// and the decode kernel: the quantized segment in 64-token pages cut into splits
+// of pps_q pages, then the tail segment in TAIL_TOK-token tail pages cut into
+// splits of pps_t tail pages (a split never mixes the two).
 // Splits of one (sequence, kv head) of length len whose query sees the first lim
 // tokens (lim = len for decode; lim < len for the earlier queries of a prefill
 // chunk).  nq: visible quantized tokens (pages in position order); nt: tail slots
@@ -58,7 +59,7 @@ constexpr int DECODE_THREADS = 32 * (NCW + 1);
 // and the visible positions nq_all .. lim-1 sit in a cyclic run of slots starting
 // at nq_all mod T: all T slots are visited and the others are masked (tail_visible).
 struct SplitCounts { int nq, nt, nqp, ntp, qsplits, tsplits, nq_all, nt_vis; };
-__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps, int lim) {
+__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps_q, int pps_t, int lim) {
   SplitCounts c;
   c.nq_all = len > T ? len - T : 0;
   c.nq = c.nq_all < lim ? c.nq_all : lim;
@@ -66,11 +67,10 @@ __host__ __device__ inline SplitCounts split_counts(int len, int T, int pps, int
   c.nt = len <= T ? c.nt_vis : (c.nt_vis > 0 ? T : 0);
   c.nqp = (c.nq + PAGE - 1) / PAGE;
   c.ntp = (c.nt + TAIL_TOK - 1) / TAIL_TOK;
-  c.qsplits = (c.nqp + pps - 1) / pps;
-  c.tsplits = (c.ntp + pps - 1) / pps;
+  c.qsplits = (c.nqp + pps_q - 1) / pps_q;
+  c.tsplits = (c.ntp + pps_t - 1) / pps_t;
   return c;
 }
-__host__ __device__ inline SplitCounts split_counts(int len, int T, int pps) { return split_counts(len, T, pps, len); }
 // Whether tail slot s holds a visible position (see split_counts).
 __host__ __device__ inline bool tail_visible(const SplitCounts& c, int T, int s) {
   return ((s - c.nq_all % T) % T + T) % T < c.nt_vis;
@@ -90,7 +90,7 @@ struct HeadInfo {                // one (layer, kv head); 32 bytes
   uint32_t off;                  // region offset inside a page
   uint32_t bytes;                // region bytes = 64 * (cbK + sbK + cbV + sbV)
   uint32_t m_off;                // float offset of M_h (r x 128) in the projection table
-  uint32_t mimg_off;             // byte offset of M_h's fp16 hi/lo tensor-core images
+  uint32_t mt_off;               // double offset of M_h^T (128 x r, exact widening) in the projection's table
 };
 
 __host__ __device__ inline int codec_bits(int c) {
@@ -152,8 +152,8 @@ struct AppendParams {
   AppendSeq seqs[MAX_APPEND_SEQS];
 };
 
-// Projection path (tcgen05): quantize items E and P of an append, or (z_out set)
-// export z = M_h x for rows of k_in.
+// Projection path: quantize items E and P of an append, or (z_out set) export
+// z = M_h x for rows of k_in.
 struct ProjParams {
   uint8_t* pool;
   uint32_t page_bytes;
@@ -164,7 +164,7 @@ struct ProjParams {
   const __half* k_in;
   const __half* v_in;
   int in_stride;                 // halves between consecutive input rows
-  const uint8_t* mimg;           // hi/lo fp16 images of every head
+  const double* mt;              // M_h^T of every head, double [128][r] at heads[h].mt_off
   int* err;
   float* z_out;                  // inspection: z rows [total_q][r] (one head, one kv)
   int head_override, kv_override;
@@ -190,7 +190,8 @@ struct DecodeParams {
   const float* s_v;              // [Hkv][128] per-channel V multiplier or null
   const float* M;                // projection table (floats), or null
   float qscale;                  // softmax scale * log2(e)
-  int pps;                       // pages per split
+  int pps_t;                     // tail pages per split
+  uint16_t pps_q[MAX_HKV];       // quantized pages per split, per kv head (work-balanced)
   int stage_bytes;               // bytes of one pipeline stage
   int n_stages;                  // 4 or 8
   int wtab_smem;                 // 1: the weight tables get their own shared memory (some head's K rows are too small)
@@ -239,7 +240,7 @@ cudaError_t launch_dequantize(const DecodeParams& p, int seq, int64_t t0, int64_
                               cudaStream_t s);
 cudaError_t launch_read_rows(const DecodeParams& p, int seq, int64_t t0, int64_t t1, int kv, uint8_t* codes,
                              uint8_t* scales, cudaStream_t s);
-cudaError_t launch_project(const ProjParams& p, int n_tiles, int n_heads, cudaStream_t s);
+cudaError_t launch_project(const ProjParams& p, int n_items, int n_heads, cudaStream_t s);
 cudaError_t launch_calibrate(int64_t n_tok, int n_ch, int64_t stride, const __half* x, float* inv, cudaStream_t s);
 cudaError_t launch_debug_rotate(const HeadInfo& h, int rot, int kv, const float* inv_s, int n, const __half* x,
                                 float* y, bool quad, bool bf16, cudaStream_t s);

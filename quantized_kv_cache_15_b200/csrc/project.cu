@@ -1,26 +1,25 @@
-// Per-head projection of the rank/bit codec on the 5th-generation tensor cores.
+// Per-head projection of the rank/bit codec: z = M_h x, then the block quantizer.
 //
 // KV-COBRA explainer, §The news: each key is projected, rotated and quantized
-// with frozen per-head settings, the rotation "fused into the same projection
-// matrix" -- z = M_h x with M_h = R_r P_h^T (r x 128).  For a tile of 128 rows
-// of one head this is a [128 x 128] x [128 x r] GEMM: the one place where the
-// hot path is a dense contraction, so it runs as tcgen05.mma (kind::f16,
-// fp32 accumulation in tensor memory).
+// with frozen per-head settings, the rotation folded into the projection matrix
+// -- M_h = R_r P_h^T (r x 128, stored fp32).  §Jargon "Scalar quantization": a
+// block's step and each value's level are integer decisions taken on z, so two
+// ways of forming z that differ in the last bits can store different codes (one
+// level, or one fp16 ulp of a step, apart), and a key or value one level off
+// moves the attention output well past the parity bar at 1-2 bits.
 //
-//  * A (the fp16 rows) is exact in fp16.  M_h is split into fp16 hi + lo
-//    (hi = fp16(M), lo = fp16(M - hi)), two MMAs per K step accumulate into the
-//    same TMEM columns, so z carries ~22 bits of M.
-//  * Operands live in shared memory in the canonical K-major layout without
-//    swizzle: 8-row x 16-byte core matrices, K-adjacent core matrices 128 B apart
-//    (leading byte offset), 8-row groups 2048 B apart (stride byte offset).  The
-//    host prebuilds M_h's hi/lo images in exactly this layout, fetched with one
-//    bulk copy; the A tile is gathered by the CTA's threads.
-//  * One thread issues the 16 MMAs (8 K steps x hi/lo) and commits them to an
-//    mbarrier; the epilogue reads the accumulator with tcgen05.ld (warp w owns
-//    TMEM lanes 32w..32w+31 = rows), stages z in shared memory and runs the same
-//    warp quantizer as the rotation path.
-// Every wait is bounded; on a timeout the kernel latches an error bit, still
-// frees its tensor memory and returns.
+// So z is formed exactly as its definition states it for fp32 M_h and fp16 x:
+// each product M_rc x_c is exact in double (24 + 11 significant bits), the 128
+// products are added in channel order c = 0 .. 127 in double, and the sum is
+// rounded once to fp32.  With an exact product, a double FMA is that same
+// multiply-then-add, so the kernel's z -- and therefore its codes and scales --
+// are the definition's, bit for bit, whatever the rows.
+//
+// One CTA: one (kv head, K|V) and up to 64 rows.  M_h^T (double, [128][r]) and
+// the rows (double, [64][128]) are staged in shared memory; warp w takes rows w,
+// w + 8, ... two at a time, lane l holds outputs 4l .. 4l+3 of both (eight
+// independent FMA chains over c), and the warp then quantizes each row with the
+// same warp quantizer as the rotation path (lane l: values 4l .. 4l+3).
 #include "kvq_internal.h"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -28,54 +27,17 @@
 namespace kvq {
 
 namespace {
-
-constexpr int TILE_M = 128;
-constexpr int A_BYTES = TILE_M * D * 2;   // 32 KiB
-
-__device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;   // descriptor version for sm_100; base offset 0, no swizzle
-  return d;
-}
-
-// kind::f16 instruction descriptor: D fp32, A and B fp16, both K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t umma_idesc_f16(int n) {
-  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TILE_M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* out) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) out[i] = __uint_as_float(r[i]);
-}
-
+constexpr int PJ_ROWS = 64;                  // rows per CTA
+constexpr int PJ_WARPS = 8;
+constexpr int PJ_THREADS = 32 * PJ_WARPS;
 }  // namespace
 
-__global__ void __launch_bounds__(128, 1) proj_kernel(const __grid_constant__ ProjParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
+size_t proj_smem_bytes(int r) {
+  return (size_t)D * r * 8 + (size_t)PJ_ROWS * D * 8 + (size_t)PJ_ROWS * (sizeof(void*) + 12);
+}
+
+__global__ void __launch_bounds__(PJ_THREADS, 1) proj_kernel(const __grid_constant__ ProjParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x;
   const int head = p.z_out ? p.head_override : (int)blockIdx.y;
@@ -85,34 +47,23 @@ __global__ void __launch_bounds__(128, 1) proj_kernel(const __grid_constant__ Pr
   if (codec != KVQ_RANK) return;                      // F16 heads of a projection plan: append kernel
   const int r = h.r;
   const int bits = kv ? h.vbits : h.kbits;
-  const uint32_t bbytes = (uint32_t)r * 256u;         // one fp16 image of M_h (r x 128)
-  const uint32_t ncols = r <= 32 ? 32u : (r <= 64 ? 64u : 128u);
 
-  uint8_t* sA = smem;                                  // 32 KiB, later reused for z
-  uint8_t* sB = smem + A_BYTES;                        // hi image then lo image
-  size_t off = A_BYTES + 2 * (size_t)bbytes;
-  const uint8_t** rbase = reinterpret_cast<const uint8_t**>(smem + off); off += TILE_M * sizeof(void*);
-  int* rstride = reinterpret_cast<int*>(smem + off); off += TILE_M * 4;
-  int* rpos = reinterpret_cast<int*>(smem + off); off += TILE_M * 4;
-  int* rseq = reinterpret_cast<int*>(smem + off); off += TILE_M * 4;
-  off = (off + 15) & ~(size_t)15;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + off); off += 16;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + off);
+  double* mt = reinterpret_cast<double*>(smem);                      // [128 c][r] = M_h^T
+  double* xs = mt + (size_t)D * r;                                   // [64 rows][128 c]
+  const uint8_t** rbase = reinterpret_cast<const uint8_t**>(xs + (size_t)PJ_ROWS * D);
+  int* rstride = reinterpret_cast<int*>(rbase + PJ_ROWS);
+  int* rpos = rstride + PJ_ROWS;
+  int* rseq = rpos + PJ_ROWS;
 
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
-                 "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    fence_mbar_init();
-  }
-  // ---- row sources: row i of the tile is quantize item tile*128 + i
+  // ---- M_h^T (exact widening of the stored fp32 M_h, precomputed by the plan)
   {
-    const int q = tile * TILE_M + tid;
+    const double2* src = reinterpret_cast<const double2*>(p.mt + h.mt_off);
+    double2* dst = reinterpret_cast<double2*>(mt);
+    for (int i = tid; i < D * r / 2; i += PJ_THREADS) dst[i] = src[i];
+  }
+  // ---- row sources: row i of the tile is quantize item tile * 64 + i
+  if (tid < PJ_ROWS) {
+    const int q = tile * PJ_ROWS + tid;
     const uint8_t* base = nullptr;
     int stride = 16, pos = -1, seq = -1;
     if (q < p.total_q) {
@@ -144,118 +95,84 @@ __global__ void __launch_bounds__(128, 1) proj_kernel(const __grid_constant__ Pr
     }
     rbase[tid] = base; rstride[tid] = stride; rpos[tid] = pos; rseq[tid] = seq;
   }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  const uint32_t tmem = *tslot;
-
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar[0], 2 * bbytes);
-    bulk_g2s(sB, p.mimg + h.mimg_off, 2 * bbytes, &bar[0]);
-  }
-  // ---- A tile in the canonical layout: 128 rows x 16 chunks of 16 bytes
-  for (int idx = tid; idx < TILE_M * 16; idx += 128) {
+  // ---- rows into shared memory as doubles (fp16 widens exactly); 16 chunks of 8 values
+  for (int idx = tid; idx < PJ_ROWS * 16; idx += PJ_THREADS) {
     const int row = idx >> 4, c = idx & 15;
     const uint8_t* b = rbase[row];
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (b) v = *reinterpret_cast<const uint4*>(b + (size_t)c * rstride[row]);
-    *reinterpret_cast<uint4*>(sA + ((row >> 3) * 16 + c) * 128 + (row & 7) * 16) = v;
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
-
-  bool ok = true;
-  if (tid == 0) {
-    if (!mbar_wait(&bar[0], 0)) { atomicOr(p.err, ERR_TIMEOUT); ok = false; }
-    if (ok) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t idesc = umma_idesc_f16(r);
-      const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    double* dst = xs + (size_t)row * D + 8 * c;
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        umma_f16(tmem, umma_smem_desc(a0 + s * 256, 128, 2048), umma_smem_desc(b0 + s * 256, 128, 2048), idesc,
-                 s > 0 ? 1u : 0u);
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        umma_f16(tmem, umma_smem_desc(a0 + s * 256, 128, 2048), umma_smem_desc(b0 + bbytes + s * 256, 128, 2048),
-                 idesc, 1u);
-      umma_commit(&bar[1]);
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      dst[2 * k] = (double)f.x;
+      dst[2 * k + 1] = (double)f.y;
     }
   }
   __syncthreads();
-  // Wait for the accumulator (every thread polls the same barrier, bounded).
-  if (!mbar_wait(&bar[1], 0)) {
-    if (tid == 0) atomicOr(p.err, ERR_TIMEOUT);
-    ok = false;
-  }
-  ok = __syncthreads_and(ok);
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
-  float* zs = reinterpret_cast<float*>(smem);          // [128][r+1], over A and B (no longer read)
-  const int zst = r + 1;
-  if (ok) {
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    for (int c0 = 0; c0 < r; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem + lane_base + (uint32_t)c0, v);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) zs[(32 * warp + lane) * zst + c0 + j] = v[j];
+  const int i0 = 4 * lane;
+  const bool own = i0 < r;
+  for (int k = 0; k < PJ_ROWS / (2 * PJ_WARPS); ++k) {
+    const int ra = warp + 2 * PJ_WARPS * k, rb = ra + PJ_WARPS;
+    const bool va = rpos[ra] >= 0, vb = rpos[rb] >= 0;
+    if (!va && !vb) continue;                             // warp-uniform
+    double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
+    if (own) {
+      const double* xa = xs + (size_t)ra * D;
+      const double* xb = xs + (size_t)rb * D;
+#pragma unroll 4
+      for (int c = 0; c < D; ++c) {
+        const double2 m01 = *reinterpret_cast<const double2*>(mt + (size_t)c * r + i0);
+        const double2 m23 = *reinterpret_cast<const double2*>(mt + (size_t)c * r + i0 + 2);
+        const double x0 = xa[c], x1 = xb[c];
+        a[0] = fma(m01.x, x0, a[0]); a[1] = fma(m01.y, x0, a[1]);
+        a[2] = fma(m23.x, x0, a[2]); a[3] = fma(m23.y, x0, a[3]);
+        b[0] = fma(m01.x, x1, b[0]); b[1] = fma(m01.y, x1, b[1]);
+        b[2] = fma(m23.x, x1, b[2]); b[3] = fma(m23.y, x1, b[3]);
+      }
     }
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
-  if (warp == 0) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
-  }
-  if (!ok) return;
-
-  // ---- epilogue: warp w quantizes (or exports) rows 32w .. 32w+31
-  for (int i = 0; i < 32; ++i) {
-    const int row = 32 * warp + i;
-    const int pos = rpos[row];
-    if (pos < 0) continue;
-    float x[4];
+    for (int which = 0; which < 2; ++which) {
+      const int row = which ? rb : ra;
+      const int pos = rpos[row];
+      if (pos < 0) continue;                              // warp-uniform
+      float z[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) x[k] = (4 * lane + k < r) ? zs[row * zst + 4 * lane + k] : 0.f;
-    if (p.z_out) {
+      for (int j = 0; j < 4; ++j) z[j] = own ? (float)(which ? b[j] : a[j]) : 0.f;
+      if (p.z_out) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (4 * lane + k < r) p.z_out[(size_t)pos * r + 4 * lane + k] = x[k];
-      continue;
+        for (int j = 0; j < 4; ++j)
+          if (i0 + j < r) p.z_out[(size_t)pos * r + i0 + j] = z[j];
+        continue;
+      }
+      const int pid = p.block_table[(size_t)rseq[row] * p.max_pages_per_seq + pos / PAGE];
+      if (pid < 0) {
+        if (lane == 0) atomicOr(p.err, ERR_NO_PAGE);
+        continue;
+      }
+      uint8_t* region = p.pool + (size_t)pid * p.page_bytes + h.off;
+      uint8_t* codes = kv ? region + PAGE * (h.cbK + h.sbK) : region;
+      const int cb = kv ? h.cbV : h.cbK;
+      uint8_t* scales = codes + PAGE * cb;
+      quantize_store_row(z, KVQ_RANK, r, bits, codes, scales, pos % PAGE, kv == 0);
     }
-    const int pid = p.block_table[(size_t)rseq[row] * p.max_pages_per_seq + pos / PAGE];
-    if (pid < 0) {
-      if (lane == 0) atomicOr(p.err, ERR_NO_PAGE);
-      continue;
-    }
-    uint8_t* region = p.pool + (size_t)pid * p.page_bytes + h.off;
-    uint8_t* codes = kv ? region + PAGE * (h.cbK + h.sbK) : region;
-    const int cb = kv ? h.cbV : h.cbK;
-    uint8_t* scales = codes + PAGE * cb;
-    quantize_store_row(x, KVQ_RANK, r, bits, codes, scales, pos % PAGE, kv == 0);
   }
 }
 
-size_t proj_smem_bytes(int r) {
-  size_t off = A_BYTES + 2 * (size_t)r * 256;
-  off += TILE_M * (sizeof(void*) + 12);
-  off = (off + 15) & ~(size_t)15;
-  off += 16 + 16;
-  const size_t zbytes = (size_t)TILE_M * (r + 1) * 4;
-  return off > zbytes ? off : zbytes + 64;
-}
-
-cudaError_t launch_project(const ProjParams& p, int n_tiles, int n_heads, cudaStream_t s) {
-  if (n_tiles <= 0) return cudaSuccess;
-  size_t smem = proj_smem_bytes(128);
+cudaError_t launch_project(const ProjParams& p, int n_items, int n_heads, cudaStream_t s) {
+  if (n_items <= 0) return cudaSuccess;
+  const size_t smem = proj_smem_bytes(128);
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  const int n_tiles = (n_items + PJ_ROWS - 1) / PJ_ROWS;
   dim3 grid(n_tiles, p.z_out ? 1 : n_heads, p.z_out ? 1 : 2);
-  proj_kernel<<<grid, 128, smem, s>>>(p);
+  proj_kernel<<<grid, PJ_THREADS, smem, s>>>(p);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -100,56 +100,3 @@ def rel_err_rows(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
     num = np.abs(got.astype(np.float64) - ref.astype(np.float64)).max(axis=-1)
     den = np.abs(ref.astype(np.float64)).max(axis=-1)
     return num / np.maximum(den, 1e-30)
-
-
-# ----------------------------------------------------------------------------- projection decisions
-# KV-COBRA explainer, §Jargon "Scalar quantization": a block's step is
-# d = fp16(max|z| / (2^(b-1) - 1/2)) and a value's level is floor(z / d).  Both are
-# integer decisions taken on the projection z = M x.  The kernel forms z on the tensor
-# cores (exact fp16 x fp16 products of x and the hi/lo halves of M, fp32 accumulation
-# over 256 products); the oracle accumulates in double.  Their difference is bounded
-# per value by PROJ_EPS * sum_c |x_c| |M_rc|: with unit roundoff u = 2^-24 and n = 256
-# products the probabilistic bound of fp32 summation (Higham and Mary 2019,
-# lambda * sqrt(n) * u with lambda = 3) is 2.9e-6; the hi/lo residual of M
-# (2^-22 relative) and one ulp of M's own rounding add less than 3e-7.
-PROJ_EPS = 3.2e-6
-
-
-def projection_error_bound(x_f16: np.ndarray, M: np.ndarray) -> np.ndarray:
-    """[n][r] bound on |z_kernel - z_oracle| for fp16 rows x [n][128] and M [r][128]."""
-    x = oracle.f16_to_f32(x_f16).astype(np.float64)
-    return PROJ_EPS * (np.abs(x) @ np.abs(M.astype(np.float64)).T)
-
-
-def projection_ambiguous_rows(x_f16: np.ndarray, M: np.ndarray, r: int, b: int) -> np.ndarray:
-    """Boolean [n]: rows with a block step or a level that the oracle places within
-    the projection error bound of a decision boundary (an fp16 rounding midpoint of
-    the step, an integer multiple of the step).  Such a row has more than one valid
-    encoding; every other row has exactly one."""
-    z = oracle.to_stored_basis(kvq.RANK, W.ROT_PROJECTION, x_f16, M=M, r=r)
-    _, sc = oracle.quantize_rows(kvq.RANK, z, r=r, b=b)
-    eps = projection_error_bound(x_f16, M)
-    n = z.shape[0]
-    blk = min(r, 32)
-    nb = r // blk
-    zb = z.astype(np.float64).reshape(n, nb, blk)
-    eb = eps.reshape(n, nb, blk)
-    L = float((1 << (b - 1)) - 0.5)
-    # step decision: fp16 rounding of amax / L (amax moves by at most the largest bound)
-    amax = np.abs(zb).max(axis=-1)
-    a = (np.float32(1.0) * (amax.astype(np.float32) / np.float32(L))).astype(np.float64)
-    hb = oracle.f16_rn(a.astype(np.float32)).astype(np.int64)
-    v = oracle.f16_to_f32(hb.astype(np.uint16)).astype(np.float64)
-    prev = oracle.f16_to_f32(np.maximum(hb - 1, 0).astype(np.uint16)).astype(np.float64)
-    nxt = oracle.f16_to_f32(np.minimum(hb + 1, 0x7BFF).astype(np.uint16)).astype(np.float64)
-    dist = np.minimum(np.where(hb > 0, np.abs(a - (prev + v) / 2), np.inf), np.abs(a - (v + nxt) / 2))
-    slack = eb.max(axis=-1) / L + a * 2.0 ** -22
-    amb = (dist <= slack) & (amax > 0)
-    # level decisions: z / d against the integers
-    df = oracle.f16_to_f32(sc).astype(np.float64).reshape(n, nb)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        t = zb / df[..., None]
-        near = np.abs(t - np.round(t)) <= eb / df[..., None] + np.abs(t) * 2.0 ** -22
-    near &= (df > 0)[..., None]
-    amb |= near.any(axis=-1)
-    return amb.any(axis=-1)

@@ -60,16 +60,13 @@ def test_packed_rows_bit_exact(cfg):
                     assert np.array_equal(gs, os_), (cfg, s, l, kv, h)
 
 
-def test_projection_codes_bit_exact_where_unique():
-    """The projection z runs on the tensor cores in fp32, the oracle's in double, so a
-    step or level that the oracle puts within the projection error bound of a
-    decision boundary has two valid encodings.  Every other row must equal the
-    oracle's bit for bit; a flagged row may differ only by one fp16 ulp of a step and
-    one level of a code."""
+def test_projection_codes_bit_exact():
+    """The per-head projection path (KV-COBRA): packed rows read back from the cache
+    equal the oracle's encoding of the same fp16 history bit for bit, every row, K and
+    V, every head of both layers."""
     w = W.make_workload(4, "small")
     plan = H.make_plan(w)
     H.fill(plan, w, chunk=512)
-    flagged = total = 0
     for l in range(w.n_layers):
         for kv, kind in enumerate("KV"):
             rows = _read(plan, w, l, 0, kv, w.ctx[0])
@@ -79,20 +76,10 @@ def test_projection_codes_bit_exact_where_unique():
                 b = w.k_bits[l][h] if kv == 0 else w.v_bits[l][h]
                 M = oracle.fuse_projection(w.proj_basis(l, h))
                 x = H.f16_bits(hist[:, h, :])
-                amb = H.projection_ambiguous_rows(x, M, r, b)
                 oc, os_ = oracle.encode_rows(kvq.RANK, W.ROT_PROJECTION, x, M=M, r=r, b=b)
                 gc, gs = rows[h]
-                assert np.array_equal(gc[~amb], oc[~amb]), (l, kv, h)
-                assert np.array_equal(gs[~amb], os_[~amb]), (l, kv, h)
-                gu = np.stack([oracle.unpack_codes(c, r, b) for c in gc[amb]]).astype(int) if amb.any() else None
-                if gu is not None:
-                    ou = np.stack([oracle.unpack_codes(c, r, b) for c in oc[amb]]).astype(int)
-                    assert np.abs(gu - ou).max() <= 1
-                    ulp = np.abs(gs[amb].astype(np.int32) - os_[amb].astype(np.int32))
-                    assert ulp.max() <= 1
-                flagged += int(amb.sum())
-                total += amb.size
-    assert flagged < total
+                assert np.array_equal(gc, oc), (l, kv, h)
+                assert np.array_equal(gs, os_), (l, kv, h)
 
 
 def test_tail_holds_newest_rows_raw_and_dequantize_matches_oracle():

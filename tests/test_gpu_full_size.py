@@ -98,11 +98,7 @@ def _read_rows(plan, w, layer, seq, kv, t0, t1):
 
 def _check_packed_rows(plan, w, cells, runs=((0, 64), (0.5, 64), (1.0, 64))):
     """Runs of packed rows (start of the quantized range, its middle, its end) of the
-    cells' (layer, seq, head), K and V, equal the oracle's encoding bit for bit.  For
-    the projection path a row the oracle places within the projection error bound of a
-    quantizer decision may differ by one level or one fp16 ulp of a step
-    (test_gpu_append.test_projection_codes_bit_exact_where_unique); every other row is
-    exact."""
+    cells' (layer, seq, head), K and V, equal the oracle's encoding bit for bit."""
     checked = 0
     for (l, s, h) in cells:
         nq = max(0, w.ctx[s] - w.tail)
@@ -119,15 +115,12 @@ def _check_packed_rows(plan, w, cells, runs=((0, 64), (0.5, 64), (1.0, 64))):
                 if w.rot == W.ROT_PROJECTION:
                     b = hp["kb"] if kv == 0 else hp["vb"]
                     oc, os_ = oracle.encode_rows(W.RANK, w.rot, x, M=hp["M"], r=hp["r"], b=b)
-                    amb = H.projection_ambiguous_rows(x, hp["M"], hp["r"], b)
-                    same = np.all(gc == oc, axis=1) & np.all(gs == os_, axis=1)
-                    assert same[~amb].all(), (l, s, h, kv, t0, np.nonzero(~same & ~amb)[0][:5])
                 else:
                     codec = hp["k_codec"] if kv == 0 else hp["v_codec"]
                     inv = hp.get("inv_s_k" if kv == 0 else "inv_s_v")
                     oc, os_ = oracle.encode_rows(codec, w.rot, x, inv_s=inv)
-                    assert np.array_equal(gc, oc), (l, s, h, kv, t0)
-                    assert np.array_equal(gs, os_), (l, s, h, kv, t0)
+                assert np.array_equal(gc, oc), (l, s, h, kv, t0)
+                assert np.array_equal(gs, os_), (l, s, h, kv, t0)
                 checked += t1 - t0
     assert checked > 0
 
@@ -156,8 +149,8 @@ def test_vbr_mix_full():
 
 
 def test_cobra_rank_bits_full():
-    """256 heads with per-head (r, b), 128k tokens, tcgen05 projection: every layer,
-    on the workload's own rows (no input is substituted)."""
+    """256 heads with per-head (r, b), 128k tokens, per-head projection: every layer,
+    on the workload's own rows."""
     w = W.make_workload(4, "full")
     plan = H.make_plan(w)
     H.fill(plan, w, chunk=8192)

@@ -26,15 +26,16 @@ int main() {
   for (int T : tails)
     for (int len = 0; len <= 1300; len += (len < 200 ? 1 : 37))
       for (int lim = 0; lim <= len; lim += (len < 200 ? 1 : 13)) {
-        for (int pps : {1, 3, 8}) {
-          const SplitCounts c = split_counts(len, T, pps, lim);
+        for (int pps : {1, 3, 8})
+        for (int ppt : {1, 2, 5}) {
+          const SplitCounts c = split_counts(len, T, pps, ppt, lim);
           const int nq_all = len > T ? len - T : 0;
           std::vector<int> seen(len > 0 ? len : 1, 0);
           // quantized pages: splits of pps pages, 64 rows each, first nq tokens
           if (c.qsplits * pps < c.nqp || (c.qsplits - 1) * pps >= c.nqp + (c.nqp == 0)) { printf("bad qsplits\n"); return 1; }
           for (int t = 0; t < c.nq; ++t) seen[t]++;
           // tail: ntp tiles of TAIL_TOK slots, slots < nt visited, then masked
-          if (c.tsplits * pps < c.ntp) { printf("bad tsplits\n"); return 1; }
+          if (c.tsplits * ppt < c.ntp || (c.tsplits - 1) * ppt >= c.ntp + (c.ntp == 0)) { printf("bad tsplits\n"); return 1; }
           for (int s = 0; s < c.ntp * TAIL_TOK; ++s) {
             if (s >= c.nt) continue;
             if (!tail_visible(c, T, s)) continue;

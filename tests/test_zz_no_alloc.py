@@ -10,6 +10,8 @@ contents, so the second call checks that nothing stale leaks in.  It must also
 leave the device's free memory and torch's allocations unchanged.  This file is
 collected last.
 """
+import gc
+
 import pytest
 import torch
 
@@ -36,15 +38,24 @@ def test_noalloc_decode_matches_the_oracle_twice(cfg):
     qs = {(step, l): torch.stack([w.queries(l, s, step, "cuda") for s in seqs])
           for step in range(2) for l in range(w.n_layers)}
     outs = {k: torch.full((len(seqs), w.n_q_heads, 128), float("nan"), device="cuda") for k in qs}
+    # objects of earlier tests that the collector frees in the middle of the calls
+    # would change the device's free memory: collect them first, then hold it off
+    gc.collect()
     torch.cuda.synchronize()
-    alloc0 = torch.cuda.memory_allocated()
-    free0, _ = torch.cuda.mem_get_info()
-    for step in range(2):
-        for l in range(w.n_layers):
-            plan.decode_noalloc(l, seqs, qs[(step, l)], outs[(step, l)])
-    torch.cuda.synchronize()
-    assert torch.cuda.memory_allocated() == alloc0
-    assert torch.cuda.mem_get_info()[0] == free0
+    gc.disable()
+    try:
+        alloc0 = torch.cuda.memory_allocated()
+        free0, _ = torch.cuda.mem_get_info()
+        for step in range(2):
+            for l in range(w.n_layers):
+                plan.decode_noalloc(l, seqs, qs[(step, l)], outs[(step, l)])
+        torch.cuda.synchronize()
+        alloc1 = torch.cuda.memory_allocated()
+        free1, _ = torch.cuda.mem_get_info()
+    finally:
+        gc.enable()
+    assert alloc1 == alloc0
+    assert free1 == free0
     plan.check_device_error()
     for (step, l), out in outs.items():
         got = out.cpu().numpy()
