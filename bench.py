@@ -164,7 +164,7 @@ def l2_note(w):
     return f"no flush: the step reads {b / 1e9:.2f} GB of packed cache, far more than L2 (126 MB)"
 
 
-DECODE_SOURCES = ("decode.cu", "decode_fast.cuh", "kvq_internal.h", "ptx.cuh", "quant.cuh")
+DECODE_SOURCES = ("decode.cu", "decode_fast.cuh", "pair_tables.h", "kvq_internal.h", "ptx.cuh", "quant.cuh")
 
 
 def kernel_source_sha256():

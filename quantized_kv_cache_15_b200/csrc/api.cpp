@@ -528,7 +528,7 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
   if (p->T > 0 && (uint32_t)TAIL_TOK * (uint32_t)(2 * D) < wtab_bytes(p->G)) dp.wtab_smem = 1;
   // Stage ring: one stage per consumer warp at least, deeper while the CTAs per SM
   // that the register allocation aims at still fit in shared memory.
-  const int want_ctas = NCW <= 4 ? 3 : 2;
+  const int want_ctas = DECODE_MIN_CTAS(p->G);
   dp.n_stages = NCW;
   for (int ns = 8; ns > NCW; --ns)
     if (decode_smem_bytes(dp.stage_bytes, ns, p->G, dp.wtab_smem) + 1024 <= (228 * 1024) / want_ctas) {
@@ -536,27 +536,22 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
       break;
     }
   const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G, dp.wtab_smem);
-  // Split sizes.  A tile's work is taken as its attention multiply-adds: a 64-token
-  // page of head h costs 64 (r_K + r_V) G (r = 128 for the block codecs, the head's
-  // rank for the projection codec), a 16-row tail tile 32 x 256 x G (only half the
-  // lanes score a 16-row tile).  Every head gets pps_q[h] pages per split such that
-  // its splits cost about the same (P unit pages, the unit being the cheapest head's
-  // page), and the tail its own pps_t.  P is the candidate with the smallest
-  // estimated makespan: the largest of (the costliest split) and (the average split
-  // cost x the waves of resident CTAs, registers and shared memory both counted),
-  // where a split of n tiles costs ceil(n / consumer warps) rounds of its tiles plus
-  // a fixed cost of three unit pages (query preparation, publishing the partial).
+  // Split sizes.  Measured per-tile times of one consumer warp barely depend on the
+  // head's rank or bits (the loops' fixed work per tile dominates), so every
+  // quantized page counts as one unit of work and a 16-row tail tile as half a
+  // unit; the machinery still allows a per-head size pps_q[h] and the tail its own
+  // pps_t.  The split size is the candidate with the smallest estimated makespan:
+  // the largest of (the costliest split) and (the average split cost x the waves of
+  // resident CTAs, registers and shared memory both counted), where a split of n
+  // tiles costs ceil(n / consumer warps) rounds of its tiles plus a fixed cost of
+  // three units (query preparation, publishing the partial).  Candidates cover the
+  // sizes just above one full wave of CTAs one by one, so a sequence whose pages
+  // would spill a few CTAs into a second wave gets a slightly larger split.
   const int per_sm = std::max(1, decode_blocks_per_sm(p->G, smem));
   const int64_t target = (int64_t)p->num_sms * per_sm;
-  std::vector<double> cq(p->Hkv);
-  double cmin = 1e300;
-  for (int h = 0; h < p->Hkv; ++h) {
-    const HeadInfo& hi = p->head(layer, h);
-    const int rk = hi.kcodec == KVQ_RANK ? hi.r : D, rv = hi.vcodec == KVQ_RANK ? hi.r : D;
-    cq[h] = 64.0 * (rk + rv) * p->G;
-    cmin = std::min(cmin, cq[h]);
-  }
-  const double ct = 32.0 * 2 * D * p->G;
+  std::vector<double> cq(p->Hkv, 1.0);
+  const double cmin = 1.0;
+  const double ct = 0.5;
   const int min_q = std::max(1, (maxq + MAX_SPLITS - 3) / (MAX_SPLITS - 2));
   const int min_t = std::max(1, (maxt + 1) / 2);
   auto sizes = [&](int P, std::vector<int>& ppq, int& ppt) {
@@ -605,10 +600,13 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
     const SplitCounts c = split_counts(dp.len[i], (int)p->T, 1, 1, dp.lim[i]);
     for (int h = 0; h < p->Hkv; ++h) unit_pages += (int64_t)std::lround(c.nqp * cq[h] / cmin + c.ntp * ct / cmin);
   }
-  int best_P = std::max<int>(1, (int)((unit_pages + target - 1) / target));
-  double best = makespan(best_P);
-  for (int cand : {4, 6, 8, 10, 12, 16, 24, 32, 48, 64, 96, 128}) {
-    if (cand >= best_P) break;
+  const int P0 = std::max<int>(1, (int)((unit_pages + target - 1) / target));
+  int best_P = P0;
+  double best = makespan(P0);
+  std::vector<int> cands = {4, 6, 8, 10, 12, 16, 24, 32, 48, 64, 96, 128};
+  for (int P = P0 + 1; P <= P0 + std::min(P0 / 2 + 1, 24); ++P) cands.push_back(P);
+  for (int cand : cands) {
+    if (cand == P0) continue;
     const double m = makespan(cand);
     if (m < best * 0.999) { best = m; best_P = cand; }
   }

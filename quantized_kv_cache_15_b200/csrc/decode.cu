@@ -226,7 +226,6 @@ size_t decode_smem_bytes(int stage_bytes, int n_stages, int G, bool wtab_smem) {
   a += (size_t)G * 4 * 4;            // qsum
   a += (size_t)G * 4 * 4;            // qsi
   a += (size_t)8 * 4;                // sq
-  a += (size_t)G * D * 2;            // qi16
   a += (size_t)2 * G * 64 * 4;       // pair tables
   a = (a + 15) & ~(size_t)15;
   if (wtab_smem) a += (size_t)NCW * wtab_bytes(G);   // per-warp weight tables
@@ -275,7 +274,9 @@ __device__ void finalize(const DecodeParams& p, const HeadInfo& h, int vbasis, i
   }
 }
 
-template <int G>
+// VA: some kv head of the layer stores V with a _1 codec (scale and minimum), whose
+// offsets need per-block accumulators; layers without one compile those away.
+template <int G, bool VA>
 __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   // launched as a programmatic dependent: the grid is set up while the previous
@@ -331,7 +332,6 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   float* qsum = reinterpret_cast<float*>(smem + off); off += (size_t)G * 4 * 4;
   int* qsi = reinterpret_cast<int*>(smem + off); off += (size_t)G * 4 * 4;
   float* sq = reinterpret_cast<float*>(smem + off); off += (size_t)8 * 4;
-  int16_t* qi16 = reinterpret_cast<int16_t*>(smem + off); off += (size_t)G * D * 2;
   uint32_t* tab = reinterpret_cast<uint32_t*>(smem + off); off += (size_t)2 * G * 64 * 4;
   off = (off + 15) & ~(size_t)15;
   uint64_t* pw2 = reinterpret_cast<uint64_t*>(smem + off);         // per-warp weight tables (p.wtab_smem)
@@ -341,31 +341,42 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   uint64_t* mmerge = full + 16;                                    // the merge's two staging buffers
 
   // The producer sets up the ring and starts the first NS page loads right away,
-  // so they overlap the query preparation below.
+  // so they overlap the query preparation below.  Its 32 lanes read the
+  // block-table entries of 32 tiles at once (lane j: tile i0 + j), so the first
+  // loads do not wait on one another's table reads; lane 0 issues the copies.
   const uint8_t* tail_base =
       is_tail ? p.tail + (((size_t)seq * p.L + p.layer) * p.Hkv + head) * (size_t)T * (D * 2 * 2) : nullptr;
-  auto issue_tile = [&](int i) {
-    const int st = i % NS;
-    const uint8_t* src;
-    if (is_tail) {
-      src = tail_base + (size_t)(pg0 + i) * TAIL_PAGE_BYTES;
-    } else {
-      int pid = p.block_table[(size_t)seq * p.max_pages_per_seq + pg0 + i];
+  auto load_pids = [&](int i0) -> int {
+    int pid = 0;
+    if (!is_tail && i0 + lane < n_tiles) {
+      pid = p.block_table[(size_t)seq * p.max_pages_per_seq + pg0 + i0 + lane];
       if (pid < 0) { atomicOr(p.err, ERR_NO_PAGE); pid = 0; }
-      src = p.pool + (size_t)pid * p.page_bytes + h.off;
     }
+    return pid;
+  };
+  auto issue_tile = [&](int i, int pid) {          // lane 0 of the producer warp
+    const int st = i % NS;
+    const uint8_t* src = is_tail ? tail_base + (size_t)(pg0 + i) * TAIL_PAGE_BYTES
+                                 : p.pool + (size_t)pid * p.page_bytes + h.off;
     // test-only fault injection: the last tile is never loaded, so its consumer's
     // bounded wait runs out (no later tile reuses the stage, no copy is left in flight)
     if (p.drop_last_tile && i == n_tiles - 1) return;
     mbar_arrive_expect_tx(&full[st], tile_bytes);
     bulk_g2s(stages + (size_t)st * p.stage_bytes, src, tile_bytes, &full[st]);
   };
-  if (warp == NCW && lane == 0) {
-    for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    mbar_init(&mmerge[0], 1);
-    mbar_init(&mmerge[1], 1);
-    fence_mbar_init();
-    for (int i = 0; i < NS && i < n_tiles; ++i) issue_tile(i);
+  int pids = 0;                                     // producer: entries of tiles 32k .. 32k+31
+  if (warp == NCW) {
+    pids = load_pids(0);
+    if (lane == 0) {
+      for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+      mbar_init(&mmerge[0], 1);
+      mbar_init(&mmerge[1], 1);
+      fence_mbar_init();
+    }
+    for (int i = 0; i < NS && i < n_tiles; ++i) {  // NS <= 8: all in the first batch
+      const int pid = __shfl_sync(0xffffffffu, pids, i);
+      if (lane == 0) issue_tile(i, pid);
+    }
   }
 
   const bool kfast = kc != KVQ_F16;                 // integer key scores (block and rank codecs)
@@ -405,13 +416,25 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
         const float amax = warp_max(fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3]))));
         const float scale = amax > 0.f ? amax * (1.0f / 32767.0f) : 1.0f;
         const float inv = 1.0f / scale;
+        // each value goes straight to its slots in the pair tables of the K codec's
+        // code planes (tab_slot inverts the order the planes' masks produce)
+        int tt0, tt1;
+        codec_tables(kbits, &tt0, &tt1);
+        uint16_t* tab16 = reinterpret_cast<uint16_t*>(tab);
         int bs = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           int v = __float2int_rn(x[i] * inv);
           v = max(-32767, min(32767, v));
-          qi16[g * D + 4 * lane + i] = (int16_t)v;
           bs += v;
+#pragma unroll
+          for (int plane = 0; plane < 2; ++plane) {
+            const int type = plane ? tt1 : tt0;
+            if (type < 0) continue;
+            int w, half;
+            tab_slot(type, 4 * lane + i, w, half);
+            tab16[((plane * G + g) * 64 + w) * 2 + half] = (uint16_t)(int16_t)v;
+          }
         }
         bs += __shfl_xor_sync(0xffffffffu, bs, 1);
         bs += __shfl_xor_sync(0xffffffffu, bs, 2);
@@ -423,21 +446,6 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   }
   __syncthreads();
 
-  // ---- pair tables of the K codec's code planes (block codecs)
-  if (kfast) {
-    int tt0, tt1;
-    codec_tables(kbits, &tt0, &tt1);
-    for (int idx = threadIdx.x; idx < 2 * G * 64; idx += blockDim.x) {
-      const int plane = idx / (G * 64), rem = idx % (G * 64), g = rem / 64, w = rem % 64;
-      const int type = plane ? tt1 : tt0;
-      if (type < 0) continue;
-      int c0, c1;
-      tab_channels(type, w, c0, c1);
-      tab[idx] = (uint32_t)(uint16_t)qi16[g * D + c0] | ((uint32_t)(uint16_t)qi16[g * D + c1] << 16);
-    }
-    __syncthreads();
-  }
-
   float m[G], l[G], acc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -447,11 +455,13 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   }
   if (warp == NCW) {
     // ---- producer: refill each stage once its consumer warp has released it
-    if (lane == 0) {
-      for (int i = NS; i < n_tiles; ++i) {
+    for (int i = NS; i < n_tiles; ++i) {
+      if ((i & 31) == 0) pids = load_pids(i);
+      const int pid = __shfl_sync(0xffffffffu, pids, i & 31);
+      if (lane == 0) {
         const int st = i % NS;
         if (!mbar_wait(&empty[st], ((i / NS) - 1) & 1, p.wait_ns)) atomicOr(p.err, ERR_TIMEOUT);
-        issue_tile(i);
+        issue_tile(i, pid);
       }
     }
   } else {
@@ -475,7 +485,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     int vclass = 0;
     if (vblock) vclass = (vbits == 8 || vbits == 4 || vbits == 2) ? vbits : (vbits == 6) ? 42 : (vbits == 5) ? 41 : 21;
     else if (vc == KVQ_RANK) vclass = (vbits == 4) ? 40 : (vbits == 3) ? 21 : (vbits == 2) ? 20 : 10;
-    const bool vasym = codec_is_asym(vc);
+    const bool vasym = VA && codec_is_asym(vc);
     const bool kasym = codec_is_asym(kc);
     const float vhalf = vblock ? (float)(1 << (vbits - 1)) : 0.f;
     // the codes' centre on the plane path, the byte offset of the high plane, the
@@ -644,48 +654,44 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   }
   __syncthreads();
 
-  // ---- merge the four warps' states
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    float M = -INFINITY;
-    for (int w = 0; w < NCW; ++w) M = fmaxf(M, mg[((size_t)w * G + g) * (D + 4)]);
-    float L = 0.f;
-    for (int w = 0; w < NCW; ++w) {
-      const float mw = mg[((size_t)w * G + g) * (D + 4)];
-      L += (mw == -INFINITY) ? 0.f : exp2f(mw - M) * mg[((size_t)w * G + g) * (D + 4) + 1];
-    }
-    fm[g] = M; fl[g] = L;
-  }
-  __syncthreads();
+  // ---- merge the consumer warps' states in warp order: one pass over (head,
+  // channel); a single split keeps the result for finalize, any other publishes it
+  // straight to its partial.  Partials are laid out [sequence, kv head][G]
+  // [MAX_SPLITS][PARTIAL_FLOATS], so one head's splits are one contiguous block for
+  // the last CTA's merge below.
+  float* pbase = p.ws + ((size_t)si * p.Hkv + head) * G * MAX_SPLITS * PARTIAL_FLOATS;
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
     const int g = idx / D, c = idx % D;
-    const float M = fm[g];
-    float A = 0.f;
+    float mw[NCW];
+    float M = -INFINITY;
+#pragma unroll
     for (int w = 0; w < NCW; ++w) {
-      const float mw = mg[((size_t)w * G + g) * (D + 4)];
-      if (mw != -INFINITY) A += exp2f(mw - M) * mg[((size_t)w * G + g) * (D + 4) + 4 + c];
+      mw[w] = mg[((size_t)w * G + g) * (D + 4)];
+      M = fmaxf(M, mw[w]);
     }
-    aq[idx] = is_tail ? 0.f : A;
-    at[idx] = is_tail ? A : 0.f;
+    float A = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+      if (mw[w] == -INFINITY) continue;
+      const float f = exp2f(mw[w] - M);
+      L += f * mg[((size_t)w * G + g) * (D + 4) + 1];
+      A += f * mg[((size_t)w * G + g) * (D + 4) + 4 + c];
+    }
+    if (S == 1) {
+      aq[idx] = is_tail ? 0.f : A;
+      at[idx] = is_tail ? A : 0.f;
+      if (c == 0) { fm[g] = M; fl[g] = L; }
+    } else {
+      float* dst = pbase + ((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS;
+      dst[4 + c] = A;
+      if (c == 0) { dst[0] = M; dst[1] = L; }
+    }
   }
   __syncthreads();
-
   if (S == 1) {
     finalize<G>(p, h, vbasis, head, aq, at, fl, out_base);
     return;
   }
-  // ---- publish the partial, take a ticket.  Partials are laid out
-  // [sequence, kv head][G][MAX_SPLITS][PARTIAL_FLOATS], so one head's splits are
-  // one contiguous block for the merge below.
-  float* pbase = p.ws + ((size_t)si * p.Hkv + head) * G * MAX_SPLITS * PARTIAL_FLOATS;
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int g = idx / D, c = idx % D;
-    pbase[((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS + 4 + c] = is_tail ? at[idx] : aq[idx];
-  }
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    pbase[((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS + 0] = fm[g];
-    pbase[((size_t)g * MAX_SPLITS + split) * PARTIAL_FLOATS + 1] = fl[g];
-  }
-  __syncthreads();
   if (threadIdx.x == 0) {
     // release: this CTA's partial (ordered before by the barrier) becomes visible
     // to whichever CTA draws the last ticket; acquire: that CTA sees all others'.
@@ -702,7 +708,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   const uint32_t per_g = (uint32_t)S * PARTIAL_FLOATS * 4;
   const size_t stage_off = (post_bytes(G) + 127) & ~(size_t)127;
   const size_t stage_room = (size_t)(reinterpret_cast<uint8_t*>(full) - smem) - stage_off;   // all dead after the loop
-  const int nbuf = min(min(G, 2), (int)(stage_room / per_g));      // >= 1: see decode_smem_bytes
+  const int nbuf = min(min(G, 2), (int)(stage_room / per_g));      // >= 1: see decode_smem_bytes; 2 barriers
   float* fsc = mg;                                                  // [G][MAX_SPLITS] split factors
   if (threadIdx.x == 0) {
     fence_proxy_async_global();          // the acquired partials, read through the bulk-copy path
@@ -815,10 +821,10 @@ cudaError_t launch_project_query(const DecodeParams& p, cudaStream_t s) {
 
 int decode_max_smem() { return 227 * 1024; }
 
-template <int G>
-static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
+template <int G, bool VA>
+static cudaError_t launch_gv(const DecodeParams& p, int grid_x, cudaStream_t s) {
   const size_t smem = decode_smem_bytes(p.stage_bytes, p.n_stages, G, p.wtab_smem != 0);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<G, VA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid_x, p.Hkv, p.n_seqs);
@@ -830,19 +836,28 @@ static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel<G>, p);
+  e = cudaLaunchKernelEx(&cfg, decode_kernel<G, VA>, p);
   note_launches(1);
   return e;
+}
+
+template <int G>
+static cudaError_t launch_g(const DecodeParams& p, int grid_x, cudaStream_t s) {
+  bool va = false;
+  for (int h = 0; h < p.Hkv; ++h) va = va || codec_is_asym(p.heads[h].vcodec);
+  return va ? launch_gv<G, true>(p, grid_x, s) : launch_gv<G, false>(p, grid_x, s);
 }
 
 // Resident CTAs per SM of the kernel for G heads with `smem` dynamic bytes (registers,
 // shared memory and the thread limit all counted), 0 on error.
 template <int G>
 static int blocks_per_sm_g(size_t smem) {
-  if (cudaFuncSetAttribute(decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  // both variants have the same launch bounds (register cap) and shared memory
+  if (cudaFuncSetAttribute(decode_kernel<G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G>, DECODE_THREADS, smem) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<G, true>, DECODE_THREADS, smem) != cudaSuccess)
+    return 0;
   return n;
 }
 

@@ -19,6 +19,7 @@
 #pragma once
 
 #include "kvq_internal.h"
+#include "pair_tables.h"
 
 namespace kvq {
 
@@ -93,29 +94,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// ---- pair tables: word w of a table packs two int16 query values (low, high)
-enum { TAB_NAT = 0, TAB_Q4 = 1, TAB_Q2 = 2, TAB_Q1 = 3 };
-__device__ __forceinline__ void tab_channels(int type, int w, int& c0, int& c1) {
-  switch (type) {
-    case TAB_NAT: c0 = 2 * w; c1 = c0 + 1; break;                              // bytes in order
-    case TAB_Q4: {                                                              // masks 0x0F0F0F0F, >>4
-      const int k = w >> 2, j = w & 3;
-      c0 = 8 * k + ((j == 0) ? 0 : (j == 1) ? 4 : (j == 2) ? 1 : 5);
-      c1 = c0 + 2;
-    } break;
-    case TAB_Q2: {                                                              // masks 0x03030303, >>2s
-      const int k = w >> 3, j = w & 7, s = j >> 1;
-      c0 = 16 * k + s + ((j & 1) ? 8 : 0);
-      c1 = c0 + 4;
-    } break;
-    default: {                                                                  // masks 0x01010101, >>s
-      const int k = w >> 4, j = w & 15, s = j >> 1;
-      c0 = 32 * k + s + ((j & 1) ? 16 : 0);
-      c1 = c0 + 8;
-    } break;
-  }
-}
-
 // Block epilogue of the integer score: s += (A - half*qsum) * d   (_0)
 //                                     s += A * d + qsum * m       (_1)
 template <int G, bool asym>
@@ -158,7 +136,7 @@ __device__ __forceinline__ void score2_block_codec(int kc, const uint8_t* kp, co
   for (int g = 0; g < G; ++g) { s0[g] = 0.f; s1[g] = 0.f; }
   const int bits = codec_bits(kc);
   const int half = 1 << (bits - 1);
-#pragma unroll 1
+  KVQ_UNROLL(KVQ_SCORE_UNROLL)
   for (int b = 0; b < 4; ++b) {
     int a0[G], a1[G];
 #pragma unroll
@@ -386,20 +364,6 @@ __device__ __forceinline__ void score2_rank(int r, const uint8_t* kp, const uint
   }
 }
 
-// Pair-table layouts of a key codec with `bits` code bits (plane 0, plane 1; -1 = none).
-__host__ __device__ inline void codec_tables(int bits, int* t0, int* t1) {
-  switch (bits) {
-    case 8: *t0 = TAB_NAT; *t1 = -1; break;
-    case 6: *t0 = TAB_Q4; *t1 = TAB_Q2; break;
-    case 5: *t0 = TAB_Q4; *t1 = TAB_Q1; break;
-    case 4: *t0 = TAB_Q4; *t1 = -1; break;
-    case 3: *t0 = TAB_Q2; *t1 = TAB_Q1; break;
-    case 2: *t0 = TAB_Q2; *t1 = -1; break;
-    case 1: *t0 = TAB_Q1; *t1 = -1; break;
-    default: *t0 = -1; *t1 = -1; break;
-  }
-}
-
 // ---- values as integer dot products
 //
 // Per 64-token tile the softmax weight of token t for block b and head g,
@@ -458,7 +422,7 @@ __device__ __forceinline__ void value_dots(const uint8_t* vp, int lane, const ui
                                            int acc[G][4]) {
   constexpr int WRS = wq_row_words<G>();
   constexpr int cbV = 16 * VB;
-#pragma unroll 8
+  KVQ_UNROLL(KVQ_VDOT_UNROLL)
   for (int j = 0; j < 32; ++j) {
     uint32_t X, Y;
     if (VB == 8) {

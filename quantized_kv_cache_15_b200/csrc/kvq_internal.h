@@ -44,8 +44,21 @@ constexpr int PARTIAL_FLOATS = 4 + D;     // m, l, kind, pad, acc[128]
 #endif
 constexpr int NCW = KVQ_DECODE_CONSUMER_WARPS;
 constexpr int DECODE_THREADS = 32 * (NCW + 1);
-// resident CTAs per SM the register allocation aims at
+// resident CTAs per SM the register allocation aims at (a build may fix it)
+#ifdef KVQ_DECODE_MIN_CTAS
+#define DECODE_MIN_CTAS(G) (KVQ_DECODE_MIN_CTAS)
+#else
 #define DECODE_MIN_CTAS(G) ((NCW <= 4) ? ((G) <= 4 ? 3 : 2) : ((G) <= 4 ? 2 : 1))
+#endif
+// unroll factors of the decode inner loops (score blocks, value token pairs)
+#ifndef KVQ_SCORE_UNROLL
+#define KVQ_SCORE_UNROLL 1
+#endif
+#ifndef KVQ_VDOT_UNROLL
+#define KVQ_VDOT_UNROLL 8
+#endif
+#define KVQ_STR_(x) #x
+#define KVQ_UNROLL(n) _Pragma(KVQ_STR_(unroll n))
 
 // Split-K layout of one sequence of `len` tokens, shared by the host (grid size)
 // and the decode kernel: the quantized segment in 64-token pages cut into splits

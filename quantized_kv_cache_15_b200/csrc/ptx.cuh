@@ -49,15 +49,19 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
 // Wait for the phase with the given parity to complete; gives up after limit_ns
 // (2 s by default).  Each try suspends the thread for up to 20 us, so a long wait
 // (a producer whose ring is full, a consumer waiting for its first page) costs a
-// handful of instructions.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
+// handful of instructions.  The slow path is a separate function so that its
+// timer arithmetic takes no registers in the callers' loops.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < (1u << 26); ++i) {
     if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
     if (globaltimer_ns() - t0 > limit_ns) break;
   }
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, limit_ns);
 }
 
 // Bulk copy (TMA, untiled) of `bytes` (multiple of 16, both addresses 16-byte

@@ -1,6 +1,8 @@
-"""Host-side check of the split and causal-visibility arithmetic that decode and
-chunked prefill share (split_counts / tail_visible in the library's internal
-header), compiled with the host compiler and run on the CPU.
+"""Host-side checks of the decode kernel's index arithmetic, compiled with the host
+compiler and run on the CPU: the split and causal-visibility arithmetic that
+decode and chunked prefill share (split_counts / tail_visible in the library's
+internal header), and the pair-table layout of the integer key scores
+(pair_tables.h: tab_slot must invert tab_channels).
 
 For every (len, tail T, visible length lim) the tiles the kernel visits and the
 slots it keeps must cover exactly positions 0 .. lim-1: the quantized pages in
@@ -67,4 +69,46 @@ def test_visited_tiles_cover_exactly_the_visible_prefix(tmp_path):
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr[-2000:]
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout[-500:]
+
+
+TAB_PROGRAM = r'''
+#include <cstdio>
+#include <cuda_runtime.h>
+#include "pair_tables.h"
+using namespace kvq;
+int main() {
+  for (int type = 0; type < 4; ++type) {
+    int seen[128] = {0};
+    for (int w = 0; w < 64; ++w) {
+      int c0, c1, w0, h0, w1, h1;
+      tab_channels(type, w, c0, c1);
+      tab_slot(type, c0, w0, h0);
+      tab_slot(type, c1, w1, h1);
+      if (w0 != w || h0 != 0 || w1 != w || h1 != 1) { printf("type %d word %d\\n", type, w); return 1; }
+      seen[c0]++; seen[c1]++;
+    }
+    for (int c = 0; c < 128; ++c)
+      if (seen[c] != 1) { printf("type %d channel %d seen %d times\\n", type, c, seen[c]); return 1; }
+  }
+  printf("ok\\n");
+  return 0;
+}
+'''
+
+
+def test_pair_table_slots_invert_the_channel_order(tmp_path):
+    """The decode prologue writes each quantized query value straight to the word and
+    half that tab_slot names; the score loop reads word w as the two channels
+    tab_channels names.  Every channel must land in exactly one slot, and the slot
+    must be the one the score loop reads it from, for every plane layout."""
+    if not os.path.isdir(CUDA_INC):
+        pytest.skip("CUDA headers not installed")
+    src = tmp_path / "tab.cpp"
+    src.write_text(TAB_PROGRAM)
+    exe = tmp_path / "tab"
+    r = subprocess.run(["g++", "-O1", "-std=c++17", "-I", CSRC, "-I", CUDA_INC, str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout[-500:]
