@@ -347,6 +347,27 @@ kvq_status kvq_debug_rotate(const kvq_plan* plan, int layer, int head, int kv, i
 kvq_status kvq_debug_quantize_f32(int codec, int r, int b, int n_rows, const float* y, void* codes,
                                   void* scales, int layout, void* stream);
 
+/* Micro-benchmarks of the CUDA-core issue pipes and of a streaming read (no
+ * counterpart in the pages: they measure the ceilings that decode attention on
+ * CUDA cores runs against).  One bounded launch of `ctas` CTAs of 256 threads on
+ * `stream`; the caller times it (events on the same stream) and divides *work by
+ * the time.
+ *  kind: KVQ_UB_FFMA (fp32 fma, work = multiply-adds), KVQ_UB_DP2A (dp2a: 2 per
+ *    instruction), KVQ_UB_DP4A (dp4a: 4), KVQ_UB_FMA2 (fma.rn.f32x2: 2), KVQ_UB_MIX
+ *    (dp2a and fp32 fma one to one: 3 per pair), each thread running `iters`
+ *    rounds of 8 independent chains; KVQ_UB_READ: `iters` passes of 16-byte
+ *    streaming loads over buf (work = bytes read).
+ *  buf: device, 16-byte aligned, buf_bytes >= 16 (KVQ_UB_READ only; else ignored).
+ *  sink: device [ctas * 256] 64-bit words, written (keeps the work alive).
+ *  work: host, the launch's work count.
+ * KVQ_ERR_INVALID_ARG for a bad kind, iters outside [1, 2^20], ctas outside
+ * [1, 65536], or missing buffers; nothing is enqueued then. */
+enum kvq_microbench_kind {
+  KVQ_UB_FFMA = 0, KVQ_UB_DP2A = 1, KVQ_UB_DP4A = 2, KVQ_UB_FMA2 = 3, KVQ_UB_MIX = 4, KVQ_UB_READ = 5
+};
+kvq_status kvq_microbench(int kind, int iters, int ctas, const void* buf, size_t buf_bytes, void* sink,
+                          double* work, void* stream);
+
 /* Fixed split-K size for this plan's decode and prefill calls (test-only; no
  * counterpart in the pages): pages_per_split > 0 cuts every sequence into splits of
  * that many pages (at least as many as the split limit needs); 0 restores the

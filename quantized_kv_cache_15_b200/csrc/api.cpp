@@ -611,14 +611,15 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
     if (m < best * 0.999) { best = m; best_P = cand; }
   }
   std::vector<int> ppq;
-  sizes(best_P, ppq, dp.pps_t);
-  for (int h = 0; h < p->Hkv; ++h) dp.pps_q[h] = (uint16_t)std::min(ppq[h], 65535);
-  for (int i = 0; i < n_seqs; ++i)
-    for (int h = 0; h < p->Hkv; ++h) {
-      const SplitCounts c = split_counts(dp.len[i], (int)p->T, dp.pps_q[h], dp.pps_t, dp.lim[i]);
-      L.grid_x = std::max(L.grid_x, c.qsplits + c.tsplits);
-    }
-  if (L.grid_x > 1 || L.proj) {
+  int ppt = 1;
+  sizes(best_P, ppq, ppt);
+  dp.pps = ppq[0];
+  dp.pps_t = ppt;
+  // CTA order of the launch (decode_item): full quantized splits, partial ones
+  // largest first, tail splits, zero-writing items
+  int max_splits = 0;
+  L.grid_x = build_decode_order(dp, &max_splits);
+  if (max_splits > 1 || L.proj) {
     const size_t need = workspace_bytes(p, n_seqs);
     if (!workspace || workspace_bytes_given < need)
       return fail(KVQ_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes_given);
@@ -918,6 +919,20 @@ kvq_status kvq_check_device_error(kvq_plan* p, void* stream) {
   cudaMemset(p->d_err, 0, sizeof(int));
   if (v & ERR_TIMEOUT) return fail(KVQ_ERR_TIMEOUT, "a bounded wait inside a kernel ran out (error word 0x%x)", v);
   return fail(KVQ_ERR_DEVICE, "a kernel latched device error word 0x%x (1 = missing page)", v);
+}
+
+kvq_status kvq_microbench(int kind, int iters, int ctas, const void* buf, size_t buf_bytes, void* sink, double* work,
+                          void* stream) {
+  if (kind < KVQ_UB_FFMA || kind > KVQ_UB_READ) return fail(KVQ_ERR_INVALID_ARG, "bad micro-benchmark kind %d", kind);
+  if (iters < 1 || iters > (1 << 20)) return fail(KVQ_ERR_INVALID_ARG, "iters must be in [1, 2^20]");
+  if (ctas < 1 || ctas > 65536) return fail(KVQ_ERR_INVALID_ARG, "ctas must be in [1, 65536]");
+  if (!sink || !work) return fail(KVQ_ERR_INVALID_ARG, "null sink or work");
+  if (kind == KVQ_UB_READ && (!buf || buf_bytes < 16 || (uintptr_t)buf % 16))
+    return fail(KVQ_ERR_INVALID_ARG, "the streaming read needs a 16-byte aligned buffer of at least 16 bytes");
+  const cudaError_t e = launch_microbench(kind, iters, buf, buf_bytes, (unsigned long long*)sink, ctas,
+                                          (cudaStream_t)stream, work);
+  if (e != cudaSuccess) return cuda_fail(e, "micro-benchmark launch");
+  return KVQ_OK;
 }
 
 kvq_status kvq_debug_set_decode_split(kvq_plan* p, int pages_per_split) {

@@ -8,10 +8,11 @@
 // is read once, in its packed form, and dequantized in registers.
 // BeeLlama v0.4.0 news, §KV cache 精度尾部: the tail segment is F16.
 //
-// Work split (split-K): grid (split, kv head, sequence).  A sequence's pages are
-// cut into splits: first the quantized pages, pps_q[kv head] per split (heads
-// with more work per page -- higher rank, more bits -- get shorter splits), then
-// the tail pages, pps_t per split (never mixed in one split).  Each CTA:
+// Work split (split-K): a sequence's pages are cut into splits, first the
+// quantized pages, pps per split, then the tail pages, pps_t per split (never
+// mixed in one split).  One CTA per (split, kv head) in a 1-D grid ordered longest
+// first (decode_item), so the CTAs the hardware starts last are the short ones and
+// the launch ends evenly.  Each CTA:
 //   * warp 4 (producer) streams one page-head region per tile into a ring of
 //     shared-memory stages with cp.async.bulk (completion on mbarriers);
 //   * warps 0-3 (consumers) take tiles round-robin, each keeping its own online
@@ -284,22 +285,21 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   griddep_launch_dependents();
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, head = blockIdx.y, si = blockIdx.z;
+  const int head = blockIdx.x % p.Hkv;
+  const DecodeItem it = decode_item(p, blockIdx.x / p.Hkv);
+  const int si = it.si, split = it.split;
   const int seq = p.seq[si], len = p.len[si];
   const int T = p.T;
-  const int pps_q = p.pps_q[head];
-  const SplitCounts sc = split_counts(len, T, pps_q, p.pps_t, p.lim[si]);
+  const SplitCounts sc = split_counts(len, T, p.pps, p.pps_t, p.lim[si]);
   const int nq = sc.nq, nt = sc.nt, NQP = sc.nqp, NTP = sc.ntp, qsplits = sc.qsplits;
   const int S = sc.qsplits + sc.tsplits;
   float* out_base = p.out + ((size_t)si * p.Hq + (size_t)head * G) * D;
-  if (S == 0) {
-    if (split == 0)
-      for (int i = threadIdx.x; i < G * D; i += blockDim.x) out_base[i] = 0.f;
+  if (it.kind == 2) {                              // nothing to attend to: zeros
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) out_base[i] = 0.f;
     return;
   }
-  if (split >= S) return;
-  const bool is_tail = split >= qsplits;
-  const int pps = is_tail ? p.pps_t : pps_q;
+  const bool is_tail = it.kind == 1;
+  const int pps = is_tail ? p.pps_t : p.pps;
   const int pg0 = (is_tail ? split - qsplits : split) * pps;
   const int pg1 = min(pg0 + pps, is_tail ? NTP : NQP);
   const int n_tiles = pg1 - pg0;
@@ -827,7 +827,7 @@ static cudaError_t launch_gv(const DecodeParams& p, int grid_x, cudaStream_t s) 
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<G, VA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid_x, p.Hkv, p.n_seqs);
+  cfg.gridDim = dim3(grid_x, 1, 1);
   cfg.blockDim = dim3(DECODE_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;

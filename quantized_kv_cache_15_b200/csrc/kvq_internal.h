@@ -21,7 +21,11 @@
 // tail does not enlarge the decode kernel's stage ring.
 #pragma once
 
+#include <algorithm>
 #include <cstdint>
+#include <utility>
+#include <vector>
+
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -55,7 +59,7 @@ constexpr int DECODE_THREADS = 32 * (NCW + 1);
 #define KVQ_SCORE_UNROLL 1
 #endif
 #ifndef KVQ_VDOT_UNROLL
-#define KVQ_VDOT_UNROLL 8
+#define KVQ_VDOT_UNROLL 4
 #endif
 #define KVQ_STR_(x) #x
 #define KVQ_UNROLL(n) _Pragma(KVQ_STR_(unroll n))
@@ -203,8 +207,15 @@ struct DecodeParams {
   const float* s_v;              // [Hkv][128] per-channel V multiplier or null
   const float* M;                // projection table (floats), or null
   float qscale;                  // softmax scale * log2(e)
+  int pps;                       // quantized pages per split
   int pps_t;                     // tail pages per split
-  uint16_t pps_q[MAX_HKV];       // quantized pages per split, per kv head (work-balanced)
+  // CTA order of the 1-D grid (see decode_item): every split of every entry, one CTA
+  // per (split, kv head), kv head fastest, longest first.
+  int n_full, n_part, n_tail, n_zero;   // items of each kind
+  int full0[MAX_BATCH + 1];      // prefix sums over entries of their full quantized splits
+  int tail0[MAX_BATCH + 1];      // prefix sums over entries of their tail splits
+  uint8_t part_order[MAX_BATCH]; // entries with a partial quantized split, largest first
+  uint8_t zero_order[MAX_BATCH]; // entries with nothing to attend to
   int stage_bytes;               // bytes of one pipeline stage
   int n_stages;                  // 4 or 8
   int wtab_smem;                 // 1: the weight tables get their own shared memory (some head's K rows are too small)
@@ -220,6 +231,82 @@ struct DecodeParams {
   int len[MAX_BATCH];
   int lim[MAX_BATCH];            // tokens the entry's query sees (len, or fewer for prefill queries)
 };
+
+// The splits of a decode launch in CTA order.  The hardware hands out CTAs in
+// grid order as slots free up, so the order is longest first: all full quantized
+// splits (pps pages each; entry by entry, splits in order), then each entry's
+// partial last quantized split (fewer pages), largest first, then the tail splits
+// (tail pages are 16-row tiles), and last one zero-writing item per entry with
+// nothing to attend to.  Item i of the grid is (decode_item(p, i / Hkv), kv head
+// i % Hkv).  kind: 0 quantized split, 1 tail split (split = index among the
+// entry's splits, quantized first), 2 nothing to attend (write zeros).
+struct DecodeItem { int si, split, kind; };
+__host__ __device__ inline int prefix_find(const int* pre, int n, int q) {
+  // the entry e with pre[e] <= q < pre[e + 1] (pre non-decreasing, pre[0] = 0)
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] <= q) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+__host__ __device__ inline DecodeItem decode_item(const DecodeParams& p, int q) {
+  DecodeItem it;
+  if (q < p.n_full) {
+    it.si = prefix_find(p.full0, p.n_seqs, q);
+    it.split = q - p.full0[it.si];
+    it.kind = 0;
+    return it;
+  }
+  q -= p.n_full;
+  if (q < p.n_part) {
+    it.si = p.part_order[q];
+    it.split = p.full0[it.si + 1] - p.full0[it.si];
+    it.kind = 0;
+    return it;
+  }
+  q -= p.n_part;
+  if (q < p.n_tail) {
+    it.si = prefix_find(p.tail0, p.n_seqs, q);
+    const SplitCounts c = split_counts(p.len[it.si], p.T, p.pps, p.pps_t, p.lim[it.si]);
+    it.split = c.qsplits + (q - p.tail0[it.si]);
+    it.kind = 1;
+    return it;
+  }
+  q -= p.n_tail;
+  it.si = p.zero_order[q];
+  it.split = 0;
+  it.kind = 2;
+  return it;
+}
+
+// Fill the CTA order of a decode launch (the fields decode_item reads) from the
+// entries' lengths, visible lengths and split sizes; returns the grid size (items
+// x kv heads) and the largest split count of one (entry, kv head) in *max_splits.
+inline int build_decode_order(DecodeParams& dp, int* max_splits) {
+  std::vector<std::pair<int, int>> parts;             // (pages of the partial split, entry)
+  int nzero = 0, most = 0;
+  dp.full0[0] = 0;
+  dp.tail0[0] = 0;
+  for (int i = 0; i < dp.n_seqs; ++i) {
+    const SplitCounts c = split_counts(dp.len[i], dp.T, dp.pps, dp.pps_t, dp.lim[i]);
+    const int full = c.nqp / dp.pps, rest = c.nqp % dp.pps;
+    dp.full0[i + 1] = dp.full0[i] + full;
+    dp.tail0[i + 1] = dp.tail0[i] + c.tsplits;
+    if (rest) parts.emplace_back(rest, i);
+    if (c.qsplits + c.tsplits == 0) dp.zero_order[nzero++] = (uint8_t)i;
+    most = std::max(most, c.qsplits + c.tsplits);
+  }
+  std::stable_sort(parts.begin(), parts.end(),
+                   [](const std::pair<int, int>& a, const std::pair<int, int>& b) { return a.first > b.first; });
+  for (size_t k = 0; k < parts.size(); ++k) dp.part_order[k] = (uint8_t)parts[k].second;
+  dp.n_full = dp.full0[dp.n_seqs];
+  dp.n_part = (int)parts.size();
+  dp.n_tail = dp.tail0[dp.n_seqs];
+  dp.n_zero = nzero;
+  *max_splits = most;
+  return (dp.n_full + dp.n_part + dp.n_tail + dp.n_zero) * dp.Hkv;
+}
 
 // ---------------------------------------------------------------- launchers (host)
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
@@ -268,6 +355,8 @@ __host__ __device__ constexpr uint32_t wtab_bytes(int G) { return 32u * (4u * (u
 constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)16 << 20;   // = KVQ_NOALLOC_SCRATCH_BYTES
 cudaError_t noalloc_scratch(int device, void** out);
 void note_launches(int n);   // counts kernel launches made by the library
+cudaError_t launch_microbench(int kind, int iters, const void* buf, size_t buf_bytes, unsigned long long* sink,
+                              int ctas, cudaStream_t s, double* work);
 int decode_max_smem();
 
 }  // namespace kvq

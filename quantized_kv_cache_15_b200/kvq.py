@@ -58,6 +58,7 @@ SIGNATURES = {
     "kvq_debug_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "kvq_debug_quantize_f32": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P]),
     "kvq_debug_set_decode_split": (_I, [_P, _I]),
+    "kvq_microbench": (_I, [_I, _I, _I, _P, _SZ, _P, ctypes.POINTER(ctypes.c_double), _P]),
     "kvq_debug_fault_injection": (_I, [_P, _I64, _I]),
 }
 
@@ -289,6 +290,19 @@ def vbr_next(k_codec, v_codec, bytes_in_use: int, budget: int, floor_codec: int)
     if st != 0:
         raise KVQError(st, "kvq_vbr_next: codecs off the ladder or bad arguments")
     return layer.value, nk.tolist(), nv.tolist()
+
+
+UB_FFMA, UB_DP2A, UB_DP4A, UB_FMA2, UB_MIX, UB_READ = range(6)   # kvq_microbench_kind
+
+
+def microbench(kind: int, iters: int, ctas: int, sink: torch.Tensor, buf: Optional[torch.Tensor] = None,
+               stream=None) -> float:
+    """Enqueue one micro-benchmark launch; returns its work count (multiply-adds or bytes)."""
+    work = ctypes.c_double()
+    nbytes = 0 if buf is None else buf.numel() * buf.element_size()
+    _check(lib().kvq_microbench(kind, iters, ctas, _ptr(buf), nbytes, _ptr(sink), ctypes.byref(work),
+                                _stream(stream)))
+    return work.value
 
 
 def launch_count() -> int:

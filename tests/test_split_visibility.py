@@ -112,3 +112,88 @@ def test_pair_table_slots_invert_the_channel_order(tmp_path):
     assert r.returncode == 0, r.stderr[-2000:]
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout[-500:]
+
+
+ORDER_PROGRAM = r'''
+#include <cstdio>
+#include <cstdlib>
+#include <vector>
+#include "kvq_internal.h"
+using namespace kvq;
+int main() {
+  unsigned rng = 12345u;
+  auto rnd = [&](int n) { rng = rng * 1103515245u + 12345u; return (int)((rng >> 8) % (unsigned)n); };
+  long checked = 0;
+  for (int trial = 0; trial < 400; ++trial) {
+    static DecodeParams dp;
+    dp.n_seqs = 1 + rnd(trial < 200 ? 8 : MAX_BATCH);
+    dp.Hkv = 1 + rnd(4);
+    const int tails[] = {0, 64, 256, 1024};
+    dp.T = tails[rnd(4)];
+    dp.pps = 1 + rnd(40);
+    dp.pps_t = 1 + rnd(8);
+    for (int i = 0; i < dp.n_seqs; ++i) {
+      dp.len[i] = rnd(5) == 0 ? 0 : rnd(6000);
+      dp.lim[i] = rnd(3) == 0 ? rnd(dp.len[i] + 1) : dp.len[i];
+    }
+    int most = 0;
+    const int grid = build_decode_order(dp, &most);
+    std::vector<std::vector<int>> seen(dp.n_seqs * dp.Hkv);
+    int prev_pages = 1 << 30, prev_kind = 0;
+    for (int b = 0; b < grid; ++b) {
+      const int head = b % dp.Hkv;
+      const DecodeItem it = decode_item(dp, b / dp.Hkv);
+      if (it.si < 0 || it.si >= dp.n_seqs) { printf("entry out of range\\n"); return 1; }
+      const SplitCounts c = split_counts(dp.len[it.si], dp.T, dp.pps, dp.pps_t, dp.lim[it.si]);
+      const int S = c.qsplits + c.tsplits;
+      if (it.kind == 2) {
+        if (S != 0) { printf("zero item for an entry with splits\\n"); return 1; }
+        seen[it.si * dp.Hkv + head].push_back(-1);
+        continue;
+      }
+      if (it.split < 0 || it.split >= S || (it.kind == 1) != (it.split >= c.qsplits)) {
+        printf("bad split %d of %d (kind %d)\\n", it.split, S, it.kind); return 1;
+      }
+      seen[it.si * dp.Hkv + head].push_back(it.split);
+      // quantized splits come longest first, then the tail splits
+      if (it.kind == 0) {
+        const int pages = std::min(dp.pps, c.nqp - it.split * dp.pps);
+        if (prev_kind == 1 || pages > prev_pages) { printf("quantized split out of order\\n"); return 1; }
+        prev_pages = pages;
+      }
+      prev_kind = it.kind;
+    }
+    for (int i = 0; i < dp.n_seqs; ++i)
+      for (int h = 0; h < dp.Hkv; ++h) {
+        const SplitCounts c = split_counts(dp.len[i], dp.T, dp.pps, dp.pps_t, dp.lim[i]);
+        const int S = c.qsplits + c.tsplits;
+        std::vector<int>& v = seen[i * dp.Hkv + h];
+        std::sort(v.begin(), v.end());
+        if (S == 0) { if (v.size() != 1 || v[0] != -1) { printf("empty entry not zeroed once\\n"); return 1; } continue; }
+        if ((int)v.size() != S) { printf("entry %d head %d: %zu of %d splits\\n", i, h, v.size(), S); return 1; }
+        for (int k = 0; k < S; ++k) if (v[k] != k) { printf("split %d missing\\n", k); return 1; }
+        if (S > most) { printf("max splits wrong\\n"); return 1; }
+        ++checked;
+      }
+  }
+  printf("ok %ld\\n", checked);
+  return 0;
+}
+'''
+
+
+def test_cta_order_covers_every_split_once_longest_first(tmp_path):
+    """The decode launch's 1-D grid (build_decode_order / decode_item) gives every
+    (entry, kv head, split) exactly one CTA, quantized splits in non-increasing page
+    count and then the tail splits, and exactly one zero-writing CTA per (entry, kv
+    head) with nothing to attend to, for random batches of lengths and split sizes."""
+    if not os.path.isdir(CUDA_INC):
+        pytest.skip("CUDA headers not installed")
+    src = tmp_path / "order.cpp"
+    src.write_text(ORDER_PROGRAM)
+    exe = tmp_path / "order"
+    r = subprocess.run(["g++", "-O1", "-std=c++17", "-I", CSRC, "-I", CUDA_INC, str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout[-500:]
