@@ -331,8 +331,9 @@ enum kvq_row_layout { KVQ_ROWS_WARP = 0, KVQ_ROWS_QUAD = 1 };
 
 /* Rows in the stored basis, fp32, exactly as the append path computes them
  * before quantization: the staged Hadamard transform (after variance
- * normalisation) for rotated codecs, z = M_h x on the tensor cores for the
- * projection path, the raw values for F16.
+ * normalisation) for rotated codecs, z = M_h x for the projection path (the
+ * exact products summed over the channels in order in double, rounded once to
+ * fp32), the raw values for F16.
  *  x: device raw rows in the plan's kv dtype [n][128];  y: device fp32 [n][128] (or [n][r]).
  *  layout: kvq_row_layout (ignored for the projection path). */
 kvq_status kvq_debug_rotate(const kvq_plan* plan, int layer, int head, int kv, int n, const void* x,

@@ -450,7 +450,7 @@ void orc_varnorm_inv_rms(int64_t n_tok, int n_ch, int64_t stride, const uint16_t
 
 /* ------------------------------------------------------------------------- */
 /* Rotation fused into the per-head projection [COBRA §The news, last but one */
-/* paragraph: "fused into the same projection matrix"]; R12                   */
+/* paragraph: the rotation is folded into the head's projection matrix]; R12  */
 /* ------------------------------------------------------------------------- */
 
 /* M = R_r P^T, with P the 128 x r orthonormal basis of the head (row-major

@@ -73,7 +73,7 @@ __device__ __forceinline__ bool row_work(const AppendParams& p, long task, RowWo
     if (k < sq.nE) return false;                 // the E row of this slot writes it
     w.write_slot = slot; w.write_row = sq.in_row0 + (f - sq.len_old);
   }
-  // rank-codec rows are quantized by the tensor-core kernel, which runs first
+  // rank-codec rows are quantized by the projection kernel, which runs first
   const HeadInfo& h = p.heads[w.head];
   if ((w.kv ? h.vcodec : h.kcodec) == KVQ_RANK) w.pos = -1;
   return true;

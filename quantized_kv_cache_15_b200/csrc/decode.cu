@@ -285,9 +285,8 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   griddep_launch_dependents();
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.x % p.Hkv;
-  const DecodeItem it = decode_item(p, blockIdx.x / p.Hkv);
-  const int si = it.si, split = it.split;
+  const DecodeItem it = decode_item(p, blockIdx.x);
+  const int si = it.si, head = it.head, split = it.split;
   const int seq = p.seq[si], len = p.len[si];
   const int T = p.T;
   const SplitCounts sc = split_counts(len, T, p.pps, p.pps_t, p.lim[si]);
@@ -354,8 +353,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     }
     return pid;
   };
-  auto issue_tile = [&](int i, int pid) {          // lane 0 of the producer warp
-    const int st = i % NS;
+  auto issue_tile = [&](int i, int st, int pid) {  // lane 0 of the producer warp; st = i % NS
     const uint8_t* src = is_tail ? tail_base + (size_t)(pg0 + i) * TAIL_PAGE_BYTES
                                  : p.pool + (size_t)pid * p.page_bytes + h.off;
     // test-only fault injection: the last tile is never loaded, so its consumer's
@@ -375,7 +373,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     }
     for (int i = 0; i < NS && i < n_tiles; ++i) {  // NS <= 8: all in the first batch
       const int pid = __shfl_sync(0xffffffffu, pids, i);
-      if (lane == 0) issue_tile(i, pid);
+      if (lane == 0) issue_tile(i, i, pid);
     }
   }
 
@@ -455,14 +453,16 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   }
   if (warp == NCW) {
     // ---- producer: refill each stage once its consumer warp has released it
+    // stage and empty-barrier phase of tile i, kept incrementally (no division)
+    int st = 0, ph = 0;
     for (int i = NS; i < n_tiles; ++i) {
       if ((i & 31) == 0) pids = load_pids(i);
       const int pid = __shfl_sync(0xffffffffu, pids, i & 31);
       if (lane == 0) {
-        const int st = i % NS;
-        if (!mbar_wait(&empty[st], ((i / NS) - 1) & 1, p.wait_ns)) atomicOr(p.err, ERR_TIMEOUT);
-        issue_tile(i, pid);
+        if (!mbar_wait(&empty[st], ph, p.wait_ns, 1024)) atomicOr(p.err, ERR_TIMEOUT);
+        issue_tile(i, st, pid);
       }
+      if (++st == NS) { st = 0; ph ^= 1; }
     }
   } else {
     // ---- consumers
@@ -507,9 +507,11 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     // 0xF0F0F0F0 and 0x80808080 as run-time values (n_seqs >= 0, so rz == 0)
     const uint32_t rz = (uint32_t)p.n_seqs >> 31;
     const uint32_t kM = 0xF0F0F0F0u ^ rz, kC = 0x80808080u ^ rz;
-    for (int i = warp; i < n_tiles; i += NCW) {
-      const int st = i % NS;
-      if (!mbar_wait(&full[st], (i / NS) & 1, p.wait_ns)) atomicOr(p.err, ERR_TIMEOUT);
+    // stage and full-barrier phase of tile i, kept incrementally: tile i sits in stage
+    // i % NS, phase (i / NS) & 1; warp w takes tiles w, w + NCW, ... and NCW <= NS
+    int st = warp, ph = 0;
+    for (int i = warp; i < n_tiles; i += NCW, st += NCW, ph ^= (st >= NS) ? 1 : 0, st -= (st >= NS) ? NS : 0) {
+      if (!mbar_wait(&full[st], ph, p.wait_ns)) atomicOr(p.err, ERR_TIMEOUT);
       const uint8_t* sp = stages + (size_t)st * p.stage_bytes;
       const uint8_t* kp = sp;
       const uint8_t* ks = kp + rows * cbK;

@@ -234,13 +234,15 @@ struct DecodeParams {
 
 // The splits of a decode launch in CTA order.  The hardware hands out CTAs in
 // grid order as slots free up, so the order is longest first: all full quantized
-// splits (pps pages each; entry by entry, splits in order), then each entry's
-// partial last quantized split (fewer pages), largest first, then the tail splits
-// (tail pages are 16-row tiles), and last one zero-writing item per entry with
-// nothing to attend to.  Item i of the grid is (decode_item(p, i / Hkv), kv head
-// i % Hkv).  kind: 0 quantized split, 1 tail split (split = index among the
-// entry's splits, quantized first), 2 nothing to attend (write zeros).
-struct DecodeItem { int si, split, kind; };
+// splits (pps pages each; entry by entry, kv head by kv head, splits in order, so
+// that the CTAs of one wave mix the heads of an entry, whose per-tile costs can
+// differ), then each entry's partial last quantized split (fewer pages), largest
+// first, then the tail splits (tail pages are 16-row tiles), and last one
+// zero-writing item per entry with nothing to attend to; after the full splits,
+// the kv head varies fastest.  kind: 0 quantized split, 1 tail split (split =
+// index among the entry's splits, quantized first), 2 nothing to attend (write
+// zeros).
+struct DecodeItem { int si, head, split, kind; };
 __host__ __device__ inline int prefix_find(const int* pre, int n, int q) {
   // the entry e with pre[e] <= q < pre[e + 1] (pre non-decreasing, pre[0] = 0)
   int lo = 0, hi = n - 1;
@@ -250,15 +252,19 @@ __host__ __device__ inline int prefix_find(const int* pre, int n, int q) {
   }
   return lo;
 }
-__host__ __device__ inline DecodeItem decode_item(const DecodeParams& p, int q) {
+__host__ __device__ inline DecodeItem decode_item(const DecodeParams& p, int b) {
   DecodeItem it;
-  if (q < p.n_full) {
-    it.si = prefix_find(p.full0, p.n_seqs, q);
-    it.split = q - p.full0[it.si];
+  if (b < p.n_full * p.Hkv) {
+    it.si = prefix_find(p.full0, p.n_seqs, b / p.Hkv);
+    const int full = p.full0[it.si + 1] - p.full0[it.si];
+    const int j = b - p.full0[it.si] * p.Hkv;
+    it.head = j / full;
+    it.split = j - it.head * full;
     it.kind = 0;
     return it;
   }
-  q -= p.n_full;
+  it.head = b % p.Hkv;
+  int q = b / p.Hkv - p.n_full;
   if (q < p.n_part) {
     it.si = p.part_order[q];
     it.split = p.full0[it.si + 1] - p.full0[it.si];

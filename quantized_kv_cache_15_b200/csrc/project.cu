@@ -17,9 +17,10 @@
 //
 // One CTA: one (kv head, K|V) and up to 64 rows.  M_h^T (double, [128][r]) and
 // the rows (double, [64][128]) are staged in shared memory; warp w takes rows w,
-// w + 8, ... two at a time, lane l holds outputs 4l .. 4l+3 of both (eight
-// independent FMA chains over c), and the warp then quantizes each row with the
-// same warp quantizer as the rotation path (lane l: values 4l .. 4l+3).
+// w + 8, ... four at a time, lane l holds outputs 4l .. 4l+3 of all four (sixteen
+// independent FMA chains over c, each M_h^T load shared by four rows), and the
+// warp then quantizes each row with the same warp quantizer as the rotation path
+// (lane l: values 4l .. 4l+3).
 #include "kvq_internal.h"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -115,36 +116,46 @@ __global__ void __launch_bounds__(PJ_THREADS, 1) proj_kernel(const __grid_consta
 
   const int i0 = 4 * lane;
   const bool own = i0 < r;
-  for (int k = 0; k < PJ_ROWS / (2 * PJ_WARPS); ++k) {
-    const int ra = warp + 2 * PJ_WARPS * k, rb = ra + PJ_WARPS;
-    const bool va = rpos[ra] >= 0, vb = rpos[rb] >= 0;
-    if (!va && !vb) continue;                             // warp-uniform
-    double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
+  constexpr int RPP = 4;                                  // rows per pass of a warp
+  for (int k = 0; k < PJ_ROWS / (RPP * PJ_WARPS); ++k) {
+    int rows[RPP];
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < RPP; ++j) {
+      rows[j] = warp + PJ_WARPS * (RPP * k + j);
+      any = any || rpos[rows[j]] >= 0;
+    }
+    if (!any) continue;                                   // warp-uniform
+    double acc[RPP][4];
+#pragma unroll
+    for (int j = 0; j < RPP; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.0;
     if (own) {
-      const double* xa = xs + (size_t)ra * D;
-      const double* xb = xs + (size_t)rb * D;
-#pragma unroll 4
+#pragma unroll 2
       for (int c = 0; c < D; ++c) {
         const double2 m01 = *reinterpret_cast<const double2*>(mt + (size_t)c * r + i0);
         const double2 m23 = *reinterpret_cast<const double2*>(mt + (size_t)c * r + i0 + 2);
-        const double x0 = xa[c], x1 = xb[c];
-        a[0] = fma(m01.x, x0, a[0]); a[1] = fma(m01.y, x0, a[1]);
-        a[2] = fma(m23.x, x0, a[2]); a[3] = fma(m23.y, x0, a[3]);
-        b[0] = fma(m01.x, x1, b[0]); b[1] = fma(m01.y, x1, b[1]);
-        b[2] = fma(m23.x, x1, b[2]); b[3] = fma(m23.y, x1, b[3]);
+#pragma unroll
+        for (int j = 0; j < RPP; ++j) {
+          const double x = xs[(size_t)rows[j] * D + c];
+          acc[j][0] = fma(m01.x, x, acc[j][0]); acc[j][1] = fma(m01.y, x, acc[j][1]);
+          acc[j][2] = fma(m23.x, x, acc[j][2]); acc[j][3] = fma(m23.y, x, acc[j][3]);
+        }
       }
     }
-    for (int which = 0; which < 2; ++which) {
-      const int row = which ? rb : ra;
+#pragma unroll
+    for (int j = 0; j < RPP; ++j) {
+      const int row = rows[j];
       const int pos = rpos[row];
       if (pos < 0) continue;                              // warp-uniform
       float z[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) z[j] = own ? (float)(which ? b[j] : a[j]) : 0.f;
+      for (int e = 0; e < 4; ++e) z[e] = own ? (float)acc[j][e] : 0.f;
       if (p.z_out) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (i0 + j < r) p.z_out[(size_t)pos * r + i0 + j] = z[j];
+        for (int e = 0; e < 4; ++e)
+          if (i0 + e < r) p.z_out[(size_t)pos * r + i0 + e] = z[e];
         continue;
       }
       const int pid = p.block_table[(size_t)rseq[row] * p.max_pages_per_seq + pos / PAGE];

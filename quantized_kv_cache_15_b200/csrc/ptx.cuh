@@ -35,33 +35,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// try_wait that may keep the thread suspended for up to `hint_ns` (it resumes as
-// soon as the phase completes), so a waiting warp takes no issue slots meanwhile.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 // Wait for the phase with the given parity to complete; gives up after limit_ns
-// (2 s by default).  Each try suspends the thread for up to 20 us, so a long wait
-// (a producer whose ring is full, a consumer waiting for its first page) costs a
-// handful of instructions.  The slow path is a separate function so that its
-// timer arithmetic takes no registers in the callers' loops.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+// (2 s by default).  A thread that expects a long wait (a producer whose ring is
+// full while the consumers compute) passes max_sleep_ns > 0: between tries it then
+// sleeps, 64 ns at first and doubling up to max_sleep_ns, so that it takes few issue
+// slots from the warps that share its scheduler.  Others retry at once (try_wait
+// itself blocks for a short while), so they resume as soon as the phase completes.
+// The timer is read every 16 tries.  The slow path is a separate function so that
+// it takes no registers in the callers' loops.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                   uint32_t max_sleep_ns) {
   const uint64_t t0 = globaltimer_ns();
+  uint32_t sleep_ns = 64;
   for (uint32_t i = 0; i < (1u << 26); ++i) {
-    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) break;
+    if (max_sleep_ns) {
+      __nanosleep(sleep_ns);
+      if (sleep_ns < max_sleep_ns) sleep_ns <<= 1;
+    }
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15) == 15 && globaltimer_ns() - t0 > limit_ns) break;
   }
   return false;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull,
+                                          uint32_t max_sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, limit_ns);
+  return mbar_wait_slow(bar, parity, limit_ns, max_sleep_ns);
 }
 
 // Bulk copy (TMA, untiled) of `bytes` (multiple of 16, both addresses 16-byte

@@ -36,7 +36,7 @@ def _time(kind, iters, ctas, sink, buf=None):
 def test_alu_rates(kind, name, lo):
     ctas = 148 * 8
     sink = torch.zeros(ctas * 256, dtype=torch.int64, device="cuda")
-    work, ms = _time(kind, 256, ctas, sink)
+    work, ms = _time(kind, 4096, ctas, sink)
     rate = work / (ms / 1e3)
     print(f"ubench {name} {rate / 1e12:.2f} Tmul-add/s ({work:.3e} in {ms:.3f} ms, {ctas} CTAs)")
     assert lo * NOMINAL_FMA_PER_S < rate < 8 * NOMINAL_FMA_PER_S

@@ -141,8 +141,9 @@ int main() {
     std::vector<std::vector<int>> seen(dp.n_seqs * dp.Hkv);
     int prev_pages = 1 << 30, prev_kind = 0;
     for (int b = 0; b < grid; ++b) {
-      const int head = b % dp.Hkv;
-      const DecodeItem it = decode_item(dp, b / dp.Hkv);
+      const DecodeItem it = decode_item(dp, b);
+      const int head = it.head;
+      if (head < 0 || head >= dp.Hkv) { printf("head out of range\\n"); return 1; }
       if (it.si < 0 || it.si >= dp.n_seqs) { printf("entry out of range\\n"); return 1; }
       const SplitCounts c = split_counts(dp.len[it.si], dp.T, dp.pps, dp.pps_t, dp.lim[it.si]);
       const int S = c.qsplits + c.tsplits;
