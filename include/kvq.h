@@ -197,9 +197,14 @@ kvq_status kvq_decode_attention(kvq_plan* plan, int layer, int n_seqs, const int
  *  q:   device raw dtype [n_q][n_q_heads][128];  out: device fp32 [n_q][n_q_heads][128]
  *  workspace: kvq_plan_workspace_bytes(plan, min(n_q, KVQ_MAX_BATCH)), zeroed before
  *    first use (the calls leave it ready for reuse).
- * Each query runs the split-K decode kernel over its visible prefix, KVQ_MAX_BATCH
- * queries per launch; keys and values are not shared between the queries of a
- * launch (beyond what L2 keeps).  KVQ_ERR_INVALID_ARG if n_q exceeds the length. */
+ * Layers whose heads all use block codecs (no F16 pages, no rank codec) under a
+ * rotation other than the projection run on the tensor cores: a CTA takes
+ * 128 / G consecutive queries of one kv head and dequantizes each 64-token
+ * key/value tile once for all of them (keys and the query as fp16 hi + lo pairs,
+ * values and softmax weights as fp16, fp32 accumulation; q and out 16-byte
+ * aligned; the workspace is not used).  Other layers run each query through the
+ * split-K decode kernel over its visible prefix, KVQ_MAX_BATCH queries per launch.
+ * KVQ_ERR_INVALID_ARG if n_q exceeds the length. */
 kvq_status kvq_prefill_attention(kvq_plan* plan, int layer, int seq_id, int n_q, const void* q, float* out,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
@@ -375,6 +380,11 @@ kvq_status kvq_microbench(int kind, int iters, int ctas, const void* buf, size_t
  * automatic choice.  The merge order is fixed either way, so results differ only
  * by the rounding of the merge.  KVQ_ERR_INVALID_ARG for a negative count. */
 kvq_status kvq_debug_set_decode_split(kvq_plan* plan, int pages_per_split);
+
+/* Prefill path selection (test-only; no counterpart in the pages): path 0 (the
+ * default) uses the tensor-core prefill wherever the layer allows it, path 1
+ * always runs the decode kernel per query.  KVQ_ERR_INVALID_ARG for other values. */
+kvq_status kvq_debug_set_prefill_path(kvq_plan* plan, int path);
 
 /* Failure injection for the failure-path tests (test-only; no counterpart in the
  * pages).  wait_limit_ns: every bounded wait inside this plan's decode kernels

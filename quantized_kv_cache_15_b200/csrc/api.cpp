@@ -76,6 +76,7 @@ struct kvq_plan {
   int debug_pps = 0;                          // fixed pages per split, 0 = chosen per call
   unsigned long long wait_ns = 2000000000ull; // give-up time of the kernels' bounded waits
   int drop_last_tile = 0;                     // decode producers skip their last tile
+  int prefill_path = 0;                       // 0: tensor cores where the layer allows, 1: decode kernel
 
   ~kvq_plan() {
     int prev = 0;
@@ -659,6 +660,28 @@ kvq_status kvq_decode_attention(kvq_plan* p, int layer, int n_seqs, const int* s
   return decode_launch(p, layer, n_seqs, seq_ids, nullptr, q, out, workspace, workspace_bytes_given, stream);
 }
 
+// The tensor-core prefill takes a layer whose heads all store block codecs (the
+// kernel dequantizes 32-value blocks; F16 pages and the rank codec go through the
+// decode kernel) under a rotation other than the projection, when two raw stages
+// of the largest page-head fit beside its operand buffers.
+static bool prefill_tc_layout(const kvq_plan* p, int layer, int* stage_bytes, int* n_raw) {
+  if (p->rot == KVQ_ROT_PROJECTION) return false;
+  int sb = 0;
+  for (int h = 0; h < p->Hkv; ++h) {
+    const HeadInfo& hi = p->head(layer, h);
+    for (int c : {(int)hi.kcodec, (int)hi.vcodec})
+      if (c == KVQ_F16 || c == KVQ_RANK) return false;
+    if (hi.cbK % 16 || hi.cbV % 16 || hi.off % 16 || hi.bytes % 16) return false;
+    sb = std::max(sb, (int)hi.bytes);
+  }
+  sb = (sb + 127) & ~127;
+  const int n = prefill_raw_stages(sb);
+  if (n < 2) return false;
+  *stage_bytes = sb;
+  *n_raw = n;
+  return true;
+}
+
 kvq_status kvq_prefill_attention(kvq_plan* p, int layer, int seq_id, int n_q, const void* q, float* out,
                                  void* workspace, size_t workspace_bytes_given, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
@@ -669,6 +692,41 @@ kvq_status kvq_prefill_attention(kvq_plan* p, int layer, int seq_id, int n_q, co
   if (n_q < 0 || n_q > len) return fail(KVQ_ERR_INVALID_ARG, "n_q %d outside [0, %lld]", n_q, (long long)len);
   if (n_q == 0) return KVQ_OK;
   if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "null q or out");
+  int stage_bytes = 0, n_raw = 0;
+  if (p->prefill_path == 0 && prefill_tc_layout(p, layer, &stage_bytes, &n_raw)) {
+    if (((uintptr_t)q % 16) || ((uintptr_t)out % 16)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+    const DecodeParams dp = p->base_params(layer);
+    PrefillParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.pool = dp.pool;
+    pp.page_bytes = dp.page_bytes;
+    pp.bt = p->d_bt + (size_t)seq_id * p->mpps;
+    pp.ring = dp.tail + ((size_t)seq_id * p->L + layer) * p->Hkv * (size_t)p->T * (D * 2 * 2);
+    pp.T = (int)p->T;
+    pp.len = (int)len;
+    pp.nq_all = len > p->T ? (int)(len - p->T) : 0;
+    pp.n_q = n_q;
+    pp.Hq = p->Hq;
+    pp.Hkv = p->Hkv;
+    pp.G = p->G;
+    pp.QB = 128 / p->G;
+    pp.rot = p->rot;
+    pp.bf16 = p->bf16;
+    pp.q = (const __half*)q;
+    pp.out = out;
+    pp.s_k = dp.s_k;
+    pp.s_v = dp.s_v;
+    pp.inv_s = (p->rot == KVQ_ROT_VARNORM_HADAMARD && p->d_inv) ? p->d_inv + (size_t)layer * p->Hkv * 2 * D : nullptr;
+    pp.qscale = dp.qscale;
+    pp.stage_bytes = stage_bytes;
+    pp.n_raw = n_raw;
+    pp.err = dp.err;
+    pp.wait_ns = dp.wait_ns;
+    for (int h = 0; h < p->Hkv; ++h) pp.heads[h] = dp.heads[h];
+    cudaError_t e = launch_prefill(pp, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    return KVQ_OK;
+  }
   int ids[MAX_BATCH], lims[MAX_BATCH];
   for (int c0 = 0; c0 < n_q; c0 += MAX_BATCH) {
     const int n = std::min(MAX_BATCH, n_q - c0);
@@ -932,6 +990,13 @@ kvq_status kvq_microbench(int kind, int iters, int ctas, const void* buf, size_t
   const cudaError_t e = launch_microbench(kind, iters, buf, buf_bytes, (unsigned long long*)sink, ctas,
                                           (cudaStream_t)stream, work);
   if (e != cudaSuccess) return cuda_fail(e, "micro-benchmark launch");
+  return KVQ_OK;
+}
+
+kvq_status kvq_debug_set_prefill_path(kvq_plan* p, int path) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (path != 0 && path != 1) return fail(KVQ_ERR_INVALID_ARG, "path must be 0 or 1");
+  p->prefill_path = path;
   return KVQ_OK;
 }
 

@@ -365,4 +365,35 @@ cudaError_t launch_microbench(int kind, int iters, const void* buf, size_t buf_b
                               int ctas, cudaStream_t s, double* work);
 int decode_max_smem();
 
+// ---------------------------------------------------------------- prefill (tensor cores)
+// Causal attention of the last n_q tokens of one sequence over one layer's cache:
+// a CTA takes QB = 128 / G consecutive queries of one kv head (rows j*G + g), and
+// every key/value tile of 64 positions is dequantized once per CTA into fp16
+// operands for tcgen05.mma.  Layers whose heads all use block codecs (not F16,
+// not the rank codec) and a rotation other than the projection take this path.
+struct PrefillParams {
+  const uint8_t* pool;           // the layer's page pool
+  uint32_t page_bytes;
+  const int* bt;                 // the sequence's block-table row
+  const uint8_t* ring;           // tail ring of (sequence, layer, kv head 0); heads T*512 bytes apart
+  int T;                         // tail length (ring slots)
+  int nq_all;                    // quantized rows of the sequence (len - T, or 0)
+  int len, n_q, Hq, Hkv, G, QB;
+  int rot, bf16;
+  const __half* q;               // [n_q][Hq][128] raw 16-bit
+  float* out;                    // [n_q][Hq][128]
+  const float* s_k;              // [Hkv][128] or null (variance normalisation)
+  const float* s_v;
+  const float* inv_s;            // [Hkv][2][128] or null: the append's multipliers (tail rows)
+  float qscale;                  // softmax scale * log2(e)
+  int stage_bytes;               // raw page-head stage (multiple of 128)
+  int n_raw;                     // raw stages (2..4)
+  int* err;
+  unsigned long long wait_ns;
+  HeadInfo heads[MAX_HKV];
+};
+size_t prefill_smem_bytes(int stage_bytes, int n_raw);
+int prefill_raw_stages(int stage_bytes);     // stages that fit, 0 if fewer than two
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t s);
+
 }  // namespace kvq

@@ -58,6 +58,7 @@ SIGNATURES = {
     "kvq_debug_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "kvq_debug_quantize_f32": (_I, [_I, _I, _I, _I, _P, _P, _P, _I, _P]),
     "kvq_debug_set_decode_split": (_I, [_P, _I]),
+    "kvq_debug_set_prefill_path": (_I, [_P, _I]),
     "kvq_microbench": (_I, [_I, _I, _I, _P, _SZ, _P, ctypes.POINTER(ctypes.c_double), _P]),
     "kvq_debug_fault_injection": (_I, [_P, _I64, _I]),
 }
@@ -250,6 +251,10 @@ class Plan:
     def debug_set_decode_split(self, pages_per_split: int):
         """Test-only: fixed pages per split-K piece (0 = automatic)."""
         _check(lib().kvq_debug_set_decode_split(self._h, pages_per_split))
+
+    def debug_set_prefill_path(self, path: int):
+        """Test-only: 0 = tensor-core prefill where the layer allows it, 1 = decode kernel."""
+        _check(lib().kvq_debug_set_prefill_path(self._h, int(path)))
 
     def debug_fault_injection(self, wait_limit_ns: int = 2_000_000_000, drop_last_tile: bool = False):
         """Test-only: bounded-wait limit of the decode kernels and dropped last tiles."""
