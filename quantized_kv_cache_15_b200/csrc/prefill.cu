@@ -60,17 +60,20 @@ namespace {
 constexpr int PF_ROWS = 128;
 constexpr int PF_TOK = 64;
 constexpr int PF_THREADS = 320;
-constexpr int PF_Q_BYTES = PF_ROWS * D * 2;            // one fp16 image of the 128 query rows
 constexpr int PF_TILE_BYTES = PF_TOK * D * 2;          // one fp16 image of a 64-token tile
 constexpr int PF_OP_BYTES = 3 * PF_TILE_BYTES;         // V, K hi, K lo
-constexpr int PF_P_BYTES = PF_ROWS * PF_TOK * 2;
-constexpr int PF_OFF_OP = 2 * PF_Q_BYTES;
-constexpr int PF_OFF_P = PF_OFF_OP + 2 * PF_OP_BYTES;
-constexpr int PF_OFF_RAW = PF_OFF_P + PF_P_BYTES;      // 180224
+constexpr int PF_NO = 3;                               // operand stages
+constexpr int PF_OFF_RAW = PF_NO * PF_OP_BYTES;        // 147456
 constexpr int PF_MISC = 256;                           // barriers, TMEM address, abort flag
 constexpr int PF_SMEM_MAX = 232448;                    // 227 KiB opt-in per CTA
-constexpr uint32_t PF_TMEM_COLS = 256;                 // S double buffer (2 x 64) + O (128)
+// Tensor memory (512 columns x 128 lanes, lane = row): S of tiles i (i even) and
+// i (i odd) in columns 0-63 and 64-127, each overwritten in place by the tile's
+// fp16 P (32 columns of pairs); O in 128-255; the query image q' hi in 256-319
+// and lo in 320-383 (fp16 pairs).
+constexpr uint32_t PF_TMEM_COLS = 512;
 constexpr uint32_t PF_O_COL = 128;
+constexpr uint32_t PF_QH_COL = 256;
+constexpr uint32_t PF_QL_COL = 320;
 constexpr float PF_RESCALE = 8.0f;                     // lazy rescale threshold (log2 units)
 
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -92,6 +95,16 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same with A read from tensor memory (M rows in lanes, K along columns, two
+// 16-bit elements per 32-bit column, the lower-indexed in the low half).
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -171,85 +184,133 @@ __device__ __forceinline__ void split8(const float x[8], uint8_t* hi, uint8_t* l
 // its codes' low plane (lo, up to 32 bytes) and high plane (hi, up to 8 bytes).
 // K planes are interleaved in 16-byte pieces (byte o of token t at
 // ((o/16)*64 + t)*16 + o%16); V planes are row-major.  Every read is aligned.
-__device__ __forceinline__ void block_planes(const uint8_t* codes, bool kplane, int cb, int t, int b, int bits,
-                                             uint32_t lo[8], uint32_t hi[2]) {
+template <int BITS, bool KPLANE>
+__device__ __forceinline__ void block_planes(const uint8_t* codes, int cb, int t, int b, uint32_t lo[8],
+                                             uint32_t hi[2]) {
   auto at = [&](int o) -> const uint8_t* {
-    return kplane ? codes + ((((o >> 4) * PAGE + t) << 4) + (o & 15)) : codes + t * cb + o;
+    return KPLANE ? codes + ((((o >> 4) * PAGE + t) << 4) + (o & 15)) : codes + t * cb + o;
   };
-  if (bits == 8) {
+  if (BITS == 8) {
     const uint4 a = *reinterpret_cast<const uint4*>(at(32 * b));
     const uint4 c = *reinterpret_cast<const uint4*>(at(32 * b + 16));
     lo[0] = a.x; lo[1] = a.y; lo[2] = a.z; lo[3] = a.w; lo[4] = c.x; lo[5] = c.y; lo[6] = c.z; lo[7] = c.w;
-  } else if (bits >= 4) {                          // 4, 5, 6: nibble plane first
+  } else if (BITS >= 4) {                          // 4, 5, 6: nibble plane first
     const uint4 a = *reinterpret_cast<const uint4*>(at(16 * b));
     lo[0] = a.x; lo[1] = a.y; lo[2] = a.z; lo[3] = a.w;
   } else {                                         // 2, 3: 2-bit plane first
     const uint2 a = *reinterpret_cast<const uint2*>(at(8 * b));
     lo[0] = a.x; lo[1] = a.y;
   }
-  if (bits == 6) {
+  if (BITS == 6) {
     const uint2 h = *reinterpret_cast<const uint2*>(at(64 + 8 * b));
     hi[0] = h.x; hi[1] = h.y;
-  } else if (bits == 5) {
+  } else if (BITS == 5) {
     hi[0] = *reinterpret_cast<const uint32_t*>(at(64 + 4 * b));
-  } else if (bits == 3) {
+  } else if (BITS == 3) {
     hi[0] = *reinterpret_cast<const uint32_t*>(at(32 + 4 * b));
   }
 }
 
-// The 8 codes of channels 8 j8 .. 8 j8 + 7 of a block (j8 a compile-time index).
-template <int J8>
-__device__ __forceinline__ void chunk_codes(int bits, const uint32_t lo[8], const uint32_t hi[2], uint32_t u[8]) {
-  if (bits == 8) {
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      u[v] = (lo[2 * J8] >> (8 * v)) & 255u;
-      u[4 + v] = (lo[2 * J8 + 1] >> (8 * v)) & 255u;
-    }
-  } else if (bits >= 4) {
-#pragma unroll
-    for (int v = 0; v < 8; ++v) u[v] = (lo[J8] >> (4 * v)) & 15u;
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ __half2 as_h2(uint32_t w) { return *reinterpret_cast<const __half2*>(&w); }
+__device__ __forceinline__ uint32_t as_u32(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+
+// The codes of channels 8J .. 8J+7 of a block as four fp16 pairs 1024 + u (bit
+// pattern 0x6400 | u, exact for u < 1024): pair e holds channels 8J+2e (low
+// half) and 8J+2e+1.  8- and 4-bit planes are spread with byte permutes (for
+// nibbles, the sign-replicating selectors 8 + k give zero bytes: every byte is
+// below 16); the other widths assemble their integer codes first.
+template <int BITS, int J>
+__device__ __forceinline__ void chunk_pairs(const uint32_t lo[8], const uint32_t hi[2], uint32_t W[4]) {
+  if (BITS == 8) {
+    const uint32_t a = lo[2 * J], c = lo[2 * J + 1];
+    W[0] = prmt(a, 0x64646464u, 0x4140u);
+    W[1] = prmt(a, 0x64646464u, 0x4342u);
+    W[2] = prmt(c, 0x64646464u, 0x4140u);
+    W[3] = prmt(c, 0x64646464u, 0x4342u);
+  } else if (BITS == 4) {
+    const uint32_t L = lo[J] & 0x0F0F0F0Fu, Hh = (lo[J] >> 4) & 0x0F0F0F0Fu;
+    W[0] = prmt(L, Hh, 0xC480u) | 0x64006400u;
+    W[1] = prmt(L, Hh, 0xD591u) | 0x64006400u;
+    W[2] = prmt(L, Hh, 0xE6A2u) | 0x64006400u;
+    W[3] = prmt(L, Hh, 0xF7B3u) | 0x64006400u;
   } else {
-    const uint32_t w = lo[J8 >> 1] >> (16 * (J8 & 1));
+    uint32_t u[8];
+    if (BITS >= 4) {
 #pragma unroll
-    for (int v = 0; v < 8; ++v) u[v] = (w >> (2 * v)) & 3u;
-  }
-  if (bits == 6) {
-    const uint32_t h = hi[J8 >> 1] >> (16 * (J8 & 1));
+      for (int v = 0; v < 8; ++v) u[v] = (lo[J] >> (4 * v)) & 15u;
+    } else {
+      const uint32_t w = lo[J >> 1] >> (16 * (J & 1));
 #pragma unroll
-    for (int v = 0; v < 8; ++v) u[v] |= ((h >> (2 * v)) & 3u) << 4;
-  } else if (bits == 5 || bits == 3) {
-    const uint32_t h = hi[0] >> (8 * J8);
-    const int sh = bits == 5 ? 4 : 2;
+      for (int v = 0; v < 8; ++v) u[v] = (w >> (2 * v)) & 3u;
+    }
+    if (BITS == 6) {
+      const uint32_t h = hi[J >> 1] >> (16 * (J & 1));
 #pragma unroll
-    for (int v = 0; v < 8; ++v) u[v] |= ((h >> v) & 1u) << sh;
+      for (int v = 0; v < 8; ++v) u[v] |= ((h >> (2 * v)) & 3u) << 4;
+    } else if (BITS == 5 || BITS == 3) {
+      const uint32_t h = hi[0] >> (8 * J);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) u[v] |= ((h >> v) & 1u) << (BITS == 5 ? 4 : 2);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) W[e] = u[2 * e] | (u[2 * e + 1] << 16) | 0x64006400u;
   }
 }
 
-// Dequantize block b of token t (32 values) of one plane into operand chunks
-// 4b .. 4b+3 of row t: hi image (and lo image for keys).  Invalid rows become zeros.
-__device__ __forceinline__ void dequant_block(const uint8_t* codes, const uint8_t* scales, bool kplane, int cb,
-                                              int sb, int bits, bool asym, int t, int b, bool valid, uint8_t* hi,
-                                              uint8_t* lo) {
+// Dequantize block b of token t (32 values) into operand chunks 4b .. 4b+3 of
+// row t: the hi image, and for keys (KEY) the lo image.  Invalid rows become
+// zeros.  In fp16 pairs: the centred code c = (1024 + u) - (1024 + 2^(BITS-1)) is
+// exact, hi = c * d is one rounding of the exact product and lo = fma(c, d, -hi)
+// is the exact remainder (c*d has at most 19 significant bits, hi the top 11, so
+// the rest fits fp16).  The _1 codecs' values u*d + m are taken in fp32 for keys
+// (the reference's rounding, then hi and lo) and as one fp16 fma for values.
+template <int BITS, bool ASYM, bool KEY>
+__device__ __forceinline__ void dequant_block(const uint8_t* codes, const uint8_t* scales, int cb, int sb, int t,
+                                              int b, bool valid, uint8_t* hi, uint8_t* lo) {
   uint32_t lw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, hw[2] = {0u, 0u};
-  float d = 0.f, off = 0.f;
+  __half2 D2 = __float2half2_rn(0.f), M2 = D2;
   if (valid) {
-    block_planes(codes, kplane, cb, t, b, bits, lw, hw);
-    if (asym) {
+    block_planes<BITS, KEY>(codes, cb, t, b, lw, hw);
+    if (ASYM) {
       const __half2 dm = *reinterpret_cast<const __half2*>(scales + t * sb + 4 * b);
-      d = __low2float(dm);
-      off = __high2float(dm);
+      D2 = __low2half2(dm);
+      M2 = __high2half2(dm);
     } else {
-      d = __half2float(*reinterpret_cast<const __half*>(scales + t * sb + 2 * b));
-      off = -(float)(1 << (bits - 1)) * d;
+      D2 = __half2half2(*reinterpret_cast<const __half*>(scales + t * sb + 2 * b));
     }
   }
-  uint32_t u[8];
-  float x[8];
-#define KVQ_PF_CHUNK(J)                                                   \
-  chunk_codes<J>(bits, lw, hw, u);                                        \
-  _Pragma("unroll") for (int v = 0; v < 8; ++v) x[v] = fmaf((float)u[v], d, off); \
-  split8(x, hi, lo, op_off(t, 4 * b + J));
+  const __half2 C0 = as_h2(ASYM ? 0x64006400u : (0x6400u + (1u << (BITS - 1))) * 0x10001u);
+  const float d = __low2float(D2), m = __low2float(M2);
+#define KVQ_PF_CHUNK(J)                                                                       \
+  {                                                                                           \
+    uint32_t W[4], H[4], L[4];                                                                \
+    chunk_pairs<BITS, J>(lw, hw, W);                                                          \
+    _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                           \
+      const __half2 C = __hsub2(as_h2(W[e]), C0);                                             \
+      if (ASYM && KEY) {                                                                      \
+        const float2 f = __half22float2(C);                                                   \
+        const float x0 = fmaf(f.x, d, m), x1 = fmaf(f.y, d, m);                               \
+        const __half2 hh = __floats2half2_rn(x0, x1);                                         \
+        const float2 hf = __half22float2(hh);                                                 \
+        H[e] = as_u32(hh);                                                                    \
+        L[e] = as_u32(__floats2half2_rn(__fsub_rn(x0, hf.x), __fsub_rn(x1, hf.y)));           \
+      } else if (ASYM) {                                                                      \
+        H[e] = as_u32(__hfma2(C, D2, M2));                                                    \
+      } else {                                                                                \
+        const __half2 hh = __hmul2(C, D2);                                                    \
+        H[e] = as_u32(hh);                                                                    \
+        if (KEY) L[e] = as_u32(__hfma2(C, D2, __hneg2(hh)));                                  \
+      }                                                                                       \
+    }                                                                                         \
+    const uint32_t o = op_off(t, 4 * b + J);                                                  \
+    *reinterpret_cast<uint4*>(hi + o) = make_uint4(H[0], H[1], H[2], H[3]);                   \
+    if (KEY) *reinterpret_cast<uint4*>(lo + o) = make_uint4(L[0], L[1], L[2], L[3]);          \
+  }
   KVQ_PF_CHUNK(0)
   KVQ_PF_CHUNK(1)
   KVQ_PF_CHUNK(2)
@@ -257,15 +318,54 @@ __device__ __forceinline__ void dequant_block(const uint8_t* codes, const uint8_
 #undef KVQ_PF_CHUNK
 }
 
+// A dequantizer thread's two units of a 64-token tile: unit u = dt + 128 k is
+// (token t, block b), 8 neighbouring threads on 8 neighbouring tokens (their
+// 16-byte stores fill 128 contiguous bytes).  Rows at or past nq_end hold no data.
+template <int BITS, bool ASYM, bool KEY>
+__device__ __forceinline__ void dequant_units(const uint8_t* codes, const uint8_t* scales, int cb, int sb, int dt,
+                                              int tok0, int nq_end, uint8_t* hi, uint8_t* lo) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int u = dt + 128 * k;
+    const int t = (u & 7) | ((u >> 5) << 3), b = (u >> 3) & 3;
+    dequant_block<BITS, ASYM, KEY>(codes, scales, cb, sb, t, b, tok0 + t < nq_end, hi, lo);
+  }
+}
+
+// One instantiation per block codec, chosen once per tile (the codec is the same
+// for every unit of a CTA, so each CTA runs one branch).
+template <bool KEY>
+__device__ __forceinline__ void dequant_tile(int codec, const uint8_t* codes, const uint8_t* scales, int cb, int sb,
+                                             int dt, int tok0, int nq_end, uint8_t* hi, uint8_t* lo) {
+  switch (codec) {
+#define KVQ_PF_CASE(C, B, A) \
+  case C: dequant_units<B, A, KEY>(codes, scales, cb, sb, dt, tok0, nq_end, hi, lo); break;
+    KVQ_PF_CASE(KVQ_Q8_0, 8, false)
+    KVQ_PF_CASE(KVQ_Q6_0, 6, false)
+    KVQ_PF_CASE(KVQ_Q5_0, 5, false)
+    KVQ_PF_CASE(KVQ_Q4_0, 4, false)
+    KVQ_PF_CASE(KVQ_Q3_0, 3, false)
+    KVQ_PF_CASE(KVQ_Q2_0, 2, false)
+    KVQ_PF_CASE(KVQ_Q8_1, 8, true)
+    KVQ_PF_CASE(KVQ_Q6_1, 6, true)
+    KVQ_PF_CASE(KVQ_Q5_1, 5, true)
+    KVQ_PF_CASE(KVQ_Q4_1, 4, true)
+    KVQ_PF_CASE(KVQ_Q3_1, 3, true)
+    KVQ_PF_CASE(KVQ_Q2_1, 2, true)
+#undef KVQ_PF_CASE
+    default: break;
+  }
+}
+
 struct PfBars {
   uint64_t* raw_full;    // [n_raw]
   uint64_t* raw_empty;   // [n_raw]
-  uint64_t* op_full;     // [2]
-  uint64_t* op_empty;    // [2]
-  uint64_t* s_full;      // [2]
-  uint64_t* s_empty;     // [2]
-  uint64_t* p_full;
-  uint64_t* p_empty;
+  uint64_t* op_full;     // [PF_NO]
+  uint64_t* opk_empty;   // [PF_NO] keys of the stage read (S done)
+  uint64_t* opv_empty;   // [PF_NO] values of the stage read (P V done)
+  uint64_t* s_full;      // [2] S of the buffer's tile complete
+  uint64_t* p_full;      // [2] P of the buffer's tile in tensor memory
+  uint64_t* p_empty;     // [2] P V of the buffer's tile complete (S buffer free again)
   uint64_t* q_ready;
   uint64_t* done;
 };
@@ -313,25 +413,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
   const int NR = p.n_raw;
   const bool rotated = p.rot != KVQ_ROT_NONE;
 
-  uint8_t* sQh = smem;
-  uint8_t* sQl = smem + PF_Q_BYTES;
-  uint8_t* sOp = smem + PF_OFF_OP;                       // [2][V | K hi | K lo]
-  uint8_t* sP = smem + PF_OFF_P;
-  uint8_t* sRaw = smem + PF_OFF_RAW;
+  uint8_t* sOp = smem;                                   // [PF_NO][V | K hi | K lo]
+  uint8_t* sRaw = smem + PF_OFF_RAW;                     // [NR] raw page-heads
   uint64_t* barmem = reinterpret_cast<uint64_t*>(sRaw + (size_t)NR * p.stage_bytes);
   PfBars B;
-  B.raw_full = barmem;
-  B.raw_empty = barmem + 4;
-  B.op_full = barmem + 8;
-  B.op_empty = barmem + 10;
-  B.s_full = barmem + 12;
-  B.s_empty = barmem + 14;
-  B.p_full = barmem + 16;
-  B.p_empty = barmem + 17;
-  B.q_ready = barmem + 18;
-  B.done = barmem + 19;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(barmem + 20);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(barmem + 21);
+  B.raw_full = barmem;              // 0-3
+  B.raw_empty = barmem + 4;         // 4-7
+  B.op_full = barmem + 8;           // 8-10
+  B.opk_empty = barmem + 11;        // 11-13
+  B.opv_empty = barmem + 14;        // 14-16
+  B.s_full = barmem + 17;           // 17-18
+  B.p_full = barmem + 19;           // 19-20
+  B.p_empty = barmem + 21;          // 21-22
+  B.q_ready = barmem + 23;
+  B.done = barmem + 24;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(barmem + 25);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(barmem + 26);
 
   if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
@@ -340,12 +437,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     if (lane == 0) {
       for (int i = 0; i < NR; ++i) { mbar_init(&B.raw_full[i], 1); mbar_init(&B.raw_empty[i], 4); }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&B.op_full[i], 4); mbar_init(&B.op_empty[i], 1);
-        mbar_init(&B.s_full[i], 1); mbar_init(&B.s_empty[i], 4);
+      for (int i = 0; i < PF_NO; ++i) {
+        mbar_init(&B.op_full[i], 4); mbar_init(&B.opk_empty[i], 1); mbar_init(&B.opv_empty[i], 1);
       }
-      mbar_init(B.p_full, 4);
-      mbar_init(B.p_empty, 1);
+      for (int i = 0; i < 2; ++i) { mbar_init(&B.s_full[i], 1); mbar_init(&B.p_full[i], 4); mbar_init(&B.p_empty[i], 1); }
       mbar_init(B.q_ready, 4);
       mbar_init(B.done, 1);
       *abort_flag = 0;
@@ -388,42 +483,61 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
       const uint32_t idS = umma_idesc(PF_TOK, false), idPV = umma_idesc(D, true);
-      const uint32_t aQh = smem_u32(sQh), aQl = smem_u32(sQl), aP = smem_u32(sP), aOp = smem_u32(sOp);
+      const uint32_t aOp = smem_u32(sOp);
       bool ok = pf_wait1(B.q_ready, 0, p, abort_flag);
-      auto issue_pv = [&](int i) {                      // O += P V of tile i
-        const uint32_t v0 = aOp + (uint32_t)(i & 1) * PF_OP_BYTES;
-#pragma unroll
-        for (int s = 0; s < PF_TOK / 16; ++s)
-          umma_f16(tmem + PF_O_COL, umma_desc(aP + 256 * s, 128, 1024), umma_desc(v0 + 4096 * s, 2048, 128), idPV,
-                   (i > 0 || s > 0) ? 1u : 0u);
-        umma_commit(B.p_empty);
-        umma_commit(&B.op_empty[i & 1]);
-      };
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int b = i & 1;
-        if (!pf_wait1(&B.op_full[b], (i >> 1) & 1, p, abort_flag)) break;
-        if (i >= 2 && !pf_wait1(&B.s_empty[b], ((i >> 1) - 1) & 1, p, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t kh = aOp + (uint32_t)b * PF_OP_BYTES + PF_TILE_BYTES, kl = kh + PF_TILE_BYTES;
-        const uint32_t dS = tmem + (uint32_t)b * PF_TOK;
+      tc_fence_after();
+      auto issue_s = [&](int i) {                       // S = Q' K^T of tile i (A: q' from tensor memory)
+        const int st = i % PF_NO;
+        const uint32_t kh = aOp + (uint32_t)st * PF_OP_BYTES + PF_TILE_BYTES, kl = kh + PF_TILE_BYTES;
+        const uint32_t dS = tmem + (uint32_t)(i & 1) * PF_TOK;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
-          const uint64_t qh = umma_desc(aQh + 256 * s, 128, 2048), ql = umma_desc(aQl + 256 * s, 128, 2048);
           const uint64_t bh = umma_desc(kh + 256 * s, 128, 2048), bl = umma_desc(kl + 256 * s, 128, 2048);
-          umma_f16(dS, qh, bh, idS, s > 0 ? 1u : 0u);
-          umma_f16(dS, ql, bh, idS, 1u);
-          umma_f16(dS, qh, bl, idS, 1u);
+          umma_f16_tmem_a(dS, tmem + PF_QH_COL + 8 * s, bh, idS, s > 0 ? 1u : 0u);
+          umma_f16_tmem_a(dS, tmem + PF_QL_COL + 8 * s, bh, idS, 1u);
+          umma_f16_tmem_a(dS, tmem + PF_QH_COL + 8 * s, bl, idS, 1u);
         }
-        umma_commit(&B.s_full[b]);
-        if (i >= 1) {
-          if (!pf_wait1(B.p_full, (i - 1) & 1, p, abort_flag)) break;
+        umma_commit(&B.s_full[i & 1]);
+        umma_commit(&B.opk_empty[st]);
+      };
+      auto issue_pv = [&](int i) {                      // O += P V of tile i (A: P from tensor memory)
+        const int st = i % PF_NO;
+        const uint32_t v0 = aOp + (uint32_t)st * PF_OP_BYTES;
+        const uint32_t pa = tmem + (uint32_t)(i & 1) * PF_TOK;
+#pragma unroll
+        for (int s = 0; s < PF_TOK / 16; ++s)
+          umma_f16_tmem_a(tmem + PF_O_COL, pa + 8 * s, umma_desc(v0 + 4096 * s, 2048, 128), idPV,
+                          (i > 0 || s > 0) ? 1u : 0u);
+        umma_commit(&B.p_empty[i & 1]);
+        umma_commit(&B.opv_empty[st]);
+      };
+      // Issue whichever product is ready, polling without suspending: P V of
+      // tile np once its P is in tensor memory (np < ns), else S of tile ns once
+      // its operands are in and P V of tile ns - 2 (the last reader of the S/P
+      // columns it overwrites) has completed.  No phase of these barriers can run
+      // ahead of the issue order, so each parity names one completion.
+      int ns = 0, np = 0;
+      uint64_t t_last = globaltimer_ns();
+      while (ok && np < n_tiles) {
+        bool progress = false;
+        if (np < ns && mbar_test_wait(&B.p_full[np & 1], (np >> 1) & 1)) {
           tc_fence_after();
-          issue_pv(i - 1);
+          issue_pv(np++);
+          progress = true;
+        } else if (ns < n_tiles && mbar_test_wait(&B.op_full[ns % PF_NO], (ns / PF_NO) & 1) &&
+                   (ns < 2 || mbar_test_wait(&B.p_empty[ns & 1], ((ns >> 1) - 1) & 1))) {
+          tc_fence_after();
+          issue_s(ns++);
+          progress = true;
         }
-        if (i == n_tiles - 1) {
-          if (!pf_wait1(B.p_full, i & 1, p, abort_flag)) break;
-          tc_fence_after();
-          issue_pv(i);
+        if (progress) {
+          t_last = globaltimer_ns();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (globaltimer_ns() - t_last > p.wait_ns) {
+          *abort_flag = 1;
+          atomicOr(p.err, ERR_TIMEOUT);
+          ok = false;
         }
       }
       // nothing of this CTA may still run on the tensor cores when it exits
@@ -434,41 +548,34 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- dequantizers
     const int dt = threadIdx.x - 128;
-    const int kc = h.kcodec, vc = h.vcodec;
-    const int kbits = h.kbits, vbits = h.vbits;
-    const bool kasym = codec_is_asym(kc), vasym = codec_is_asym(vc);
     for (int i = 0; i < n_tiles; ++i) {
-      const int b = i & 1;
-      if (i >= 2 && !pf_wait(&B.op_empty[b], ((i >> 1) - 1) & 1, p, abort_flag)) break;
-      uint8_t* opV = sOp + (size_t)b * PF_OP_BYTES;
+      const int st = i % PF_NO;
+      const uint32_t prev = ((i / PF_NO) - 1) & 1;      // phase of the stage's previous tile
+      uint8_t* opV = sOp + (size_t)st * PF_OP_BYTES;
       uint8_t* opKh = opV + PF_TILE_BYTES;
       uint8_t* opKl = opKh + PF_TILE_BYTES;
       if (i < n_qt) {
-        const int st = i % NR;
-        if (!pf_wait(&B.raw_full[st], (i / NR) & 1, p, abort_flag)) break;
-        const uint8_t* kcodes = sRaw + (size_t)st * p.stage_bytes;
+        const int rs = i % NR;
+        if (!pf_wait(&B.raw_full[rs], (i / NR) & 1, p, abort_flag)) break;
+        if (i >= PF_NO && !pf_wait(&B.opk_empty[st], prev, p, abort_flag)) break;
+        const uint8_t* kcodes = sRaw + (size_t)rs * p.stage_bytes;
         const uint8_t* kscales = kcodes + PAGE * h.cbK;
         const uint8_t* vcodes = kscales + PAGE * h.sbK;
         const uint8_t* vscales = vcodes + PAGE * h.cbV;
-#pragma unroll 1
-        for (int k = 0; k < 2; ++k) {
-          // unit (token t, block bb): 8 neighbouring threads take 8 neighbouring tokens
-          const int u = dt + 128 * k;
-          const int t = (u & 7) | ((u >> 5) << 3), bb = (u >> 3) & 3;
-          const bool valid = i * PF_TOK + t < p.nq_all;   // rows past the last quantized row hold no data
-          dequant_block(kcodes, kscales, true, h.cbK, h.sbK, kbits, kasym, t, bb, valid, opKh, opKl);
-          dequant_block(vcodes, vscales, false, h.cbV, h.sbV, vbits, vasym, t, bb, valid, opV, nullptr);
-        }
+        dequant_tile<true>(h.kcodec, kcodes, kscales, h.cbK, h.sbK, dt, i * PF_TOK, p.nq_all, opKh, opKl);
+        if (i >= PF_NO && !pf_wait(&B.opv_empty[st], prev, p, abort_flag)) break;
+        dequant_tile<false>(h.vcodec, vcodes, vscales, h.cbV, h.sbV, dt, i * PF_TOK, p.nq_all, opV, nullptr);
         fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&B.raw_empty[st]);
-          mbar_arrive(&B.op_full[b]);
+          mbar_arrive(&B.raw_empty[rs]);
+          mbar_arrive(&B.op_full[st]);
         }
       } else {
         // tail tile: thread dt takes key row dt (dt < 64) or value row dt - 64,
         // reads it from the ring and brings it into the quantized rows' basis
-        const int r = dt & 63, kv = dt >> 6;
+        const int r = dt & 63, kv = dt >> 6;            // warp-uniform: warps 4, 5 keys, 6, 7 values
+        if (i >= PF_NO && !pf_wait(kv ? &B.opv_empty[st] : &B.opk_empty[st], prev, p, abort_flag)) break;
         const int pos = p.nq_all + (i - n_qt) * PF_TOK + r;
         float x[D];
         if (pos < vis_end) {
@@ -486,9 +593,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
           }
           if (rotated) {
             if (p.inv_s) {
-              const float* s = p.inv_s + ((size_t)head * 2 + kv) * D;
+              const float* sc = p.inv_s + ((size_t)head * 2 + kv) * D;
 #pragma unroll
-              for (int c = 0; c < D; ++c) x[c] = __fmul_rn(x[c], s[c]);
+              for (int c = 0; c < D; ++c) x[c] = __fmul_rn(x[c], sc[c]);
             }
             fwht128(x);
           }
@@ -501,7 +608,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
           split8(x + 8 * c8, kv == 0 ? opKh : opV, kv == 0 ? opKl : nullptr, op_off(r, c8));
         fence_proxy_async_shared();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&B.op_full[b]);
+        if (lane == 0) mbar_arrive(&B.op_full[st]);
       }
     }
   } else {
@@ -512,7 +619,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
     const int pos_r = valid ? P0 + j : vis_end - 1;      // padding rows see what the block sees
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     {
-      // query image: q' = R (s_k * q) * scale (log2 units), fp16 hi and lo
+      // query image in tensor memory: q' = R (s_k * q) * scale (log2 units), fp16 hi and lo
       float x[D];
       if (valid) {
         const __half* src = p.q + ((size_t)(q0 + j) * p.Hq + (size_t)head * G + g) * D;
@@ -539,8 +646,21 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
         for (int c = 0; c < D; ++c) x[c] = 0.f;
       }
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) split8(x + 8 * c8, sQh, sQl, op_off(row, c8));
-      fence_proxy_async_shared();
+      for (int half = 0; half < 2; ++half) {             // columns of 64 values each
+        uint32_t hw[32], lw[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float a = x[64 * half + 2 * e], bq = x[64 * half + 2 * e + 1];
+          const __half2 hh = __floats2half2_rn(a, bq);
+          const float2 hf = __half22float2(hh);
+          hw[e] = as_u32(hh);
+          lw[e] = as_u32(__floats2half2_rn(__fsub_rn(a, hf.x), __fsub_rn(bq, hf.y)));
+        }
+        tmem_st32(lane_base + PF_QH_COL + 32 * half, hw);
+        tmem_st32(lane_base + PF_QL_COL + 32 * half, lw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(B.q_ready);
     }
@@ -560,9 +680,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
 #pragma unroll
         for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(r[c]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B.s_empty[b]);
       // causal mask and the end of the tile's segment (quantized rows, tail rows)
       const bool quant = i < n_qt;
       const int tok0 = quant ? i * PF_TOK : p.nq_all + (i - n_qt) * PF_TOK;
@@ -581,10 +698,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
         l *= alpha;
         m_run = mt;
       }
-      // P's buffer and O are free once P V of the previous tile has completed
-      if (i >= 1 && !pf_wait(B.p_empty, (i - 1) & 1, p, abort_flag)) { ok = false; break; }
-      tc_fence_after();
+      uint32_t pw[PF_TOK / 2];
+      float ls = 0.f;
+#pragma unroll
+      for (int e = 0; e < PF_TOK / 2; ++e) {
+        const float a = pf_ex2(s[2 * e] - m_run), bq = pf_ex2(s[2 * e + 1] - m_run);
+        ls += a + bq;
+        pw[e] = as_u32(__floats2half2_rn(a, bq));
+      }
+      l += ls;
+      // O is touched only by a rescale, which waits for P V of the previous tile
       if (i >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!pf_wait(&B.p_empty[(i - 1) & 1], ((i - 1) >> 1) & 1, p, abort_flag)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t r[32];
@@ -593,29 +719,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
           for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
           tmem_st32(lane_base + PF_O_COL + c0, r);
         }
-        tmem_wait_st();
       }
-      float ls = 0.f;
-#pragma unroll
-      for (int c8 = 0; c8 < PF_TOK / 8; ++c8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = pf_ex2(s[8 * c8 + 2 * e] - m_run), bq = pf_ex2(s[8 * c8 + 2 * e + 1] - m_run);
-          ls += a + bq;
-          const __half2 hh = __floats2half2_rn(a, bq);
-          w[e] = *reinterpret_cast<const uint32_t*>(&hh);
-        }
-        *reinterpret_cast<uint4*>(sP + (((row >> 3) * 8 + c8) << 7) + ((row & 7) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      l += ls;
-      fence_proxy_async_shared();
+      // P over the first half of this tile's S columns (S is in registers)
+      tmem_st32(lane_base + (uint32_t)b * PF_TOK, pw);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(B.p_full);
+      if (lane == 0) mbar_arrive(&B.p_full[b]);
     }
     // ---- epilogue: O / l, back to the original basis
-    if (ok && n_tiles > 0 && pf_wait(B.p_empty, (n_tiles - 1) & 1, p, abort_flag)) {
+    if (ok && n_tiles > 0 && pf_wait(&B.p_empty[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p, abort_flag)) {
       tc_fence_after();
       float x[D];
 #pragma unroll
