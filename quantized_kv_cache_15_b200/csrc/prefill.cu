@@ -39,13 +39,17 @@
 //   warp 9     tensor memory allocation and, on one thread, the MMA issue: S of
 //              tile i is issued before P V of tile i-1, so the softmax of tile i
 //              overlaps the value product of the tile before.
-// Operands use the canonical no-swizzle layouts: 8-row x 16-byte core matrices;
-// an operand "tile" of 64 tokens x 128 channels stores element (t, c) at byte
-// ((t/8)*16 + c/8)*128 + (t%8)*16 + (c%8)*2.  Read as K-major with rows = tokens
-// (keys: B of S) the leading byte offset is 128 and the stride byte offset 2048;
-// read as MN-major with N = channels and K = tokens (values: B of P V) the
-// 8-channel groups are 128 bytes apart (stride byte offset) and the 8-token
-// groups 2048 (leading byte offset).
+// The key and value images in shared memory use the canonical 128-byte-swizzled
+// layout: a 64-token x 128-channel tile is two 8 KiB halves (channels 0-63 and
+// 64-127); in a half, token t owns the 128-byte row t, and its 16-byte chunk j
+// (channels 8j .. 8j+7 of the half) sits at chunk position j XOR (t % 8), so
+// the eight rows of an 8-token group spread every chunk over all banks.  Read as
+// K-major with rows = tokens (keys: B of S) the 8-token groups are 1024 bytes
+// apart (stride byte offset) and a 16-channel step moves the start 32 bytes
+// inside the half; read as MN-major with N = channels and K = tokens (values: B
+// of P V) the two halves are 8 KiB apart (leading byte offset), the 8-token
+// groups 1024 (stride byte offset), and a 16-token step moves the start 2 KiB.
+// The query image and P live in tensor memory (A operands).
 // Every wait is bounded; a timeout latches an error bit and sends every role out
 // of its loop; in-flight copies and MMAs are waited for (bounded) and the tensor
 // memory is always freed.
@@ -76,12 +80,15 @@ constexpr uint32_t PF_QH_COL = 256;
 constexpr uint32_t PF_QL_COL = 320;
 constexpr float PF_RESCALE = 8.0f;                     // lazy rescale threshold (log2 units)
 
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand (atoms 1024-byte
+// aligned, so the base offset is 0).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;   // descriptor version for sm_100; base offset 0, no swizzle
+  d |= (uint64_t)1 << 46;   // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;   // layout: 128-byte swizzle
   return d;
 }
 // kind::f16 instruction descriptor: D fp32, A and B fp16, A K-major, B K-major or
@@ -159,9 +166,11 @@ __device__ __forceinline__ void fwht128(float x[D]) {
   for (int i = 0; i < D; ++i) x[i] = __fmul_rn(x[i], c);
 }
 
-// Byte offset of 16-byte chunk c8 (channels 8 c8 .. 8 c8 + 7) of row t in an
-// operand image (64-token tiles and the 128-row query image alike).
-__device__ __forceinline__ uint32_t op_off(int t, int c8) { return (uint32_t)((((t >> 3) << 4) + c8) << 7) + ((t & 7) << 4); }
+// Byte offset of 16-byte chunk c8 (channels 8 c8 .. 8 c8 + 7) of token t in a key
+// or value image: half c8 / 8, row t, chunk position (c8 % 8) XOR (t % 8).
+__device__ __forceinline__ uint32_t op_off(int t, int c8) {
+  return (uint32_t)(((c8 >> 3) << 13) + ((t >> 3) << 10) + ((t & 7) << 7) + (((c8 & 7) ^ (t & 7)) << 4));
+}
 
 // Eight values -> fp16 hi words and, when lo != null, the fp16 remainders.
 __device__ __forceinline__ void split8(const float x[8], uint8_t* hi, uint8_t* lo, uint32_t off) {
@@ -492,7 +501,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
         const uint32_t dS = tmem + (uint32_t)(i & 1) * PF_TOK;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
-          const uint64_t bh = umma_desc(kh + 256 * s, 128, 2048), bl = umma_desc(kl + 256 * s, 128, 2048);
+          const uint32_t ko = (uint32_t)(s >> 2) * 8192u + (uint32_t)(s & 3) * 32u;
+          const uint64_t bh = umma_desc_sw128(kh + ko, 16, 1024), bl = umma_desc_sw128(kl + ko, 16, 1024);
           umma_f16_tmem_a(dS, tmem + PF_QH_COL + 8 * s, bh, idS, s > 0 ? 1u : 0u);
           umma_f16_tmem_a(dS, tmem + PF_QL_COL + 8 * s, bh, idS, 1u);
           umma_f16_tmem_a(dS, tmem + PF_QH_COL + 8 * s, bl, idS, 1u);
@@ -506,7 +516,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(const __grid_con
         const uint32_t pa = tmem + (uint32_t)(i & 1) * PF_TOK;
 #pragma unroll
         for (int s = 0; s < PF_TOK / 16; ++s)
-          umma_f16_tmem_a(tmem + PF_O_COL, pa + 8 * s, umma_desc(v0 + 4096 * s, 2048, 128), idPV,
+          umma_f16_tmem_a(tmem + PF_O_COL, pa + 8 * s, umma_desc_sw128(v0 + 2048 * s, 8192, 1024), idPV,
                           (i > 0 || s > 0) ? 1u : 0u);
         umma_commit(&B.p_empty[i & 1]);
         umma_commit(&B.opv_empty[st]);
