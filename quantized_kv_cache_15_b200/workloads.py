@@ -8,15 +8,19 @@ rows can be regenerated on either device, chunk by chunk.
 
 Random numbers come from a counter-based generator: a 32-bit integer hash of
 (stream key, element index) evaluated with int64 torch ops, which gives the
-same bits on CPU and CUDA.  Gaussian-like values are the Irwin-Hall sum of
-four 16-bit uniforms, rescaled to unit variance, using only correctly rounded
-fp32 adds and multiplies (also device independent).  The heavy-tailed term is
-a Student-t (nu = 3) built as Z / sqrt(chi2_3 / 3) from four such values.
+same bits on CPU and CUDA.  Normal N(0,1) values come by inversion: the top 16
+bits of a 32-bit uniform pick a cell of a table of standard-normal quantiles
+(65537 fp32 values at u = k / 65536, computed once on the host; the two end
+points at u = 2^-33 and 1 - 2^-33, about 6.2 sigma) and the low 16 bits
+interpolate linearly inside the cell, with correctly rounded fp32 subtract,
+multiply and add (also device independent).  The heavy-tailed term is a
+Student-t (nu = 3) built as Z / sqrt(chi2_3 / 3) from four such values.
 """
 from __future__ import annotations
 
 import dataclasses
 import math
+import statistics
 from typing import Dict, List, Optional, Tuple
 
 import numpy as np
@@ -81,13 +85,33 @@ def uniform16(key: int, start: int, n: int, device) -> torch.Tensor:
     return (u.to(torch.float32) + 0.5) * (1.0 / 65536.0)
 
 
+_QUANTILES: Dict[str, torch.Tensor] = {}
+
+
+def normal_quantiles(device) -> torch.Tensor:
+    """fp32 standard-normal quantiles at u = k / 65536, k = 0 .. 65536, the ends
+    taken at u = 2^-33 and 1 - 2^-33 (host double precision, rounded once)."""
+    dev = str(torch.device(device))
+    if dev not in _QUANTILES:
+        if "cpu" not in _QUANTILES:
+            nd = statistics.NormalDist()
+            eps = 2.0 ** -33
+            q = [nd.inv_cdf(min(max(k / 65536.0, eps), 1.0 - eps)) for k in range(65537)]
+            _QUANTILES["cpu"] = torch.tensor(q, dtype=torch.float64).to(torch.float32)
+        _QUANTILES[dev] = _QUANTILES["cpu"].to(device)
+    return _QUANTILES[dev]
+
+
 def gauss(key: int, start: int, n: int, device) -> torch.Tensor:
-    """Unit-variance Irwin-Hall(4) values, fp32, exactly reproducible on any device."""
-    bits = random_bits(key, 2 * start, 2 * n, device).reshape(n, 2)
-    u = [((bits[:, j // 2] >> (16 * (j % 2))) & 0xFFFF).to(torch.float32) for j in range(4)]
-    s = (u[0] + u[1]) + (u[2] + u[3])                 # integer-valued, exact
-    s = (s + 2.0) * (1.0 / 65536.0) - 2.0              # sum of (k+1/2)/65536 minus the mean
-    return s * float(np.float32(math.sqrt(3.0)))
+    """N(0,1) values by inversion (see the module docstring), fp32, exactly
+    reproducible on any device: cell k = bits >> 16, f = ((bits & 0xFFFF) + 1/2) / 65536,
+    x = T[k] + (T[k+1] - T[k]) * f."""
+    bits = random_bits(key, start, n, device)
+    t = normal_quantiles(device)
+    k = bits >> 16
+    f = ((bits & 0xFFFF).to(torch.float32) + 0.5) * (1.0 / 65536.0)
+    lo = t[k]
+    return lo + (t[k + 1] - lo) * f
 
 
 def student_t3(key: int, start: int, n: int, device) -> torch.Tensor:

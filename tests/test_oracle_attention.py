@@ -165,10 +165,14 @@ def test_projection_full_rank_identity_basis_matches_hadamard_path():
 @pytest.mark.slow
 def test_quality_orderings_synthetic_analogue():
     """Synthetic analogues of the KLD table's orderings (BeeLlama v0.4.0 news,
-    KLD 基准 table): error falls as bits rise; a 1024-token F16 tail beats no tail
-    at low bits; variance-normalised + rotated 4-bit beats plain (unrotated) q4_0
-    on keys with outlier channels.  Metric: relative L2 error of the attention
-    output against exact F16 attention, over config-1-shaped data.  Not parity."""
+    KLD 基准 table): error falls as bits rise; at a fixed low bit width the error
+    falls as the F16 tail grows from 0 to 1024 to 2048 tokens (the table's tail
+    rows); variance-normalised + rotated 4-bit beats plain (unrotated) q4_0 on
+    keys with outlier channels.  Metric: relative L2 error of the attention
+    output against exact F16 attention, over config-1-shaped data.  Not parity.
+    The tail ordering is taken at 3 and 4 bits: at 2 bits the keys' outlier
+    channels leave an output error above 100 % (no longer correlated with the
+    exact attention), where the ordering is noise."""
     g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "kld_table.json")))["rows"]
     assert g["q2_0"][1] < g["q2_0"][0] and g["kvarn4"][0] < g["q4_0"][0]
     assert g["q8_0"][0] < g["q6_0"][0] < g["q4_0"][0] < g["q3_0"][0] < g["q2_0"][0]
@@ -185,7 +189,9 @@ def test_quality_orderings_synthetic_analogue():
 
     e = {c: err(c, c, ROT_HADAMARD) for c in (Q8_0, Q6_0, Q4_0, Q3_0, Q2_0)}
     assert e[Q8_0] < e[Q6_0] < e[Q4_0] < e[Q3_0] < e[Q2_0]
-    assert err(Q2_0, Q2_0, ROT_HADAMARD, tail=1024) < e[Q2_0]
+    for c in (Q4_0, Q3_0):
+        t1024, t2048 = err(c, c, ROT_HADAMARD, tail=1024), err(c, c, ROT_HADAMARD, tail=2048)
+        assert t2048 < t1024 < e[c] < 1.0
     invk = oracle.varnorm_inv_rms(w.rows("K", 0, 7, 0, 512)[:, 0, :].numpy().view(np.uint16))
     o_kvarn = oracle.decode_head(K, V, qs, Q4_0, Q4_0, ROT_VARNORM_HADAMARD, inv_s_k=invk,
                                  inv_s_v=np.ones(128, np.float32))
