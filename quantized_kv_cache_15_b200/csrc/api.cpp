@@ -537,12 +537,15 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
       break;
     }
   const size_t smem = decode_smem_bytes(dp.stage_bytes, dp.n_stages, p->G, dp.wtab_smem);
-  // Split sizes.  Measured per-tile times of one consumer warp barely depend on the
-  // head's rank or bits (the loops' fixed work per tile dominates), so every
-  // quantized page counts as one unit of work and a 16-row tail tile as half a
-  // unit; the machinery still allows a per-head size pps_q[h] and the tail its own
-  // pps_t.  The split size is the candidate with the smallest estimated makespan:
-  // the largest of (the costliest split) and (the average split cost x the waves of
+  // Split sizes, per kv head.  A quantized page counts as one unit of work for
+  // the block codecs (a layer's heads share a codec in the workloads) and a
+  // 16-row tail tile as half a unit.  For the rank codec the measured per-tile
+  // time of a CTA grows with the head's bit width and hardly with its rank (the
+  // loops' fixed work per tile dominates): 0.86, 0.95, 1.35 and 1.45 us per tile
+  // at 1 .. 4 bits (config-4 layer, one wave), modelled as 0.7 + 0.18 b units.
+  // Each head's split size is P / cost, so full splits of every head cost about
+  // the same.  P is the candidate with the smallest estimated makespan: the
+  // largest of (the costliest split) and (the average split cost x the waves of
   // resident CTAs, registers and shared memory both counted), where a split of n
   // tiles costs ceil(n / consumer warps) rounds of its tiles plus a fixed cost of
   // three units (query preparation, publishing the partial).  Candidates cover the
@@ -551,8 +554,12 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
   const int per_sm = std::max(1, decode_blocks_per_sm(p->G, smem));
   const int64_t target = (int64_t)p->num_sms * per_sm;
   std::vector<double> cq(p->Hkv, 1.0);
-  const double cmin = 1.0;
-  const double ct = 0.5;
+  for (int h = 0; h < p->Hkv; ++h) {
+    const HeadInfo& hi = p->head(layer, h);
+    if (hi.kcodec == KVQ_RANK) cq[h] = 0.7 + 0.18 * std::max(hi.kbits, hi.vbits);
+  }
+  const double cmin = *std::min_element(cq.begin(), cq.end());
+  const double ct = 0.5 * cmin;
   const int min_q = std::max(1, (maxq + MAX_SPLITS - 3) / (MAX_SPLITS - 2));
   const int min_t = std::max(1, (maxt + 1) / 2);
   auto sizes = [&](int P, std::vector<int>& ppq, int& ppt) {
@@ -614,7 +621,7 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
   std::vector<int> ppq;
   int ppt = 1;
   sizes(best_P, ppq, ppt);
-  dp.pps = ppq[0];
+  for (int h = 0; h < p->Hkv; ++h) dp.pps[h] = (uint16_t)ppq[h];
   dp.pps_t = ppt;
   // CTA order of the launch (decode_item): full quantized splits, partial ones
   // largest first, tail splits, zero-writing items

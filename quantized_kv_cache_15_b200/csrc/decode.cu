@@ -286,10 +286,11 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const DecodeItem it = decode_item(p, blockIdx.x);
+  if (it.kind == 3) return;                        // a head whose pages divide evenly: no partial split
   const int si = it.si, head = it.head, split = it.split;
   const int seq = p.seq[si], len = p.len[si];
   const int T = p.T;
-  const SplitCounts sc = split_counts(len, T, p.pps, p.pps_t, p.lim[si]);
+  const SplitCounts sc = split_counts(len, T, p.pps[head], p.pps_t, p.lim[si]);
   const int nq = sc.nq, nt = sc.nt, NQP = sc.nqp, NTP = sc.ntp, qsplits = sc.qsplits;
   const int S = sc.qsplits + sc.tsplits;
   float* out_base = p.out + ((size_t)si * p.Hq + (size_t)head * G) * D;
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(DECODE_THREADS, DECODE_MIN_CTAS(G)) decode_ker
     return;
   }
   const bool is_tail = it.kind == 1;
-  const int pps = is_tail ? p.pps_t : p.pps;
+  const int pps = is_tail ? p.pps_t : p.pps[head];
   const int pg0 = (is_tail ? split - qsplits : split) * pps;
   const int pg1 = min(pg0 + pps, is_tail ? NTP : NQP);
   const int n_tiles = pg1 - pg0;

@@ -207,12 +207,12 @@ struct DecodeParams {
   const float* s_v;              // [Hkv][128] per-channel V multiplier or null
   const float* M;                // projection table (floats), or null
   float qscale;                  // softmax scale * log2(e)
-  int pps;                       // quantized pages per split
+  uint16_t pps[MAX_HKV];         // quantized pages per split, per kv head
   int pps_t;                     // tail pages per split
   // CTA order of the 1-D grid (see decode_item): every split of every entry, one CTA
-  // per (split, kv head), kv head fastest, longest first.
+  // per (split, kv head), longest first.
   int n_full, n_part, n_tail, n_zero;   // items of each kind
-  int full0[MAX_BATCH + 1];      // prefix sums over entries of their full quantized splits
+  int full0[MAX_BATCH + 1];      // prefix sums over entries of their full quantized splits (all heads)
   int tail0[MAX_BATCH + 1];      // prefix sums over entries of their tail splits
   uint8_t part_order[MAX_BATCH]; // entries with a partial quantized split, largest first
   uint8_t zero_order[MAX_BATCH]; // entries with nothing to attend to
@@ -234,14 +234,15 @@ struct DecodeParams {
 
 // The splits of a decode launch in CTA order.  The hardware hands out CTAs in
 // grid order as slots free up, so the order is longest first: all full quantized
-// splits (pps pages each; entry by entry, kv head by kv head, splits in order, so
-// that the CTAs of one wave mix the heads of an entry, whose per-tile costs can
-// differ), then each entry's partial last quantized split (fewer pages), largest
-// first, then the tail splits (tail pages are 16-row tiles), and last one
-// zero-writing item per entry with nothing to attend to; after the full splits,
-// the kv head varies fastest.  kind: 0 quantized split, 1 tail split (split =
-// index among the entry's splits, quantized first), 2 nothing to attend (write
-// zeros).
+// splits (pps[head] pages each, the split sizes chosen so that full splits of
+// every head cost about the same; entry by entry, kv head by kv head, splits in
+// order), then, per entry that has any, one item per kv head for the entry's
+// partial last quantized split (entries largest first; a head whose pages divide
+// evenly gets an item that does nothing), then the tail splits (tail pages are
+// 16-row tiles), and last one zero-writing item per entry with nothing to attend
+// to; after the full splits, the kv head varies fastest.  kind: 0 quantized split,
+// 1 tail split (split = index among the entry's splits, quantized first), 2
+// nothing to attend (write zeros), 3 no work.
 struct DecodeItem { int si, head, split, kind; };
 __host__ __device__ inline int prefix_find(const int* pre, int n, int q) {
   // the entry e with pre[e] <= q < pre[e + 1] (pre non-decreasing, pre[0] = 0)
@@ -254,27 +255,34 @@ __host__ __device__ inline int prefix_find(const int* pre, int n, int q) {
 }
 __host__ __device__ inline DecodeItem decode_item(const DecodeParams& p, int b) {
   DecodeItem it;
-  if (b < p.n_full * p.Hkv) {
-    it.si = prefix_find(p.full0, p.n_seqs, b / p.Hkv);
-    const int full = p.full0[it.si + 1] - p.full0[it.si];
-    const int j = b - p.full0[it.si] * p.Hkv;
-    it.head = j / full;
-    it.split = j - it.head * full;
+  if (b < p.n_full) {
+    it.si = prefix_find(p.full0, p.n_seqs, b);
+    const int nqp = split_counts(p.len[it.si], p.T, 1, 1, p.lim[it.si]).nqp;
+    int j = b - p.full0[it.si];
+    int h = 0;
+    for (; h < p.Hkv - 1; ++h) {                // the entry's full splits, head by head
+      const int f = nqp / p.pps[h];
+      if (j < f) break;
+      j -= f;
+    }
+    it.head = h;
+    it.split = j;
     it.kind = 0;
     return it;
   }
-  it.head = b % p.Hkv;
-  int q = b / p.Hkv - p.n_full;
+  it.head = (b - p.n_full) % p.Hkv;
+  int q = (b - p.n_full) / p.Hkv;
   if (q < p.n_part) {
     it.si = p.part_order[q];
-    it.split = p.full0[it.si + 1] - p.full0[it.si];
-    it.kind = 0;
+    const int nqp = split_counts(p.len[it.si], p.T, 1, 1, p.lim[it.si]).nqp;
+    it.split = nqp / p.pps[it.head];
+    it.kind = (nqp % p.pps[it.head]) ? 0 : 3;
     return it;
   }
   q -= p.n_part;
   if (q < p.n_tail) {
     it.si = prefix_find(p.tail0, p.n_seqs, q);
-    const SplitCounts c = split_counts(p.len[it.si], p.T, p.pps, p.pps_t, p.lim[it.si]);
+    const SplitCounts c = split_counts(p.len[it.si], p.T, p.pps[it.head], p.pps_t, p.lim[it.si]);
     it.split = c.qsplits + (q - p.tail0[it.si]);
     it.kind = 1;
     return it;
@@ -290,18 +298,23 @@ __host__ __device__ inline DecodeItem decode_item(const DecodeParams& p, int b) 
 // entries' lengths, visible lengths and split sizes; returns the grid size (items
 // x kv heads) and the largest split count of one (entry, kv head) in *max_splits.
 inline int build_decode_order(DecodeParams& dp, int* max_splits) {
-  std::vector<std::pair<int, int>> parts;             // (pages of the partial split, entry)
+  std::vector<std::pair<int, int>> parts;             // (pages of the largest partial split, entry)
   int nzero = 0, most = 0;
   dp.full0[0] = 0;
   dp.tail0[0] = 0;
   for (int i = 0; i < dp.n_seqs; ++i) {
-    const SplitCounts c = split_counts(dp.len[i], dp.T, dp.pps, dp.pps_t, dp.lim[i]);
-    const int full = c.nqp / dp.pps, rest = c.nqp % dp.pps;
+    const SplitCounts c1 = split_counts(dp.len[i], dp.T, 1, dp.pps_t, dp.lim[i]);
+    int full = 0, rest = 0;
+    for (int h = 0; h < dp.Hkv; ++h) {
+      full += c1.nqp / dp.pps[h];
+      rest = std::max(rest, c1.nqp % (int)dp.pps[h]);
+      const SplitCounts c = split_counts(dp.len[i], dp.T, dp.pps[h], dp.pps_t, dp.lim[i]);
+      most = std::max(most, c.qsplits + c.tsplits);
+    }
     dp.full0[i + 1] = dp.full0[i] + full;
-    dp.tail0[i + 1] = dp.tail0[i] + c.tsplits;
+    dp.tail0[i + 1] = dp.tail0[i] + c1.tsplits;
     if (rest) parts.emplace_back(rest, i);
-    if (c.qsplits + c.tsplits == 0) dp.zero_order[nzero++] = (uint8_t)i;
-    most = std::max(most, c.qsplits + c.tsplits);
+    if (c1.nqp + c1.ntp == 0) dp.zero_order[nzero++] = (uint8_t)i;
   }
   std::stable_sort(parts.begin(), parts.end(),
                    [](const std::pair<int, int>& a, const std::pair<int, int>& b) { return a.first > b.first; });
@@ -311,7 +324,7 @@ inline int build_decode_order(DecodeParams& dp, int* max_splits) {
   dp.n_tail = dp.tail0[dp.n_seqs];
   dp.n_zero = nzero;
   *max_splits = most;
-  return (dp.n_full + dp.n_part + dp.n_tail + dp.n_zero) * dp.Hkv;
+  return dp.n_full + (dp.n_part + dp.n_tail + dp.n_zero) * dp.Hkv;
 }
 
 // ---------------------------------------------------------------- launchers (host)

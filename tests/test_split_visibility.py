@@ -127,10 +127,11 @@ int main() {
   for (int trial = 0; trial < 400; ++trial) {
     static DecodeParams dp;
     dp.n_seqs = 1 + rnd(trial < 200 ? 8 : MAX_BATCH);
-    dp.Hkv = 1 + rnd(4);
+    dp.Hkv = 1 + rnd(trial < 100 ? 4 : 12);
     const int tails[] = {0, 64, 256, 1024};
     dp.T = tails[rnd(4)];
-    dp.pps = 1 + rnd(40);
+    const int base = 1 + rnd(40);
+    for (int h = 0; h < dp.Hkv; ++h) dp.pps[h] = (uint16_t)(trial % 3 == 0 ? base : 1 + rnd(40));
     dp.pps_t = 1 + rnd(8);
     for (int i = 0; i < dp.n_seqs; ++i) {
       dp.len[i] = rnd(5) == 0 ? 0 : rnd(6000);
@@ -139,14 +140,21 @@ int main() {
     int most = 0;
     const int grid = build_decode_order(dp, &most);
     std::vector<std::vector<int>> seen(dp.n_seqs * dp.Hkv);
-    int prev_pages = 1 << 30, prev_kind = 0;
+    int prev_kind = 0;
     for (int b = 0; b < grid; ++b) {
       const DecodeItem it = decode_item(dp, b);
       const int head = it.head;
       if (head < 0 || head >= dp.Hkv) { printf("head out of range\\n"); return 1; }
       if (it.si < 0 || it.si >= dp.n_seqs) { printf("entry out of range\\n"); return 1; }
-      const SplitCounts c = split_counts(dp.len[it.si], dp.T, dp.pps, dp.pps_t, dp.lim[it.si]);
+      const SplitCounts c = split_counts(dp.len[it.si], dp.T, dp.pps[head], dp.pps_t, dp.lim[it.si]);
       const int S = c.qsplits + c.tsplits;
+      if (it.kind == 3) {                       // no-op item: only for a head without a partial split
+        if (b < dp.n_full || c.nqp % dp.pps[head] != 0) { printf("misplaced no-op item\\n"); return 1; }
+        continue;
+      }
+      // kinds in order: quantized splits, tail splits, zero items
+      if (it.kind < prev_kind) { printf("item kinds out of order\\n"); return 1; }
+      prev_kind = it.kind;
       if (it.kind == 2) {
         if (S != 0) { printf("zero item for an entry with splits\\n"); return 1; }
         seen[it.si * dp.Hkv + head].push_back(-1);
@@ -155,18 +163,14 @@ int main() {
       if (it.split < 0 || it.split >= S || (it.kind == 1) != (it.split >= c.qsplits)) {
         printf("bad split %d of %d (kind %d)\\n", it.split, S, it.kind); return 1;
       }
+      // full splits first (every one of pps[head] pages), then the partial ones
+      const bool full = it.kind == 0 && (it.split + 1) * dp.pps[head] <= c.nqp;
+      if ((b < dp.n_full) != full) { printf("full/partial split misplaced\\n"); return 1; }
       seen[it.si * dp.Hkv + head].push_back(it.split);
-      // quantized splits come longest first, then the tail splits
-      if (it.kind == 0) {
-        const int pages = std::min(dp.pps, c.nqp - it.split * dp.pps);
-        if (prev_kind == 1 || pages > prev_pages) { printf("quantized split out of order\\n"); return 1; }
-        prev_pages = pages;
-      }
-      prev_kind = it.kind;
     }
     for (int i = 0; i < dp.n_seqs; ++i)
       for (int h = 0; h < dp.Hkv; ++h) {
-        const SplitCounts c = split_counts(dp.len[i], dp.T, dp.pps, dp.pps_t, dp.lim[i]);
+        const SplitCounts c = split_counts(dp.len[i], dp.T, dp.pps[h], dp.pps_t, dp.lim[i]);
         const int S = c.qsplits + c.tsplits;
         std::vector<int>& v = seen[i * dp.Hkv + h];
         std::sort(v.begin(), v.end());
@@ -185,9 +189,10 @@ int main() {
 
 def test_cta_order_covers_every_split_once_longest_first(tmp_path):
     """The decode launch's 1-D grid (build_decode_order / decode_item) gives every
-    (entry, kv head, split) exactly one CTA, quantized splits in non-increasing page
-    count and then the tail splits, and exactly one zero-writing CTA per (entry, kv
-    head) with nothing to attend to, for random batches of lengths and split sizes."""
+    (entry, kv head, split) exactly one CTA -- full quantized splits first, then the
+    partial ones (no-op items only for heads without one), then the tail splits --
+    and exactly one zero-writing CTA per (entry, kv head) with nothing to attend to,
+    for random batches of lengths and per-head split sizes."""
     if not os.path.isdir(CUDA_INC):
         pytest.skip("CUDA headers not installed")
     src = tmp_path / "order.cpp"
