@@ -147,3 +147,19 @@ def test_prefill_rejects_more_queries_than_tokens():
     out = torch.empty((n + 1, w.n_q_heads, 128), dtype=torch.float32, device="cuda")
     with pytest.raises(kvq.KVQError):
         plan.prefill(0, 0, q, out, plan.new_workspace(256))
+
+
+def test_prefill_at_bench_scale_sampled():
+    """The bench's prefill call at scale: 2048 queries at the end of one long
+    KVarN q4_0 sequence (the batch workload's recipe, 256-token tail), every query
+    block of 32 positions on the tensor cores; sampled queries (the first and last
+    blocks' edges and a stride) against the oracle."""
+    w = W.make_workload(5, "full", ctx=[24576])
+    w.n_layers = 1
+    w.k_codec, w.v_codec = w.k_codec[:1], w.v_codec[:1]
+    plan = H.make_plan(w)
+    H.fill(plan, w, chunk=2048)
+    n_q = 2048
+    sample = sorted({0, 1, 31, 32, 1023, 1024, 2015, 2016, 2046, 2047} | set(range(5, n_q, 97)))
+    _, _, worst = _check(plan, w, 0, 0, n_q, sample)
+    assert worst <= H.TOL
