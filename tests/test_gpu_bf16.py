@@ -137,3 +137,39 @@ def test_bf16_plans_keep_raw_rows_in_the_tail_only():
         kvq.Plan(1, 8, 2, max_seqs=1, max_tokens_per_seq=128, k_codec=[kvq.F16, kvq.Q4_0],
                  v_codec=[kvq.Q4_0, kvq.Q4_0], rot=kvq.ROT_HADAMARD, kv_dtype=kvq.KV_BF16)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("path", [0, 1])
+def test_bf16_prefill_matches_oracle(path):
+    """Chunked prefill of a bf16 plan (bf16 queries, bf16 raw tail rows) on the
+    tensor-core path (0) and the decode-kernel path (1): sampled causal queries
+    against the oracle's bf16 encoding of the rows older than the tail."""
+    w = W.make_workload(5, "small")
+    plan = _plan(w)
+    _fill(plan, w, chunk=640)
+    plan.debug_set_prefill_path(path)
+    seq, layer = 1, 1
+    n = w.ctx[seq]
+    nq_all = n - w.tail
+    n_q = 150
+    q = torch.stack([w.queries(layer, seq, i, "cuda") for i in range(n_q)]).to(torch.bfloat16).contiguous()
+    out = torch.empty((n_q, w.n_q_heads, 128), dtype=torch.float32, device="cuda")
+    plan.prefill(layer, seq, q, out, plan.new_workspace(min(n_q, 256)))
+    torch.cuda.synchronize()
+    plan.check_device_error()
+    out = out.cpu().numpy()
+    K = _bits(_rows(w, "K", layer, seq, 0, n))
+    V = _bits(_rows(w, "V", layer, seq, 0, n))
+    for h in range(w.n_kv_heads):
+        args = H.head_params(w, layer, h)
+        ck, sk = oracle.encode_rows(args["k_codec"], w.rot, K[:nq_all, h, :], inv_s=args.get("inv_s_k"), bf16=True)
+        cv, sv = oracle.encode_rows(args["v_codec"], w.rot, V[:nq_all, h, :], inv_s=args.get("inv_s_v"), bf16=True)
+        for i in sorted({0, 31, 32, 63, 64, 85, 86, 117, 118, 149} | set(range(3, n_q, 11))):
+            lim = n - n_q + i + 1
+            nqv = min(lim, nq_all)
+            ref = oracle.decode_packed(ck[:nqv], sk[:nqv], cv[:nqv], sv[:nqv], K[nq_all:lim, h, :],
+                                       V[nq_all:lim, h, :], _bits(q[i, h * w.G:(h + 1) * w.G]), args["k_codec"],
+                                       args["v_codec"], w.rot, inv_s_k=args.get("inv_s_k"),
+                                       inv_s_v=args.get("inv_s_v"), bf16=True)
+            err = H.rel_err_rows(out[i, h * w.G:(h + 1) * w.G], ref)
+            assert err.max() <= H.TOL, (path, h, i, err.max())
