@@ -12,10 +12,11 @@
 //   P   = exp2(S - m) (online softmax, causal mask, one thread per row)
 //   O  += P V         [128 x 128]  (tcgen05, M = 128, N = 128, K = 64 tokens)
 //
-// Keys and values are dequantized once per CTA into fp16 operands in shared
+// Keys and values are dequantized once per CTA into fp16 operand images in shared
 // memory, in the stored (rotated) basis: y = d * (u - 2^(b-1)) for the _0
-// codecs, y = u * d + m for the _1 codecs, each one correctly rounded fp32
-// operation as in the reference dequantizer.  fp16 holds 11 significant bits,
+// codecs, y = u * d + m for the _1 codecs (the keys' hi part is one rounding of
+// the exact product, the lo part the exact remainder; the _1 keys go through the
+// reference dequantizer's fp32 value).  fp16 holds 11 significant bits,
 // so the keys are split y = y_hi + y_lo (both fp16) and the query
 // q' = R (s_k * q) * softmax_scale * log2(e) likewise, and S accumulates the
 // three products Qhi Khi + Qlo Khi + Qhi Klo (the fourth is below fp32's
@@ -28,17 +29,21 @@
 // transform before quantization, so one query image and one accumulator serve
 // every tile; the output is O_row / l taken back through R and s_v.
 //
-// Warp roles (320 threads, one CTA per SM: 211 KiB of shared memory at most):
-//   warps 0-3  softmax: thread = row = TMEM lane; query image, online softmax
-//              with a lazy rescale (O is rescaled only when the running max
-//              grows by more than 8 in log2 units), P to shared memory, and the
-//              epilogue;
-//   warps 4-7  dequantizers: quantized tiles from the raw ring, tail tiles
-//              straight from the ring in global memory, into the operand ring;
+// Warp roles (320 threads, one CTA per SM: 512 tensor-memory columns, at most
+// 227 KiB of shared memory -- three operand stages of 48 KiB and two to four raw
+// page-head stages):
+//   warps 0-3  softmax: thread = row = TMEM lane; the query image (into tensor
+//              memory), online softmax with a lazy rescale (O is rescaled only
+//              when the running max grows by more than 8 in log2 units), P over
+//              its tile's S columns, and the epilogue;
+//   warps 4-7  dequantizers (one instantiation per block codec): quantized tiles
+//              from the raw ring, tail tiles straight from the ring in global
+//              memory, into the operand stages (key half released when S
+//              completes, value half when P V does);
 //   warp 8     producer: one cp.async.bulk per 64-token page-head into the raw ring;
-//   warp 9     tensor memory allocation and, on one thread, the MMA issue: S of
-//              tile i is issued before P V of tile i-1, so the softmax of tile i
-//              overlaps the value product of the tile before.
+//   warp 9     tensor memory allocation and, on one thread, the MMA issue, which
+//              polls its barriers without suspending and issues whichever of S
+//              (next tile) and P V (oldest tile with P ready) can go.
 // The key and value images in shared memory use the canonical 128-byte-swizzled
 // layout: a 64-token x 128-channel tile is two 8 KiB halves (channels 0-63 and
 // 64-127); in a half, token t owns the 128-byte row t, and its 16-byte chunk j
