@@ -136,6 +136,14 @@ def decode_bytes(w, layer, lengths):
     return tot + len(lengths) * w.n_q_heads * 128 * (2 + 4)
 
 
+def decode_macs(w, layer, lengths):
+    """Multiply-adds of one decode launch: every visible (token, kv head) costs a score
+    and a value product of G query heads over the head's stored width (128, or the
+    rank r of a projected head)."""
+    width = sum((w.rank[layer][h] if w.rank is not None else 128) for h in range(w.n_kv_heads))
+    return sum(lengths) * 2 * w.G * width
+
+
 def append_bytes(w, layer, len_old, n):
     """Algorithmic bytes of appending n tokens to a sequence of len_old tokens in one
     layer: raw input rows read; rows leaving the tail read from the ring; quantized
@@ -510,6 +518,7 @@ def measure_workload(kvq, w, dev, K, Wm, world, log, headline):
     plan.check_device_error(stream)
     dec_bytes_all = [decode_bytes(w, l, lengths[l]) for l in range(L)]
     dec_bytes = statistics.mean(dec_bytes_all)
+    dec_macs = statistics.mean(decode_macs(w, l, lengths[l]) for l in range(L))
 
     res = {"workload": w.name, "ms_per_step": step_ms, "us_per_token": step_ms * 1e3 / B,
            "gpu_launches_per_step": launches_per_step, "l2": l2_note(w)}
@@ -570,7 +579,7 @@ def measure_workload(kvq, w, dev, K, Wm, world, log, headline):
                               "bytes_per_launch": app_b / L, "launch_ms": app_ms / L,
                               "achieved": app_b / (app_ms / 1e3) / 1e9, "unit": "GB/s",
                               "note": "raw rows read (input and ring) + packed rows and ring rows written"}
-    res["decode"] = {"bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
+    res["decode"] = {"bytes_per_launch": dec_bytes, "macs_per_launch": dec_macs, "launch_ms": dec_ms,
                      "achieved": dec_bytes / (dec_ms / 1e3) / 1e9, "kernel": f"decode_kernel<{w.G}>",
                      "traffic": traffic_from_profile(w.name)}
     del ck, cv, ga
@@ -639,6 +648,22 @@ def measure_workload(kvq, w, dev, K, Wm, world, log, headline):
     return res
 
 
+# The decode loops' multiply-adds run as dp2a (two per lane per instruction) on the
+# fmaheavy pipe: 148 SMs x 4 schedulers x 16 lanes x 2 multiply-adds x 1.965 GHz.
+DP2A_PEAK_TMACS = 148 * 4 * 16 * 2 * 1.965e9 / 1e12
+
+
+def alu_roofline(d):
+    """The decode launch against its multiply-add ceiling (the dp2a pipe); the HBM
+    roofline above is the metric the workloads name, this one the kernel's own bound
+    where its multiply-add floor lies above its HBM floor."""
+    achieved = d["macs_per_launch"] / (d["launch_ms"] / 1e3) / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": DP2A_PEAK_TMACS, "unit": "Tmul-add/s",
+            "frac": achieved / DP2A_PEAK_TMACS, "kernel": d.get("kernel"), "macs_per_launch": d["macs_per_launch"],
+            "peak_source": "unit counts x clock (dp2a on the fmaheavy pipe); tests/test_gpu_ubench.py measures "
+                           "about 36 T/s"}
+
+
 def roofline(d, peak, peaks):
     return {"bound": "hbm", "achieved": d["achieved"], "peak": peak, "unit": "GB/s", "frac": d["achieved"] / peak,
             "traffic": d.get("traffic"), "kernel": d.get("kernel"), "bytes_per_launch": d["bytes_per_launch"],
@@ -681,6 +706,7 @@ def run_kvq(args, world, rank, local):
         "regrade": h.get("regrade"),
         "prefill": h.get("prefill"),
         "roofline": roofline(h["decode"], peak, peaks),
+        "alu_roofline": alu_roofline(h["decode"]),
         "e2e": h["e2e"],
         "gpu_launches": h["gpu_launches_per_step"] * K,
         "clocks": h["clocks"],

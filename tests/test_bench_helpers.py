@@ -55,3 +55,15 @@ def test_kernel_source_hash_covers_the_decode_sources():
     assert len(h) == 64
     for name in bench.DECODE_SOURCES:
         assert os.path.exists(os.path.join(ROOT, "quantized_kv_cache_15_b200", "csrc", name))
+
+
+def test_decode_multiply_adds():
+    """A decode launch's multiply-adds: per visible (token, kv head), G query heads x
+    (score + value) x the head's stored width (128, or the rank of a projected head)."""
+    import bench
+    from quantized_kv_cache_15_b200 import workloads as W
+    w = W.make_workload(1, "full")                                   # 1024 tokens, 2 kv heads, G = 4
+    assert bench.decode_macs(w, 0, w.ctx) == 1024 * 4 * 2 * (2 * 128)
+    w4 = W.make_workload(4, "full")
+    assert bench.decode_macs(w4, 3, [100]) == 100 * w4.G * 2 * sum(w4.rank[3])
+    assert 36.0 < bench.DP2A_PEAK_TMACS < 38.0
