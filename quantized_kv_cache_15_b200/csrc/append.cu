@@ -87,11 +87,15 @@ __device__ __forceinline__ uint8_t* ring_chunk(uint8_t* ring, int slot, int kv, 
   return kv == 0 ? tp + (c * TAIL_TOK + row) * 16 : tp + TAIL_TOK * D * 2 + row * (D * 2) + 16 * c;
 }
 
-// Destination page row of a quantized position; false (and the error bit) when
-// the block table has no page there.
-__device__ __forceinline__ bool page_row(const AppendParams& p, const RowWork& w, uint8_t** codes, uint8_t** scales,
-                                         bool report) {
-  const int pid = p.block_table[(size_t)w.sq->seq * p.max_pages_per_seq + w.pos / PAGE];
+// Destination page of a quantized position (the block-table entry; read before
+// the row itself so that the two global loads are in flight together) and the
+// page row's code and scale planes; false (and the error bit) when the block
+// table has no page there.
+__device__ __forceinline__ int page_of(const AppendParams& p, const RowWork& w) {
+  return p.block_table[(size_t)w.sq->seq * p.max_pages_per_seq + w.pos / PAGE];
+}
+__device__ __forceinline__ bool page_row(const AppendParams& p, const RowWork& w, int pid, uint8_t** codes,
+                                         uint8_t** scales, bool report) {
   if (pid < 0) {
     if (report) atomicOr(p.err, ERR_NO_PAGE);
     return false;
@@ -120,6 +124,7 @@ __global__ void __launch_bounds__(256) append_warp_kernel(const __grid_constant_
   const __half* in = kv ? p.v_in : p.k_in;
   if (w.pos >= 0) {
     const int codec = kv ? h.vcodec : h.kcodec;
+    const int pid = page_of(p, w);
     float x[4];
     if (w.ring_slot >= 0) {
       const uint2 r = *reinterpret_cast<const uint2*>(ring_chunk(w.ring, w.ring_slot, kv, lane >> 1) + 8 * (lane & 1));
@@ -130,7 +135,7 @@ __global__ void __launch_bounds__(256) append_warp_kernel(const __grid_constant_
     }
     transform_row(x, codec, p.rot, p.inv_s ? p.inv_s + ((size_t)w.head * 2 + kv) * D : nullptr);
     uint8_t *codes, *scales;
-    if (!page_row(p, w, &codes, &scales, lane == 0)) return;
+    if (!page_row(p, w, pid, &codes, &scales, lane == 0)) return;
     quantize_store_row(x, codec, h.r, kv ? h.vbits : h.kbits, codes, scales, w.pos % PAGE, kv == 0, p.bf16);
   }
   if (w.write_slot >= 0) {
@@ -155,16 +160,18 @@ __global__ void __launch_bounds__(256) append_quad_kernel(const __grid_constant_
   const __half* in = kv ? p.v_in : p.k_in;
   if (w.pos >= 0) {
     const int codec = kv ? h.vcodec : h.kcodec;
+    const int pid = page_of(p, w);
+    uint4 r[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      r[c] = w.ring_slot >= 0
+                 ? *reinterpret_cast<const uint4*>(ring_chunk(w.ring, w.ring_slot, kv, 4 * q + c))
+                 : *reinterpret_cast<const uint4*>(in + ((size_t)w.src_row * p.Hkv + w.head) * D + 32 * q + 8 * c);
+    uint8_t *codes, *scales;
+    if (!page_row(p, w, pid, &codes, &scales, q == 0)) return;
     float v[32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 r = w.ring_slot >= 0
-                          ? *reinterpret_cast<const uint4*>(ring_chunk(w.ring, w.ring_slot, kv, 4 * q + c))
-                          : *reinterpret_cast<const uint4*>(in + ((size_t)w.src_row * p.Hkv + w.head) * D + 32 * q + 8 * c);
-      chunk_to_float(r, v + 8 * c, p.bf16);
-    }
-    uint8_t *codes, *scales;
-    if (!page_row(p, w, &codes, &scales, q == 0)) return;
+    for (int c = 0; c < 4; ++c) chunk_to_float(r[c], v + 8 * c, p.bf16);
     if (codec != KVQ_F16)
       transform_row_quad(v, p.rot, p.inv_s ? p.inv_s + ((size_t)w.head * 2 + kv) * D : nullptr);
     quantize_row_quad(codec, v, codes, scales, w.pos % PAGE, kv == 0, kv ? h.cbV : h.cbK, kv ? h.sbV : h.sbK, p.bf16);
