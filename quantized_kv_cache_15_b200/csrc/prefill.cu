@@ -789,12 +789,10 @@ int prefill_raw_stages(int stage_bytes) {
 
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t s) {
   if (p.n_q <= 0) return cudaSuccess;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_MAX);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // the shared-memory opt-in is a property of the kernel on the current device:
+  // set it on every launch (a host call; the plan may live on any device)
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_MAX);
+  if (e != cudaSuccess) return e;
   const int n_blocks = (p.n_q + p.QB - 1) / p.QB;
   dim3 grid(n_blocks, p.Hkv);
   prefill_kernel<<<grid, PF_THREADS, prefill_smem_bytes(p.stage_bytes, p.n_raw), s>>>(p);

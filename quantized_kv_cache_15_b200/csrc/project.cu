@@ -175,12 +175,10 @@ __global__ void __launch_bounds__(PJ_THREADS, 1) proj_kernel(const __grid_consta
 cudaError_t launch_project(const ProjParams& p, int n_items, int n_heads, cudaStream_t s) {
   if (n_items <= 0) return cudaSuccess;
   const size_t smem = proj_smem_bytes(128);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // the shared-memory opt-in is a property of the kernel on the current device:
+  // set it on every launch (a host call; the plan may live on any device)
+  cudaError_t e = cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   const int n_tiles = (n_items + PJ_ROWS - 1) / PJ_ROWS;
   dim3 grid(n_tiles, p.z_out ? 1 : n_heads, p.z_out ? 1 : 2);
   proj_kernel<<<grid, PJ_THREADS, smem, s>>>(p);
