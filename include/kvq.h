@@ -31,6 +31,10 @@
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *    enqueued asynchronously on it; argument errors are reported synchronously,
  *    before anything is enqueued, and leave the plan unchanged.
+ *  - A call that enqueues work on a plan (append, decode, prefill, dequantize,
+ *    row reads, regrade, the debug transforms) needs the plan's device (the one
+ *    current at kvq_plan_create) to be current: otherwise it returns
+ *    KVQ_ERR_STATE and enqueues nothing.
  *  - Errors never throw across the ABI.  Every call returns a kvq_status;
  *    kvq_last_error() gives a thread-local message for the last failure.
  *    Conditions that only a kernel can see (a missing page, an exhausted wait)

@@ -119,6 +119,18 @@ struct kvq_plan {
   }
 };
 
+// Kernels are launched on the current device and read the plan's memory, so a call
+// that enqueues work needs the plan's device current: on another device (through
+// the legacy stream, say) they would reach that memory only by peer access, which
+// this library never enables.  Checked before anything is enqueued.
+static kvq_status require_plan_device(const kvq_plan* p) {
+  int dev = -1;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != p->device) return fail(KVQ_ERR_STATE, "current device %d is not the plan's device %d", dev, p->device);
+  return KVQ_OK;
+}
+
 extern "C" {
 
 const char* kvq_last_error(void) { return g_err.c_str(); }
@@ -354,6 +366,7 @@ kvq_status kvq_cache_bind(kvq_plan* p, void* dev, size_t bytes) {
 kvq_status kvq_append_quantize(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* n_new,
                                const void* k_new, const void* v_new, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   if (n_seqs < 0 || n_seqs > MAX_BATCH) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [0, %d]", MAX_BATCH);
@@ -654,6 +667,8 @@ static kvq_status decode_enqueue(const DecodeLaunch& L, void* stream) {
 static kvq_status decode_launch(kvq_plan* p, int layer, int n_seqs, const int* seq_ids, const int* lims,
                                 const void* q, float* out, void* workspace, size_t workspace_bytes_given,
                                 void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   DecodeLaunch L;
   const kvq_status st = decode_prepare(p, layer, n_seqs, seq_ids, lims, q, out, workspace, workspace_bytes_given, L);
   if (st != KVQ_OK) return st;
@@ -692,6 +707,7 @@ static bool prefill_tc_layout(const kvq_plan* p, int layer, int* stage_bytes, in
 kvq_status kvq_prefill_attention(kvq_plan* p, int layer, int seq_id, int n_q, const void* q, float* out,
                                  void* workspace, size_t workspace_bytes_given, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d out of range", seq_id);
@@ -781,6 +797,7 @@ kvq_status kvq_decode_attention_noalloc(kvq_plan* p, int layer, int n_seqs, cons
 kvq_status kvq_dequantize(const kvq_plan* p, int layer, int seq_id, int64_t t0, int64_t t1, float* k_out,
                           float* v_out, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id out of range");
@@ -808,6 +825,7 @@ kvq_status kvq_row_bytes(const kvq_plan* p, int layer, int head, int kv, int* cb
 kvq_status kvq_read_rows(const kvq_plan* p, int layer, int seq_id, int64_t t0, int64_t t1, int kv, void* codes,
                          void* scales, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "null plan");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L || (kv != 0 && kv != 1)) return fail(KVQ_ERR_INVALID_ARG, "layer or kv out of range");
   if (seq_id < 0 || seq_id >= p->max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id out of range");
@@ -878,6 +896,7 @@ kvq_status kvq_plan_regrade_bytes(const kvq_plan* p, int layer, const int* k_cod
 kvq_status kvq_regrade_layer(kvq_plan* p, int layer, const int* k_codec, const int* v_codec, void* scratch,
                              size_t scratch_bytes, void* stream) {
   if (!p || !k_codec || !v_codec) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   if (!p->cache) return fail(KVQ_ERR_STATE, "no cache bound");
   if (layer < 0 || layer >= p->L) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   std::vector<HeadInfo> heads;
@@ -1027,6 +1046,7 @@ kvq_status kvq_debug_fault_injection(kvq_plan* p, int64_t wait_limit_ns, int dro
 kvq_status kvq_debug_rotate(const kvq_plan* p, int layer, int head, int kv, int n, const void* x, float* y,
                             int layout, void* stream) {
   if (!p || !x || !y) return fail(KVQ_ERR_INVALID_ARG, "null argument");
+  if (const kvq_status st = require_plan_device(p); st != KVQ_OK) return st;
   if (layout != KVQ_ROWS_WARP && layout != KVQ_ROWS_QUAD) return fail(KVQ_ERR_INVALID_ARG, "bad row layout");
   if (layer < 0 || layer >= p->L || head < 0 || head >= p->Hkv || (kv != 0 && kv != 1) || n < 0)
     return fail(KVQ_ERR_INVALID_ARG, "argument out of range");
