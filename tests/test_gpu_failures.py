@@ -10,7 +10,6 @@
 import ctypes
 import os
 
-import numpy as np
 import pytest
 import torch
 

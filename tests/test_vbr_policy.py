@@ -2,7 +2,6 @@
 Rate)": quantize layer by layer as the session grows, within --vbr-vram, above
 --vbr-floor).  Ladder F16 > q8_0 > q6_0 > q4_1 > q2_1, V on a rung and K one rung
 richer, the deepest layer on the richest rung moves first."""
-import numpy as np
 import pytest
 
 from quantized_kv_cache_15_b200 import kvq
