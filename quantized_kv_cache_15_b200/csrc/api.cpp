@@ -545,7 +545,7 @@ static kvq_status decode_prepare(const kvq_plan* p, int layer, int n_seqs, const
   const int want_ctas = DECODE_MIN_CTAS(p->G);
   dp.n_stages = NCW;
   for (int ns = 8; ns > NCW; --ns)
-    if (decode_smem_bytes(dp.stage_bytes, ns, p->G, dp.wtab_smem) + 1024 <= (228 * 1024) / want_ctas) {
+    if (decode_smem_bytes(dp.stage_bytes, ns, p->G, dp.wtab_smem) + 1024 <= (size_t)((228 * 1024) / want_ctas)) {
       dp.n_stages = ns;
       break;
     }
