@@ -351,13 +351,16 @@ void orc_unpack_codes(const uint8_t* in, int n, int bits, uint8_t* u) {
         case 1: unpack_field(in, n, 1, u); break;
         case 6:
             unpack_field(in, n, 4, lo); unpack_field(in + n / 2, n, 2, hi);
-            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 4)); break;
+            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 4));
+            break;
         case 5:
             unpack_field(in, n, 4, lo); unpack_field(in + n / 2, n, 1, hi);
-            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 4)); break;
+            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 4));
+            break;
         case 3:
             unpack_field(in, n, 2, lo); unpack_field(in + n / 4, n, 1, hi);
-            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 2)); break;
+            for (int j = 0; j < n; ++j) u[j] = (uint8_t)(lo[j] | (hi[j] << 2));
+            break;
         default: break;
     }
 }
