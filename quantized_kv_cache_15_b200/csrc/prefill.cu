@@ -101,16 +101,10 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
 __device__ __forceinline__ uint32_t umma_idesc(int n, bool b_mn_major) {
   return (1u << 4) | (b_mn_major ? (1u << 16) : 0u) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(PF_ROWS >> 4) << 24);
 }
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// The same with A read from tensor memory (M rows in lanes, K along columns, two
-// 16-bit elements per 32-bit column, the lower-indexed in the low half).
+// D (tensor memory) = A B (+ D when `accumulate` is nonzero), kind::f16, with A
+// read from tensor memory (M rows in lanes, K along columns, two 16-bit elements
+// per 32-bit column, the lower-indexed in the low half) and B from shared memory
+// through its descriptor.
 __device__ __forceinline__ void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
                                                 uint32_t accumulate) {
   asm volatile(
